@@ -1,0 +1,309 @@
+/*
+ * CPU oracle for Stem block-sparse causal prefill.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load or call this library. The product path (the CUDA
+ * library) never links, loads or calls it, and it shares no code with it.
+ *
+ * It restates, in plain double-precision loops, what the method computes, as
+ * described for "Stem: Rethinking Causal Information Flow in Sparse Attention"
+ * (arXiv 2603.06274). Page tags used below, all titled with that name:
+ *   [es] gist.science/es, "Resumen tecnico"        (sections 1-5)
+ *   [it] gist.science/it, "Sommario tecnico"       (sections 1-5)
+ *   [nl] gist.science/nl, "Technische samenvatting" (Methodologie, Implementatie)
+ *   [fr] gist.science/fr, "Resume technique"        (sections 1-5)
+ *   [zh] shd-paper.top index page, English abstract and "key design" paragraph
+ *
+ * The pages describe three stages (block downsampling; a position-dependent
+ * budget; top-k by the output-aware metric and exact attention over the kept
+ * blocks): [es] section 2 "Implementacion", [it] section 2.C, [nl]
+ * "Implementatie", [fr] section 2.C. Where the pages leave a step open, the
+ * parameterised reading used here is:
+ *   budget   k(i) = min(i+1, max(k_min, ceil(rho(i)*(i+1)))),
+ *            rho(i) = rho_min + (1-rho_min)*exp(-i/tau), i = query-block index;
+ *            for i >= 1 at least 2 blocks (sink and diagonal); k(0) = 1;
+ *   pooling  arithmetic mean of Q rows and of K rows per block; mean of the
+ *            per-row L2 norms of V per block;
+ *   metric   m_ij = softmax_{j<=i}(qbar_i . kbar_j / sqrt(D)) * n_j;
+ *   keep     block 0, block i, and the k(i)-2 best other blocks j in [1, i-1]
+ *            by (m descending, j ascending);
+ *   attend   exact softmax attention of each query token over all tokens of
+ *            the kept blocks, token-causal inside the diagonal block.
+ *
+ * Layouts: Q [B,Hq,S,D], K and V [B,Hkv,S,D], contiguous. Query head h reads
+ * key/value head h / (Hq/Hkv). dtype 0 = bfloat16 (raw 16-bit patterns),
+ * dtype 1 = float32. Every value is widened to double before any arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int stem_oracle_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* Exact widening of one stored element to double. */
+static double elem(const void* base, int dtype, int64_t idx) {
+  if (dtype == 1) return (double)((const float*)base)[idx];
+  uint32_t bits = (uint32_t)((const uint16_t*)base)[idx] << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+/*
+ * Token Position-Decay budget ([es] 2.A, [it] 2.A, [nl] TPD, [fr] 2.A: a budget
+ * that is large for early query positions and shrinks with position; [zh] key
+ * design: the decay is usually exponential). The exponential-ratio form above
+ * is the reading used. Returns sum_i k(i); writes k[nb] and the prefix sums
+ * off[nb+1] (off[0] = 0).
+ */
+int64_t stem_oracle_budget(int nb, double rho_min, double tau, int k_min,
+                           int32_t* k_out, int64_t* off_out) {
+  int64_t total = 0;
+  for (int i = 0; i < nb; ++i) {
+    double rho = rho_min + (1.0 - rho_min) * exp(-(double)i / tau);
+    double want = ceil(rho * (double)(i + 1));
+    double kk = want > (double)k_min ? want : (double)k_min;
+    if (kk > (double)(i + 1)) kk = (double)(i + 1);
+    int k = (int)kk;
+    if (i == 0) {
+      k = 1; /* only the block itself exists */
+    } else if (k < 2) {
+      k = 2; /* the sink and the diagonal are always kept */
+    }
+    if (off_out) off_out[i] = total;
+    if (k_out) k_out[i] = k;
+    total += k;
+  }
+  if (off_out) off_out[nb] = total;
+  return total;
+}
+
+/*
+ * Block downsampling ([es] 2 "Implementacion" step 1: block-level Q, K and V
+ * magnitude; [it] 2.C step 1; [nl] Implementatie step 1; [fr] 2.C step 1).
+ * qbar [B,Hq,nb,D], kbar [B,Hkv,nb,D]: mean over the block's rows.
+ * vnorm [B,Hkv,nb]: mean over the block's rows of the row's Euclidean norm.
+ */
+void stem_oracle_pool(const void* q, const void* k, const void* v, int dtype, int B,
+                      int Hq, int Hkv, int S, int D, int block, double* qbar,
+                      double* kbar, double* vnorm) {
+  const int nb = S / block;
+  const int64_t nq = (int64_t)B * Hq * nb;
+  const int64_t nk = (int64_t)B * Hkv * nb;
+#pragma omp parallel for schedule(static)
+  for (int64_t u = 0; u < nq; ++u) {
+    const int64_t bh = u / nb, i = u % nb;
+    const int64_t row0 = bh * S + i * block;
+    for (int d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int r = 0; r < block; ++r) acc += elem(q, dtype, (row0 + r) * D + d);
+      qbar[u * D + d] = acc / block;
+    }
+  }
+#pragma omp parallel for schedule(static)
+  for (int64_t u = 0; u < nk; ++u) {
+    const int64_t bh = u / nb, i = u % nb;
+    const int64_t row0 = bh * S + i * block;
+    for (int d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int r = 0; r < block; ++r) acc += elem(k, dtype, (row0 + r) * D + d);
+      kbar[u * D + d] = acc / block;
+    }
+    double nacc = 0.0;
+    for (int r = 0; r < block; ++r) {
+      double sq = 0.0;
+      for (int d = 0; d < D; ++d) {
+        double x = elem(v, dtype, (row0 + r) * D + d);
+        sq += x * x;
+      }
+      nacc += sqrt(sq);
+    }
+    vnorm[u] = nacc / block;
+  }
+}
+
+/*
+ * Output-Aware Metric on pooled blocks ([es] 2.B, [it] 2.B, [nl] OAM, [fr] 2.B:
+ * routing relevance combined with value magnitude, since a block whose values
+ * are near zero contributes little to the output; [zh] English abstract:
+ * prioritises blocks by approximate output magnitude). Reading used: the
+ * pooled attention probability times the pooled value norm,
+ *   s_ij = qbar_i . kbar_j / sqrt(D),  p_ij = exp(s_ij - max_j s) / sum_j exp(...),
+ *   m_ij = p_ij * n_j,   for j = 0..i.
+ * Output packed by row: m[(b*Hq+h)*T + i*(i+1)/2 + j], T = nb*(nb+1)/2.
+ */
+void stem_oracle_metric(const double* qbar, const double* kbar, const double* vnorm,
+                        int B, int Hq, int Hkv, int nb, int D, double* m) {
+  const int G = Hq / Hkv;
+  const int64_t T = (int64_t)nb * (nb + 1) / 2;
+  const double scale = 1.0 / sqrt((double)D);
+  const int64_t rows = (int64_t)B * Hq * nb;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t u = 0; u < rows; ++u) {
+    const int64_t bh = u / nb;
+    const int i = (int)(u % nb);
+    const int64_t b = bh / Hq, h = bh % Hq;
+    const int64_t bg = b * Hkv + h / G;
+    const double* qi = qbar + u * D;
+    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;
+    double mx = -INFINITY;
+    for (int j = 0; j <= i; ++j) {
+      const double* kj = kbar + (bg * nb + j) * D;
+      double dot = 0.0;
+      for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+      mrow[j] = dot * scale; /* s_ij, kept here until normalised */
+      if (mrow[j] > mx) mx = mrow[j];
+    }
+    double z = 0.0;
+    for (int j = 0; j <= i; ++j) z += exp(mrow[j] - mx);
+    for (int j = 0; j <= i; ++j) {
+      double p = exp(mrow[j] - mx) / z;
+      mrow[j] = p * vnorm[bg * nb + j];
+    }
+  }
+}
+
+typedef struct {
+  double m;
+  int j;
+} cand_t;
+
+/* Larger metric first; equal metrics: lower block index first. */
+static int cand_cmp(const void* pa, const void* pb) {
+  const cand_t* a = (const cand_t*)pa;
+  const cand_t* b = (const cand_t*)pb;
+  if (a->m > b->m) return -1;
+  if (a->m < b->m) return 1;
+  return (a->j > b->j) - (a->j < b->j);
+}
+
+static int int_cmp(const void* pa, const void* pb) {
+  int a = *(const int*)pa, b = *(const int*)pb;
+  return (a > b) - (a < b);
+}
+
+/*
+ * Top-k block selection with the position-dependent budget ([es] 2
+ * "Implementacion" steps 2-3; [it] 2.C step 2; [nl] Implementatie steps 2-3;
+ * [fr] 2.C steps 2-3), keeping the initial block that every later token depends
+ * on ([es] 1 and 2.A; [fr] 2.A; [zh] abstract: initial tokens are retained)
+ * and the query block itself. Rows are written in ascending block order:
+ *   sel_idx[(b*Hq+h)*cap + off[i] + t], t < k[i];  sel_cnt[(b*Hq+h)*nb + i] = k[i].
+ */
+void stem_oracle_select(const double* m, const int32_t* k, const int64_t* off, int B,
+                        int Hq, int nb, int64_t cap, int32_t* sel_idx, int32_t* sel_cnt) {
+  const int64_t T = (int64_t)nb * (nb + 1) / 2;
+  const int64_t rows = (int64_t)B * Hq * nb;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t u = 0; u < rows; ++u) {
+    const int64_t bh = u / nb;
+    const int i = (int)(u % nb);
+    const double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;
+    int32_t* dst = sel_idx + bh * cap + off[i];
+    const int ki = k[i];
+    sel_cnt[u] = ki;
+    if (i == 0) {
+      dst[0] = 0;
+      continue;
+    }
+    int* chosen = (int*)malloc(sizeof(int) * (size_t)ki);
+    int n = 0;
+    chosen[n++] = 0;
+    chosen[n++] = i;
+    const int ncand = i - 1; /* blocks 1 .. i-1 */
+    if (ncand > 0 && ki > 2) {
+      cand_t* c = (cand_t*)malloc(sizeof(cand_t) * (size_t)ncand);
+      for (int j = 1; j < i; ++j) {
+        c[j - 1].m = mrow[j];
+        c[j - 1].j = j;
+      }
+      qsort(c, (size_t)ncand, sizeof(cand_t), cand_cmp);
+      for (int t = 0; t < ki - 2; ++t) chosen[n++] = c[t].j;
+      free(c);
+    }
+    qsort(chosen, (size_t)n, sizeof(int), int_cmp);
+    for (int t = 0; t < n; ++t) dst[t] = chosen[t];
+    free(chosen);
+  }
+}
+
+/*
+ * Exact attention over the kept blocks ([es] 2 "Implementacion" step 3: exact
+ * softmax and aggregation only over the selected blocks; [it] 2.C step 3;
+ * [nl] Implementatie step 3; [fr] 2.C step 3). For query token r of block i:
+ * keys are every token of every kept block j < i, plus tokens i*block .. r of
+ * the diagonal block; logits Q[r].K[c] / sqrt(D); output sum_c softmax_c * V[c].
+ *
+ * Computes the listed query blocks only: rows[t] = (b*Hq + h)*nb + i.
+ * out_rows [nrows, block, D] (double).
+ */
+void stem_oracle_attention(const void* q, const void* k, const void* v, int dtype, int B,
+                           int Hq, int Hkv, int S, int D, int block,
+                           const int32_t* sel_idx, const int32_t* sel_cnt,
+                           const int64_t* off, int64_t cap, const int64_t* rows,
+                           int64_t nrows, double* out_rows) {
+  const int nb = S / block;
+  const int G = Hq / Hkv;
+  const double scale = 1.0 / sqrt((double)D);
+  (void)B;
+#pragma omp parallel
+  {
+    /* per-thread scratch: logits for every key a query token may see */
+    double* logit = (double*)malloc(sizeof(double) * (size_t)S);
+    double* qrow = (double*)malloc(sizeof(double) * (size_t)D);
+    int64_t* keyrow = (int64_t*)malloc(sizeof(int64_t) * (size_t)S);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nrows; ++t) {
+      const int64_t u = rows[t];
+      const int64_t bh = u / nb;
+      const int i = (int)(u % nb);
+      const int64_t b = bh / Hq, h = bh % Hq;
+      const int64_t kvbase = (b * Hkv + h / G) * (int64_t)S; /* row index of token 0 */
+      const int32_t* list = sel_idx + bh * cap + off[i];
+      const int cnt = sel_cnt[u];
+      for (int r = 0; r < block; ++r) {
+        const int64_t qtok = (int64_t)i * block + r;
+        for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, (bh * S + qtok) * D + d);
+        int nkeys = 0;
+        double mx = -INFINITY;
+        for (int e = 0; e < cnt; ++e) {
+          const int j = list[e];
+          const int last = (j == i) ? r : block - 1; /* token-causal on the diagonal */
+          for (int c = 0; c <= last; ++c) {
+            const int64_t krow = kvbase + (int64_t)j * block + c;
+            double dot = 0.0;
+            for (int d = 0; d < D; ++d) dot += qrow[d] * elem(k, dtype, krow * D + d);
+            logit[nkeys] = dot * scale;
+            keyrow[nkeys] = krow;
+            if (logit[nkeys] > mx) mx = logit[nkeys];
+            ++nkeys;
+          }
+        }
+        double z = 0.0;
+        for (int c = 0; c < nkeys; ++c) {
+          logit[c] = exp(logit[c] - mx);
+          z += logit[c];
+        }
+        double* o = out_rows + (t * block + r) * (int64_t)D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (int c = 0; c < nkeys; ++c) {
+          const double w = logit[c] / z;
+          for (int d = 0; d < D; ++d) o[d] += w * elem(v, dtype, keyrow[c] * D + d);
+        }
+      }
+    }
+    free(logit);
+    free(qrow);
+    free(keyrow);
+  }
+}
