@@ -1,0 +1,373 @@
+"""Benchmark of Stem block-sparse causal prefill on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the whole hot path (block pooling, budget, metric + top-k selection,
+block-sparse attention) over one batch of synthetic input, through the library's C ABI
+(stem_prefill_ex). Default workload: the Llama-3-8B-shaped layer at S = 131072 (B 1, Hq 32,
+Hkv 8, D 128, block 128, rho_min 0.05, tau 64, k_min 8), bf16.
+
+Metric: effective TFLOP/s = 4*block^2*D FLOP per kept (b, q-head, query block, key block) pair
+divided by the step time (whole job: summed over ranks); the step latency is ms_per_step.
+Timing: CUDA events on the launching stream, W >= 3 warm-up steps, barrier + synchronize on
+both sides of exactly K timed steps, max over ranks. Inputs (1.61 GB) are larger than the
+126 MB L2, so no flush runs between steps. Per-stage durations come from four events the
+library records around its kernels inside the timed steps.
+
+N > 1 (torchrun): each rank runs its own independent problem (seed + rank) on its own GPU; no
+data-path collective (the path partitions by (batch, kv-head group)); weak scaling.
+
+--impl reference: the CPU oracle (oracle/), as it stands, on this host's cores, on a bounded
+sample of the same workload per step (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_causal_pooling_b200 import workloads as wl  # noqa: E402
+
+METRIC = "Stem prefill attention latency (ms) & effective TFLOP/s at S=128K, % of BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        # nvidia-smi numbers GPUs physically; select ours by UUID
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:  # noqa: BLE001
+            self.gpu = str(device.index or 0)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags)
+                          if f.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle (reference arm)
+
+
+def oracle_sample_step(w, q, k, v, rows):
+    """The oracle as it stands on one kv-head group: pooling, metric, selection for every query
+    block of the group's heads, then exact attention for the listed rows. Returns (effective
+    FLOP of the listed rows, seconds for attention + selection prorated to those rows)."""
+    import oracle
+
+    G = w.Hq // w.Hkv
+    qs, ks, vs = q[:, :G].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous()
+    t0 = time.perf_counter()
+    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+    qb, kb, vn = oracle.pool(qs, ks, vs, w.block)
+    m = oracle.metric(qb, kb, vn)
+    si, sc = oracle.select(m, kk, off)
+    t1 = time.perf_counter()
+    oracle.attention(qs, ks, vs, w.block, si, sc, off, rows)
+    t2 = time.perf_counter()
+    flop = sum(wl.effective_flops(int(kk[i]), w.block, w.D) for (_, _, i) in rows)
+    share = len(rows) / float(G * w.nb)
+    return flop, (t2 - t1) + (t1 - t0) * share, dict(select_s=t1 - t0, attn_s=t2 - t1)
+
+
+def cpu_inputs(w, seed_offset=0):
+    wr = w.replace(seed=w.seed + seed_offset, Hq=w.Hq // w.Hkv, Hkv=1)
+    return wl.make_inputs(wr, "cpu")
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+
+    w = wl.WORKLOADS[args.workload]
+    q, k, v = cpu_inputs(w)
+    G = w.Hq // w.Hkv
+    import random
+
+    rng = random.Random(7)
+    n_rows = max(4, oracle.threads())  # the oracle parallelises over query blocks
+    samples = []
+    for step in range(args.warmup + args.steps):
+        rows = [(0, rng.randrange(G), rng.randrange(w.nb)) for _ in range(n_rows)]
+        flop, sec, _ = oracle_sample_step(w, q, k, v, rows)
+        if step >= args.warmup:
+            samples.append((flop, sec))
+    flop = sum(f for f, _ in samples)
+    sec = sum(s for _, s in samples)
+    value = flop / sec / 1e12
+    sample = (f"per step: pooling + metric + selection of one kv-head group ({G} q-heads x "
+              f"{w.nb} query blocks, time prorated to the sampled rows) + exact attention of "
+              f"{n_rows} random query blocks (seed 7)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sec / len(samples), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU path
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
+            "block": w.block, "rho_min": w.rho_min, "tau": w.tau, "k_min": w.k_min,
+            "input_dtype": w.dtype, "l2": "inputs (Q+K+V) larger than L2; no flush"}
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_causal_pooling_b200 import stem as S
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.workload]
+    wr = w.replace(seed=w.seed + rank)
+    q, k, v = wl.make_inputs(wr, dev)
+    out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min)
+    ws = S.alloc_workspace(q, k, w.block)
+    kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
+    pairs = w.B * w.Hq * int(kk.sum())
+    flop = wl.effective_flops(pairs, w.block, w.D)
+    stream = torch.cuda.current_stream(dev)
+
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    args_warm = S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
+                            ws)
+    call_args = [S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
+                             ws, events=ev[s]) for s in range(K)]
+    lib = S.lib()
+    hstream = S.ctypes.c_void_p(stream.cuda_stream)
+
+    def step(a):
+        rc = lib.stem_prefill_ex(S.ctypes.byref(a), hstream)
+        if rc != 0:
+            raise S.StemError(rc, "stem_prefill_ex")
+
+    for _ in range(W):
+        step(args_warm)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clocks:
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for s in range(K):
+            step(call_args[s])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(stop)
+    stage_ms = {"pool": [], "select": [], "attn": []}
+    for s in range(K):
+        e = ev[s]
+        stage_ms["pool"].append(e[0].elapsed_time(e[1]))
+        stage_ms["select"].append(e[1].elapsed_time(e[2]))
+        stage_ms["attn"].append(e[2].elapsed_time(e[3]))
+    ms = total_ms / K
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    clk = clocks.summary()
+
+    # end to end through the host-buffer entry point: pinned inputs in, output + CSR back
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        hsi = torch.empty(sel_idx.shape, dtype=torch.int32).pin_memory()
+        hsc = torch.empty(sel_cnt.shape, dtype=torch.int32).pin_memory()
+        S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc)
+        if world > 1:
+            torch.distributed.barrier()
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc)
+        e2e_s = (time.perf_counter() - t0) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_s = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = sum(t.numel() * t.element_size() for t in (hout, hsi, hsc))
+        e2e = {"value": world * flop / e2e_s / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": 1e3 * e2e_s}
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    attn_ms = statistics.mean(stage_ms["attn"])
+    pool_ms = statistics.mean(stage_ms["pool"])
+    sel_ms = statistics.mean(stage_ms["select"])
+    long_region = total_ms > 1000.0
+    peak_tf = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
+    achieved = flop / (attn_ms * 1e-3) / 1e12
+    elt = 2 if w.dtype == "bf16" else 4
+    pool_bytes = (w.B * (w.Hq + 2 * w.Hkv) * w.S * w.D * elt +
+                  4 * (w.B * (w.Hq + w.Hkv) * w.nb * w.D + w.B * w.Hkv * w.nb))
+    line = {
+        "metric": METRIC, "value": world * flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": f"synthetic, seeded ({w.name}: N(0,1) Q/K/V, RoPE theta {w.rope_theta}, K row 0 "
+                f"x{w.sink_scale}, {w.n_v_outliers()} V rows per kv-head x{w.v_outlier_scale}, "
+                f"heavy-tail fraction {w.heavy_tail_frac})",
+        "config": dict(config_of(w), kept_pairs=pairs, effective_tflop=flop / 1e12,
+                       causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
+        "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                     "traffic": None,
+                     "peak_source": f"{pk_kind} {'sustained' if long_region else 'burst'} "
+                                    "bf16 dense"},
+        "kernels": {
+            "pool": {"ms": pool_ms, "bound": "hbm", "bytes": pool_bytes,
+                     "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                     "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "select": {"ms": sel_ms},
+            "attn": {"ms": attn_ms, "tflops": achieved},
+        },
+        "clocks": clk,
+        "gpu_launches": 3 * K,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w):
+    """The oracle, as it stands, on a bounded sample: one kv-head group's selection plus exact
+    attention of 64 query blocks per q-head (blocks 0, 1, nb-1 and 61 random, seed 7)."""
+    import oracle
+
+    q, k, v = cpu_inputs(w)
+    G = w.Hq // w.Hkv
+    wg = w.replace(Hq=G, Hkv=1)
+    rows = wl.sample_rows(wg, n_random=61, seed=7)
+    flop, sec, parts = oracle_sample_step(w, q, k, v, rows)
+    return {"value": flop / sec / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": (f"one kv-head group ({G} q-heads): pooling, metric and selection of all "
+                       f"{w.nb} query blocks ({parts['select_s']:.2f} s, prorated to the sampled "
+                       f"rows) + exact fp64 attention of {len(rows)} query blocks "
+                       f"({parts['attn_s']:.2f} s)")}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,490 @@
+// C ABI of the Stem block-sparse causal prefill library (declared in include/stem.h).
+//
+// Host responsibilities: argument validation (before anything is enqueued), the Token
+// Position-Decay budget in double precision ("Stem: Rethinking Causal Information Flow in
+// Sparse Attention", gist.science/es "Resumen tecnico" 2.A; gist.science/it 2.A; exponential
+// decay per the shd-paper.top "key design" paragraph), a per-parameter plan cache, the
+// workspace carve-up, and the launch sequence pool -> select -> sparse attention.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "stem.h"
+#include "stem_internal.h"
+
+namespace stem {
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ------------------------------------------------------------------ budget
+
+bool budget_params_ok(int nb, float rho_min, float tau, int k_min) {
+  return nb >= 0 && std::isfinite(rho_min) && rho_min > 0.0f && rho_min <= 1.0f &&
+         std::isfinite(tau) && tau > 0.0f && k_min >= 1;
+}
+
+// k(i) = min(i+1, max(k_min, ceil(rho(i) (i+1)))), rho(i) = rho_min + (1-rho_min) e^{-i/tau};
+// block 0 alone at i = 0, at least the sink and the diagonal for i >= 1.
+int budget_k(int i, double rho_min, double tau, int k_min) {
+  if (i == 0) return 1;
+  const double rho = rho_min + (1.0 - rho_min) * std::exp(-static_cast<double>(i) / tau);
+  const double want = std::ceil(rho * static_cast<double>(i + 1));
+  double kk = std::max(want, static_cast<double>(k_min));
+  kk = std::min(kk, static_cast<double>(i + 1));
+  return std::max(2, static_cast<int>(kk));
+}
+
+struct Plan {
+  int nb = 0;
+  int64_t cap = 0;
+  int32_t* host = nullptr;  // pinned: k[nb] | off[nb+1] | order[nb]
+  size_t bytes = 0;
+};
+
+using PlanKey = std::tuple<int, uint32_t, uint32_t, int>;
+std::mutex g_plan_mu;
+std::map<PlanKey, Plan> g_plans;
+
+uint32_t fbits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return u;
+}
+
+size_t plan_bytes(int nb) { return align_up(sizeof(int32_t) * (3 * static_cast<size_t>(nb) + 1)); }
+
+// Returns the cached plan (building it on first use), or nullptr on a pinned-allocation failure.
+const Plan* get_plan(int nb, float rho_min, float tau, int k_min) {
+  std::lock_guard<std::mutex> lock(g_plan_mu);
+  const PlanKey key{nb, fbits(rho_min), fbits(tau), k_min};
+  auto it = g_plans.find(key);
+  if (it != g_plans.end()) return &it->second;
+  Plan p;
+  p.nb = nb;
+  p.bytes = plan_bytes(nb);
+  if (cudaMallocHost(reinterpret_cast<void**>(&p.host), p.bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::memset(p.host, 0, p.bytes);
+  int32_t* k = p.host;
+  int32_t* off = k + nb;
+  int32_t* order = off + nb + 1;
+  int64_t tot = 0;
+  for (int i = 0; i < nb; ++i) {
+    k[i] = budget_k(i, rho_min, tau, k_min);
+    off[i] = static_cast<int32_t>(tot);
+    tot += k[i];
+  }
+  off[nb] = static_cast<int32_t>(tot);
+  p.cap = tot;
+  for (int i = 0; i < nb; ++i) order[i] = i;
+  // heaviest query blocks first; equal budgets: later blocks first
+  std::stable_sort(order, order + nb, [&](int a, int b) {
+    return k[a] != k[b] ? k[a] > k[b] : a > b;
+  });
+  return &g_plans.emplace(key, p).first->second;
+}
+
+// ------------------------------------------------------------------ workspace layout
+
+struct Layout {
+  size_t status = 0, plan = 0, qbar = 0, kbar = 0, vnorm = 0, total = 0;
+};
+
+Layout layout(int B, int Hq, int Hkv, int nb, int D) {
+  Layout L;
+  size_t o = 0;
+  L.status = o;
+  o += kAlign;
+  L.plan = o;
+  o += plan_bytes(nb);
+  L.qbar = o;
+  o += align_up(sizeof(float) * static_cast<size_t>(B) * Hq * nb * D);
+  L.kbar = o;
+  o += align_up(sizeof(float) * static_cast<size_t>(B) * Hkv * nb * D);
+  L.vnorm = o;
+  o += align_up(sizeof(float) * static_cast<size_t>(B) * Hkv * nb);
+  L.total = o;
+  return L;
+}
+
+// ------------------------------------------------------------------ validation
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int B, int Hq, int Hkv, int S, int D, int block, int dtype) {
+  if (B < 0 || S < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return STEM_ERR_ARG;
+  if (D != 64 && D != 128) return STEM_ERR_ARG;
+  if (block != 64 && block != 128) return STEM_ERR_ARG;
+  if (dtype != STEM_BF16 && dtype != STEM_F32) return STEM_ERR_ARG;
+  if (S % block != 0) return STEM_ERR_ARG;
+  // element counts must fit comfortably in int64 and grid sizes in int32
+  const int64_t nb = S / block;
+  if (static_cast<int64_t>(B) * Hq * nb > 0x7fffffffLL / 4) return STEM_ERR_UNSUPPORTED;
+  if (nb > STEM_MAX_NB) return STEM_ERR_UNSUPPORTED;
+  return STEM_OK;
+}
+
+bool is_empty(int B, int S) { return B == 0 || S == 0; }
+
+int check_params(int nb, float rho_min, float tau, int k_min) {
+  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
+  // off[] is int32: the capacity must fit
+  const int64_t cap = stem_sel_capacity(nb, rho_min, tau, k_min);
+  if (cap < 0 || cap > 0x7fffffffLL) return STEM_ERR_UNSUPPORTED;
+  return STEM_OK;
+}
+
+int cuda_err(cudaError_t e) {
+  if (e == cudaSuccess) return STEM_OK;
+  cudaGetLastError();  // clear a sticky launch error in this thread's runtime state
+  return STEM_ERR_CUDA;
+}
+
+int upload_plan(const Plan* p, void* ws, const Layout& L, cudaStream_t st, PlanDev* dev) {
+  auto* base = static_cast<unsigned char*>(ws) + L.plan;
+  const cudaError_t e = cudaMemcpyAsync(base, p->host, p->bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_err(e);
+  const auto* k = reinterpret_cast<const int32_t*>(base);
+  dev->k = k;
+  dev->off = k + p->nb;
+  dev->order = k + 2 * p->nb + 1;
+  return STEM_OK;
+}
+
+int elem_size(int dtype) { return dtype == STEM_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------------ the path
+
+int run_prefill(const stem_args_t* a, cudaStream_t st) {
+  if (a == nullptr) return STEM_ERR_ARG;
+  int rc = check_shape(a->B, a->Hq, a->Hkv, a->S, a->D, a->block, a->dtype);
+  if (rc != STEM_OK) return rc;
+  const int nb = a->S / a->block;
+  rc = check_params(nb, a->rho_min, a->tau, a->k_min);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(a->B, a->S)) return STEM_OK;
+  if (!a->q || !a->k || !a->v || !a->out || !a->sel_idx || !a->sel_cnt) return STEM_ERR_ARG;
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->out, 16) ||
+      !aligned(a->sel_idx, 4) || !aligned(a->sel_cnt, 4) || !aligned(a->status, 4))
+    return STEM_ERR_ARG;
+  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D);
+  if (a->workspace == nullptr || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total)
+    return STEM_ERR_WORKSPACE;
+  const Plan* plan = get_plan(nb, a->rho_min, a->tau, a->k_min);
+  if (plan == nullptr) return STEM_ERR_CUDA;
+
+  auto* ws = static_cast<unsigned char*>(a->workspace);
+  if (a->status) {
+    rc = cuda_err(cudaMemsetAsync(a->status, 0, sizeof(int32_t), st));
+    if (rc != STEM_OK) return rc;
+  }
+  PlanDev pd;
+  rc = upload_plan(plan, ws, L, st, &pd);
+  if (rc != STEM_OK) return rc;
+  float* qbar = reinterpret_cast<float*>(ws + L.qbar);
+  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  float* vnorm = reinterpret_cast<float*>(ws + L.vnorm);
+  auto mark = [&](int n) -> int {
+    if (a->events == nullptr || a->events[n] == nullptr) return STEM_OK;
+    return cuda_err(cudaEventRecord(static_cast<cudaEvent_t>(a->events[n]), st));
+  };
+  if ((rc = mark(0)) != STEM_OK) return rc;
+  rc = cuda_err(launch_pool(a->q, a->k, a->v, a->dtype, a->B, a->Hq, a->Hkv, a->S, a->D,
+                            a->block, qbar, kbar, vnorm, st));
+  if (rc != STEM_OK) return rc;
+  if ((rc = mark(1)) != STEM_OK) return rc;
+  rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, plan->cap,
+                              a->sel_idx, a->sel_cnt, nullptr, st));
+  if (rc != STEM_OK) return rc;
+  if ((rc = mark(2)) != STEM_OK) return rc;
+  if (a->dtype == STEM_BF16) {
+    rc = cuda_err(launch_attn_bf16(a->q, a->k, a->v, a->B, a->Hq, a->Hkv, a->S, a->D, a->block,
+                                   pd, plan->cap, a->sel_idx, a->sel_cnt, a->out, a->status, st));
+  } else {
+    rc = cuda_err(launch_attn_f32(static_cast<const float*>(a->q),
+                                  static_cast<const float*>(a->k),
+                                  static_cast<const float*>(a->v), a->B, a->Hq, a->Hkv, a->S,
+                                  a->D, a->block, pd, plan->cap, a->sel_idx, a->sel_cnt,
+                                  static_cast<float*>(a->out), st));
+  }
+  if (rc != STEM_OK) return rc;
+  return mark(3);
+}
+
+// Internal grow-only device buffers, one per (device, user): slot 0 is stem_prefill's
+// workspace, slot 1 the arena of stem_prefill_host.
+struct DeviceScratch {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_scratch_mu;
+std::map<std::pair<int, int>, DeviceScratch> g_scratch;
+
+int get_scratch(size_t need, void** out, int slot) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  DeviceScratch& s = g_scratch[{dev, slot}];
+  if (s.bytes < need) {
+    if (s.ptr) {
+      // the previous buffer may still be read by queued work
+      e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_err(e);
+      cudaFree(s.ptr);
+      s.ptr = nullptr;
+      s.bytes = 0;
+    }
+    e = cudaMalloc(&s.ptr, need);
+    if (e != cudaSuccess) return cuda_err(e);
+    s.bytes = need;
+  }
+  *out = s.ptr;
+  return STEM_OK;
+}
+
+}  // namespace
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace stem
+
+using namespace stem;
+
+extern "C" {
+
+int stem_budget(int nb, float rho_min, float tau, int k_min, int32_t* k_out, int32_t* off_out) {
+  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
+  int64_t tot = 0;
+  for (int i = 0; i < nb; ++i) {
+    const int k = budget_k(i, rho_min, tau, k_min);
+    if (off_out) off_out[i] = static_cast<int32_t>(tot);
+    if (k_out) k_out[i] = k;
+    tot += k;
+    if (tot > 0x7fffffffLL) return STEM_ERR_ARG;
+  }
+  if (off_out) off_out[nb] = static_cast<int32_t>(tot);
+  return STEM_OK;
+}
+
+int64_t stem_sel_capacity(int nb, float rho_min, float tau, int k_min) {
+  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
+  int64_t tot = 0;
+  for (int i = 0; i < nb; ++i) tot += budget_k(i, rho_min, tau, k_min);
+  return tot;
+}
+
+size_t stem_workspace_size(int B, int Hq, int Hkv, int S, int D, int block) {
+  if (check_shape(B, Hq, Hkv, S, D, block, STEM_BF16) != STEM_OK) return 0;
+  if (is_empty(B, S)) return 0;
+  return layout(B, Hq, Hkv, S / block, D).total;
+}
+
+const char* stem_strerror(int code) {
+  switch (code) {
+    case STEM_OK: return "success";
+    case STEM_ERR_ARG: return "invalid argument (pointer, shape or budget parameter)";
+    case STEM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case STEM_ERR_CUDA: return "CUDA error (launch failure, no device or no sm_100a support)";
+    case STEM_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
+    case STEM_ERR_UNSUPPORTED: return "request exceeds this build's limits";
+    default: return "unknown error code";
+  }
+}
+
+int stem_prefill_ex(const stem_args_t* a, void* stream) {
+  return run_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int S,
+                 int D, int block, float rho_min, float tau, int k_min, void* out,
+                 int32_t* sel_idx, int32_t* sel_cnt) {
+  stem_args_t a;
+  std::memset(&a, 0, sizeof a);
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S = S;
+  a.D = D;
+  a.block = block;
+  a.rho_min = rho_min;
+  a.tau = tau;
+  a.k_min = k_min;
+  a.dtype = STEM_BF16;
+  a.out = out;
+  a.sel_idx = sel_idx;
+  a.sel_cnt = sel_cnt;
+  int rc = check_shape(B, Hq, Hkv, S, D, block, STEM_BF16);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, S)) return run_prefill(&a, nullptr);
+  rc = check_params(S / block, rho_min, tau, k_min);
+  if (rc != STEM_OK) return rc;
+  a.workspace_bytes = stem_workspace_size(B, Hq, Hkv, S, D, block);
+  rc = get_scratch(a.workspace_bytes, &a.workspace, 0);
+  if (rc != STEM_OK) return rc;
+  return run_prefill(&a, nullptr);
+}
+
+int stem_prefill_host(const stem_args_t* h) {
+  if (h == nullptr) return STEM_ERR_ARG;
+  int rc = check_shape(h->B, h->Hq, h->Hkv, h->S, h->D, h->block, h->dtype);
+  if (rc != STEM_OK) return rc;
+  const int nb = h->S / h->block;
+  rc = check_params(nb, h->rho_min, h->tau, h->k_min);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(h->B, h->S)) return STEM_OK;
+  if (!h->q || !h->k || !h->v || !h->out || !h->sel_idx || !h->sel_cnt) return STEM_ERR_ARG;
+  const size_t es = elem_size(h->dtype);
+  const size_t qb = es * static_cast<size_t>(h->B) * h->Hq * h->S * h->D;
+  const size_t kvb = es * static_cast<size_t>(h->B) * h->Hkv * h->S * h->D;
+  const int64_t cap = stem_sel_capacity(nb, h->rho_min, h->tau, h->k_min);
+  const size_t sib = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * cap;
+  const size_t scb = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * nb;
+  const Layout L = layout(h->B, h->Hq, h->Hkv, nb, h->D);
+  // device arena: workspace | q | k | v | out | sel_idx | sel_cnt
+  const size_t o_q = L.total, o_k = o_q + align_up(qb), o_v = o_k + align_up(kvb),
+               o_out = o_v + align_up(kvb), o_si = o_out + align_up(qb),
+               o_sc = o_si + align_up(sib), total = o_sc + align_up(scb);
+  static std::mutex host_mu;  // host-buffer calls share one arena: one at a time
+  std::lock_guard<std::mutex> lock(host_mu);
+  void* arena = nullptr;
+  rc = get_scratch(total, &arena, 1);
+  if (rc != STEM_OK) return rc;
+  auto* base = static_cast<unsigned char*>(arena);
+  cudaStream_t st = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_err(e);
+  stem_args_t d = *h;
+  d.q = base + o_q;
+  d.k = base + o_k;
+  d.v = base + o_v;
+  d.out = base + o_out;
+  d.sel_idx = reinterpret_cast<int32_t*>(base + o_si);
+  d.sel_cnt = reinterpret_cast<int32_t*>(base + o_sc);
+  d.workspace = base;
+  d.workspace_bytes = L.total;
+  d.status = reinterpret_cast<int32_t*>(base + L.status);
+  d.events = nullptr;
+  int32_t status = 0;
+  do {
+    if ((e = cudaMemcpyAsync(const_cast<void*>(d.q), h->q, qb, cudaMemcpyHostToDevice, st))) break;
+    if ((e = cudaMemcpyAsync(const_cast<void*>(d.k), h->k, kvb, cudaMemcpyHostToDevice, st))) break;
+    if ((e = cudaMemcpyAsync(const_cast<void*>(d.v), h->v, kvb, cudaMemcpyHostToDevice, st))) break;
+    rc = run_prefill(&d, st);
+    if (rc != STEM_OK) break;
+    if ((e = cudaMemcpyAsync(h->out, d.out, qb, cudaMemcpyDeviceToHost, st))) break;
+    if ((e = cudaMemcpyAsync(h->sel_idx, d.sel_idx, sib, cudaMemcpyDeviceToHost, st))) break;
+    if ((e = cudaMemcpyAsync(h->sel_cnt, d.sel_cnt, scb, cudaMemcpyDeviceToHost, st))) break;
+    if ((e = cudaMemcpyAsync(&status, d.status, sizeof status, cudaMemcpyDeviceToHost, st))) break;
+    e = cudaStreamSynchronize(st);
+  } while (false);
+  cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  if (rc != STEM_OK) return rc;
+  if (e != cudaSuccess) return cuda_err(e);
+  return status < 0 ? status : STEM_OK;
+}
+
+int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+              int S, int D, int block, float* qbar, float* kbar, float* vnorm, void* stream) {
+  int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, S)) return STEM_OK;
+  if (!q || !k || !v || !qbar || !kbar || !vnorm) return STEM_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(qbar, 16) ||
+      !aligned(kbar, 16) || !aligned(vnorm, 4))
+    return STEM_ERR_ARG;
+  return cuda_err(launch_pool(q, k, v, dtype, B, Hq, Hkv, S, D, block, qbar, kbar, vnorm,
+                              static_cast<cudaStream_t>(stream)));
+}
+
+int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
+                int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  if (nb < 0) return STEM_ERR_ARG;
+  if (nb > STEM_MAX_NB) return STEM_ERR_UNSUPPORTED;
+  // the selection sees blocks only: validate as a shape with block 64
+  int rc = check_shape(B, Hq, Hkv, nb * 64, D, 64, STEM_F32);
+  if (rc != STEM_OK) return rc;
+  rc = check_params(nb, rho_min, tau, k_min);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, nb)) return STEM_OK;
+  if (!qbar || !kbar || !vnorm || !sel_idx || !sel_cnt) return STEM_ERR_ARG;
+  if (!aligned(qbar, 16) || !aligned(kbar, 16) || !aligned(vnorm, 4) || !aligned(sel_idx, 4) ||
+      !aligned(sel_cnt, 4) || !aligned(m_out, 4))
+    return STEM_ERR_ARG;
+  const Layout L = layout(B, Hq, Hkv, nb, D);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.plan + plan_bytes(nb))
+    return STEM_ERR_WORKSPACE;
+  const Plan* plan = get_plan(nb, rho_min, tau, k_min);
+  if (plan == nullptr) return STEM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PlanDev pd;
+  rc = upload_plan(plan, workspace, L, st, &pd);
+  if (rc != STEM_OK) return rc;
+  return cuda_err(launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, plan->cap, sel_idx,
+                                sel_cnt, m_out, st));
+}
+
+int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                     int Hkv, int S, int D, int block, float rho_min, float tau, int k_min,
+                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
+                     size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
+  if (rc != STEM_OK) return rc;
+  const int nb = S / block;
+  rc = check_params(nb, rho_min, tau, k_min);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, S)) return STEM_OK;
+  if (!q || !k || !v || !out || !sel_idx || !sel_cnt) return STEM_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) || !aligned(status, 4))
+    return STEM_ERR_ARG;
+  const Layout L = layout(B, Hq, Hkv, nb, D);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.plan + plan_bytes(nb))
+    return STEM_ERR_WORKSPACE;
+  const Plan* plan = get_plan(nb, rho_min, tau, k_min);
+  if (plan == nullptr) return STEM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (status) {
+    rc = cuda_err(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    if (rc != STEM_OK) return rc;
+  }
+  PlanDev pd;
+  rc = upload_plan(plan, workspace, L, st, &pd);
+  if (rc != STEM_OK) return rc;
+  if (dtype == STEM_BF16)
+    return cuda_err(launch_attn_bf16(q, k, v, B, Hq, Hkv, S, D, block, pd, plan->cap, sel_idx,
+                                     sel_cnt, out, status, st));
+  return cuda_err(launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(k),
+                                  static_cast<const float*>(v), B, Hq, Hkv, S, D, block, pd,
+                                  plan->cap, sel_idx, sel_cnt, static_cast<float*>(out), st));
+}
+
+}  // extern "C"

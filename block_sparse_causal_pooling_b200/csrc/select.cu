@@ -1,0 +1,332 @@
+// Output-Aware Metric and variable-k top-k block selection, fused in one kernel.
+//
+// Method ("Stem: Rethinking Causal Information Flow in Sparse Attention"): rank the key blocks
+// of each query block by routing probability times value magnitude (gist.science/es "Resumen
+// tecnico" 2.B; gist.science/it 2.B; gist.science/nl OAM; gist.science/fr 2.B), keep the
+// position-dependent number k(i) of them (es 2.A, it 2.A, nl TPD, fr 2.A), always including
+// the initial (sink) block (es 1, shd-paper.top English abstract) and the diagonal block.
+// On pooled blocks:
+//   s_ij = qbar_i . kbar_j / sqrt(D),  m_ij = softmax_{j<=i}(s_ij) * n_j.
+// Within row i, log m_ij = s_ij + ln n_j - logsumexp_j(s_ij), so ranking by
+//   key_ij = s_ij + ln n_j
+// ranks exactly like m_ij; the kernel ranks by key_ij in double (s_ij from a float32 dot
+// product, ln n_j in double) and never materialises m unless asked for it.
+//
+// Kept set of row i: {0, i} plus the k(i)-2 largest key_ij over j in [1, i-1], larger first,
+// equal keys to the lower j. Written ascending into the CSR slot of row (b, h, i).
+//
+// Design: one CTA (8 warps) per (b, h, R consecutive query blocks).
+//   phase 1 - s for the R rows and every j < i0+R: a float32 SIMT tile product (kbar tiles of
+//             64 blocks staged in shared memory, qbar rows broadcast), kept in shared memory;
+//   phase 2 - one warp per row: an exact radix select on the 64-bit order-preserving image of
+//             key_ij (8-bit digits, starting at the highest bit where the row's keys differ),
+//             then an ascending ballot compaction that takes the threshold ties lowest-j first.
+// Rows never touch HBM except for the CSR they write (and m_out when requested).
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "stem_internal.h"
+
+namespace stem {
+namespace {
+
+constexpr int kSelThreads = 256;
+constexpr int kWarps = kSelThreads / 32;
+constexpr int kTileJ = 64;
+
+__device__ __forceinline__ uint64_t order_bits(double x) {
+  // order-preserving map from double to uint64 (no NaNs expected)
+  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(x + 0.0));  // -0 -> +0
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+struct SelSmem {
+  float* s;       // [R][ldS] scaled logits
+  float* qs;      // [R][D]
+  float* ks;      // [kTileJ][D+4]
+  double* lnn;    // [ldS]
+  int* hist;      // [kWarps][256]
+};
+
+template <int D, int R>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar,
+    const float* __restrict__ vnorm, int BH, int Hq, int Hkv, int nb, int ldS, PlanDev plan,
+    int64_t cap, int32_t* __restrict__ sel_idx, int32_t* __restrict__ sel_cnt,
+    float* __restrict__ m_out) {
+  constexpr int RPW = R / kWarps;  // rows per warp in phase 1
+  constexpr int KLD = D + 4;       // padded kbar row (conflict-free 16-byte column reads)
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelSmem sm;
+  sm.s = reinterpret_cast<float*>(smem_raw);
+  sm.qs = sm.s + R * ldS;
+  sm.ks = sm.qs + R * D;
+  sm.lnn = reinterpret_cast<double*>(sm.ks + kTileJ * KLD);
+  sm.hist = reinterpret_cast<int*>(sm.lnn + ldS);
+
+  const int ntiles = (nb + R - 1) / R;
+  const int tile = ntiles - 1 - static_cast<int>(blockIdx.x / BH);  // heaviest tiles first
+  const int bh = static_cast<int>(blockIdx.x % BH);
+  const int b = bh / Hq, h = bh % Hq;
+  const int G = Hq / Hkv;
+  const int64_t bg = static_cast<int64_t>(b) * Hkv + h / G;
+  const int i0 = tile * R;
+  const int rows = min(R, nb - i0);
+  const int jend = i0 + rows;  // columns 0 .. jend-1
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+
+  const float* qsrc = qbar + (static_cast<int64_t>(bh) * nb + i0) * D;
+  const float* ksrc = kbar + bg * nb * D;
+  const float* nsrc = vnorm + bg * nb;
+
+  for (int idx = t; idx < R * D / 4; idx += kSelThreads) {
+    const int r = idx / (D / 4), c4 = idx % (D / 4);
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows) val = reinterpret_cast<const float4*>(qsrc + r * D)[c4];
+    reinterpret_cast<float4*>(sm.qs + r * D)[c4] = val;
+  }
+  for (int j = t; j < jend; j += kSelThreads) sm.lnn[j] = log(static_cast<double>(nsrc[j]));
+
+  const float scale = rsqrtf(static_cast<float>(D));
+  // ---- phase 1: s[r][j] for r < rows, j < jend
+  for (int j0 = 0; j0 < jend; j0 += kTileJ) {
+    __syncthreads();  // previous tile consumed (and qs / lnn visible on the first pass)
+    for (int idx = t; idx < kTileJ * D / 4; idx += kSelThreads) {
+      const int r = idx / (D / 4), c4 = idx % (D / 4);
+      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + r < jend) val = reinterpret_cast<const float4*>(ksrc + (j0 + r) * D)[c4];
+      *reinterpret_cast<float4*>(sm.ks + r * KLD + c4 * 4) = val;
+    }
+    __syncthreads();
+    float acc[RPW][2];
+#pragma unroll
+    for (int a = 0; a < RPW; ++a) acc[a][0] = acc[a][1] = 0.f;
+    const float* k0 = sm.ks + lane * KLD;
+    const float* k1 = sm.ks + (lane + 32) * KLD;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+      const float4 x0 = *reinterpret_cast<const float4*>(k0 + d);
+      const float4 x1 = *reinterpret_cast<const float4*>(k1 + d);
+#pragma unroll
+      for (int a = 0; a < RPW; ++a) {
+        const float4 qv = *reinterpret_cast<const float4*>(sm.qs + (warp * RPW + a) * D + d);
+        acc[a][0] = fmaf(qv.x, x0.x, acc[a][0]);
+        acc[a][0] = fmaf(qv.y, x0.y, acc[a][0]);
+        acc[a][0] = fmaf(qv.z, x0.z, acc[a][0]);
+        acc[a][0] = fmaf(qv.w, x0.w, acc[a][0]);
+        acc[a][1] = fmaf(qv.x, x1.x, acc[a][1]);
+        acc[a][1] = fmaf(qv.y, x1.y, acc[a][1]);
+        acc[a][1] = fmaf(qv.z, x1.z, acc[a][1]);
+        acc[a][1] = fmaf(qv.w, x1.w, acc[a][1]);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < RPW; ++a) {
+      const int r = warp * RPW + a;
+      if (j0 + lane < jend) sm.s[r * ldS + j0 + lane] = acc[a][0] * scale;
+      if (j0 + lane + 32 < jend) sm.s[r * ldS + j0 + lane + 32] = acc[a][1] * scale;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 2: one warp per row
+  int* hist = sm.hist + warp * 256;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int r = warp; r < rows; r += kWarps) {
+    const int i = i0 + r;
+    const float* srow = sm.s + r * ldS;
+    const int kk = plan.k[i];
+    int32_t* dst = sel_idx + static_cast<int64_t>(bh) * cap + plan.off[i];
+    if (lane == 0) sel_cnt[static_cast<int64_t>(bh) * nb + i] = kk;
+
+    if (m_out != nullptr) {  // diagnostic metric row, float32 softmax
+      float mx = -INFINITY;
+      for (int j = lane; j <= i; j += 32) mx = fmaxf(mx, srow[j]);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float z = 0.f;
+      for (int j = lane; j <= i; j += 32) z += expf(srow[j] - mx);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      float* mrow = m_out + static_cast<int64_t>(bh) * (static_cast<int64_t>(nb) * (nb + 1) / 2) +
+                    static_cast<int64_t>(i) * (i + 1) / 2;
+      for (int j = lane; j <= i; j += 32) mrow[j] = expf(srow[j] - mx) / z * nsrc[j];
+    }
+
+    if (i == 0) {
+      if (lane == 0) dst[0] = 0;
+      continue;
+    }
+    const int need = kk - 2;  // picks among j in [1, i-1]
+    if (need >= i - 1) {      // every causal block
+      for (int j = lane; j <= i; j += 32) dst[j] = j;
+      continue;
+    }
+    if (need <= 0) {
+      if (lane == 0) {
+        dst[0] = 0;
+        dst[1] = i;
+      }
+      continue;
+    }
+    auto key_bits = [&](int j) -> uint64_t {
+      return order_bits(static_cast<double>(srow[j]) + sm.lnn[j]);
+    };
+    // the highest bit where this row's candidate keys differ
+    uint64_t umin = ~0ull, umax = 0ull;
+    for (int j = 1 + lane; j < i; j += 32) {
+      const uint64_t u = key_bits(j);
+      umin = u < umin ? u : umin;
+      umax = u > umax ? u : umax;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const uint64_t a = __shfl_xor_sync(0xffffffffu, umin, o);
+      const uint64_t c = __shfl_xor_sync(0xffffffffu, umax, o);
+      umin = a < umin ? a : umin;
+      umax = c > umax ? c : umax;
+    }
+    uint64_t prefix, pmask;
+    int rem = need;
+    bool exact = false;
+    if (umin == umax) {  // all candidates tie: lowest indices
+      prefix = umin;
+      pmask = ~0ull;
+    } else {
+      const int top = 63 - __clzll(static_cast<long long>(umin ^ umax));  // highest differing bit
+      pmask = top >= 63 ? 0ull : (~0ull << (top + 1));
+      prefix = umin & pmask;
+      int shift = top - 7 < 0 ? 0 : top - 7;
+      while (true) {
+        for (int bin = lane; bin < 256; bin += 32) hist[bin] = 0;
+        __syncwarp();
+        for (int j = 1 + lane; j < i; j += 32) {
+          const uint64_t u = key_bits(j);
+          if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xff], 1);
+        }
+        __syncwarp();
+        // lane l owns bins 255-8l .. 248-8l (descending)
+        int cnt[8];
+        int local = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cnt[e] = hist[255 - 8 * lane - e];
+          local += cnt[e];
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int excl = incl - local;
+        const bool owner = excl < rem && rem <= incl;
+        int digit = 0, above = 0, dcount = 0;
+        if (owner) {
+          int run = excl;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (run + cnt[e] >= rem) {
+              digit = 255 - 8 * lane - e;
+              above = run;
+              dcount = cnt[e];
+              break;
+            }
+            run += cnt[e];
+          }
+        }
+        const int src = __ffs(__ballot_sync(0xffffffffu, owner)) - 1;
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        dcount = __shfl_sync(0xffffffffu, dcount, src);
+        __syncwarp();
+        rem -= above;
+        prefix = (prefix & ~(0xffull << shift)) | (static_cast<uint64_t>(digit) << shift);
+        pmask |= 0xffull << shift;
+        if (dcount == rem) {
+          exact = true;
+          break;
+        }
+        if (shift == 0) break;
+        shift = shift - 8 < 0 ? 0 : shift - 8;
+      }
+    }
+    // ascending emission; threshold ties (full key equal) lowest-j first
+    int written = 0, ties = 0;
+    for (int j0 = 0; j0 <= i; j0 += 32) {
+      const int j = j0 + lane;
+      bool sel = false, tie = false;
+      if (j <= i) {
+        if (j == 0 || j == i) {
+          sel = true;
+        } else {
+          const uint64_t um = key_bits(j) & pmask;
+          if (um > prefix) {
+            sel = true;
+          } else if (um == prefix) {
+            if (exact) sel = true;
+            else tie = true;
+          }
+        }
+      }
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      if (tie && ties + __popc(tb & lt_mask) < rem) sel = true;
+      ties += __popc(tb);
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      const int pos = written + __popc(sb & lt_mask);
+      if (sel && pos < kk) dst[pos] = j;  // never past this row's slot
+      written += __popc(sb);
+    }
+  }
+}
+
+template <int D, int R>
+cudaError_t launch_rt(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                      int Hkv, int nb, PlanDev plan, int64_t cap, int32_t* sel_idx,
+                      int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  const int ldS = (nb + 3) & ~3;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(R) * ldS + R * D + kTileJ * (D + 4)) +
+                      sizeof(double) * ldS + sizeof(int) * kWarps * 256;
+  auto kern = select_kernel<D, R>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int BH = B * Hq;
+  const int64_t grid = static_cast<int64_t>(BH) * ((nb + R - 1) / R);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kSelThreads, smem, st>>>(qbar, kbar, vnorm, BH, Hq, Hkv,
+                                                             nb, ldS, plan, cap, sel_idx,
+                                                             sel_cnt, m_out);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                     int Hkv, int nb, PlanDev plan, int64_t cap, int32_t* sel_idx,
+                     int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  if (nb <= 1024)
+    return launch_rt<D, 32>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt,
+                            m_out, st);
+  if (nb <= 2048)
+    return launch_rt<D, 16>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt,
+                            m_out, st);
+  return launch_rt<D, 8>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
+                         st);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
+                          int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
+                          int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  if (B * Hq == 0 || nb == 0) return cudaSuccess;
+  if (D == 128)
+    return launch_d<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
+                         st);
+  if (D == 64)
+    return launch_d<64>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
+                        st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace stem

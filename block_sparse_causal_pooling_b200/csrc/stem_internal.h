@@ -1,0 +1,41 @@
+// Internal declarations shared by the host API (api.cpp) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace stem {
+
+// Device view of the budget plan (int32 arrays inside the workspace).
+struct PlanDev {
+  const int32_t* k;      // [nb]   k(i)
+  const int32_t* off;    // [nb+1] prefix sums of k
+  const int32_t* order;  // [nb]   query blocks sorted by k(i) descending (heaviest first)
+};
+
+// Block pooling (pool.cu). dtype: 0 bf16, 1 f32.
+cudaError_t launch_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                        int Hkv, int S, int D, int block, float* qbar, float* kbar,
+                        float* vnorm, cudaStream_t st);
+
+// Metric + top-k selection (select.cu).
+cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
+                          int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
+                          int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st);
+
+// Block-sparse attention, bfloat16 inputs on the tensor cores (attn_bf16.cu).
+cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
+                             int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
+                             const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
+                             int32_t* status, cudaStream_t st);
+
+// Block-sparse attention, float32 inputs on the CUDA cores (attn_f32.cu).
+cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, int B, int Hq,
+                            int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
+                            const int32_t* sel_idx, const int32_t* sel_cnt, float* out,
+                            cudaStream_t st);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+}  // namespace stem

@@ -1,0 +1,266 @@
+"""Python binding of libstem.so (the C ABI in include/stem.h), via ctypes.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels. The
+binding allocates outputs and the workspace with torch when the caller does not pass them,
+reads device pointers and the current CUDA stream from torch, and raises StemError on a
+non-zero return code. There is no fallback: if libstem.so is missing or cannot be loaded,
+importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libstem.so")
+
+STEM_OK = 0
+STEM_ERR_ARG = -1
+STEM_ERR_WORKSPACE = -2
+STEM_ERR_CUDA = -3
+STEM_ERR_TIMEOUT = -4
+STEM_ERR_UNSUPPORTED = -5
+STEM_BF16 = 0
+STEM_F32 = 1
+STEM_MAX_NB = 4096
+
+
+class StemError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+class stem_args_t(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+        ("S", ctypes.c_int32), ("D", ctypes.c_int32), ("block", ctypes.c_int32),
+        ("rho_min", ctypes.c_float), ("tau", ctypes.c_float), ("k_min", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("status", ctypes.c_void_p),
+        ("events", ctypes.POINTER(ctypes.c_void_p)),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m block_sparse_causal_pooling_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "stem_prefill": (I, [P, P, P, I, I, I, I, I, I, F, F, I, P, P, P]),
+        "stem_prefill_ex": (I, [ctypes.POINTER(stem_args_t), P]),
+        "stem_prefill_host": (I, [ctypes.POINTER(stem_args_t)]),
+        "stem_budget": (I, [I, F, F, I, P, P]),
+        "stem_sel_capacity": (ctypes.c_int64, [I, F, F, I]),
+        "stem_workspace_size": (Z, [I, I, I, I, I, I]),
+        "stem_strerror": (ctypes.c_char_p, [I]),
+        "stem_pool": (I, [P, P, P, I, I, I, I, I, I, I, P, P, P, P]),
+        "stem_select": (I, [P, P, P, I, I, I, I, I, F, F, I, P, P, P, P, Z, P]),
+        "stem_sparse_attn": (I, [P, P, P, I, I, I, I, I, I, I, F, F, I, P, P, P, P, Z, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+# Every symbol include/stem.h declares.
+EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget",
+            "stem_sel_capacity", "stem_workspace_size", "stem_strerror", "stem_pool",
+            "stem_select", "stem_sparse_attn")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return _lib.stem_strerror(int(code)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != STEM_OK:
+        raise StemError(rc, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return STEM_BF16
+    if t.dtype == torch.float32:
+        return STEM_F32
+    raise TypeError(f"inputs must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ host-only helpers
+
+
+def stem_budget(nb: int, rho_min: float, tau: float, k_min: int):
+    """(k [nb] int32, off [nb+1] int32) of the position-decay budget (host)."""
+    k = torch.zeros(max(nb, 1), dtype=torch.int32)
+    off = torch.zeros(nb + 1, dtype=torch.int32)
+    _check(_lib.stem_budget(nb, rho_min, tau, k_min, _ptr(k), _ptr(off)), "stem_budget")
+    return k[:nb].clone(), off
+
+
+def stem_sel_capacity(nb: int, rho_min: float, tau: float, k_min: int) -> int:
+    cap = int(_lib.stem_sel_capacity(nb, rho_min, tau, k_min))
+    if cap < 0:
+        raise StemError(cap, "stem_sel_capacity")
+    return cap
+
+
+def stem_workspace_size(B: int, Hq: int, Hkv: int, S: int, D: int, block: int) -> int:
+    return int(_lib.stem_workspace_size(B, Hq, Hkv, S, D, block))
+
+
+# ------------------------------------------------------------------ device calls
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor):
+    B, Hq, S, D = q.shape
+    return B, Hq, k.shape[1], S, D
+
+
+def alloc_outputs(q: torch.Tensor, k: torch.Tensor, block: int, rho_min: float, tau: float,
+                  k_min: int):
+    """(out, sel_idx, sel_cnt) allocated on q's device."""
+    B, Hq, Hkv, S, D = _shape(q, k)
+    nb = S // block
+    cap = stem_sel_capacity(nb, rho_min, tau, k_min)
+    out = torch.empty_like(q)
+    sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=q.device)
+    sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=q.device)
+    return out, sel_idx, sel_cnt
+
+
+def alloc_workspace(q: torch.Tensor, k: torch.Tensor, block: int) -> torch.Tensor:
+    B, Hq, Hkv, S, D = _shape(q, k)
+    n = stem_workspace_size(B, Hq, Hkv, S, D, block)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
+def make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, workspace=None,
+              status=None, events=None) -> stem_args_t:
+    B, Hq, Hkv, S, D = _shape(q, k)
+    a = stem_args_t()
+    a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    a.B, a.Hq, a.Hkv, a.S, a.D, a.block = B, Hq, Hkv, S, D, block
+    a.rho_min, a.tau, a.k_min = rho_min, tau, k_min
+    a.dtype = _dtype_code(q)
+    a.out, a.sel_idx, a.sel_cnt = out.data_ptr(), sel_idx.data_ptr(), sel_cnt.data_ptr()
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    if status is not None:
+        a.status = status.data_ptr()
+    if events is not None:  # 4 torch.cuda.Event (already created with timing enabled)
+        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        a._events_keepalive = arr
+        a.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    return a
+
+
+def stem_prefill_ex(q, k, v, block, rho_min, tau, k_min, out=None, sel_idx=None, sel_cnt=None,
+                    workspace=None, status=None, stream=None, events=None):
+    """Whole path on device tensors [B,H,S,D] (bf16 or f32). Returns (out, sel_idx, sel_cnt).
+    Asynchronous on `stream` (default: torch's current stream). `events`: optional four
+    torch.cuda.Event recorded before pooling, selection, attention and after attention."""
+    if out is None or sel_idx is None or sel_cnt is None:
+        out, sel_idx, sel_cnt = alloc_outputs(q, k, block, rho_min, tau, k_min)
+    if workspace is None:
+        workspace = alloc_workspace(q, k, block)
+    a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, workspace, status,
+                  events)
+    _check(_lib.stem_prefill_ex(ctypes.byref(a), _stream(stream)), "stem_prefill_ex")
+    return out, sel_idx, sel_cnt
+
+
+def stem_prefill(q, k, v, block, rho_min, tau, k_min, out=None, sel_idx=None, sel_cnt=None):
+    """Whole path, bf16 device tensors, the legacy default stream, the library's own workspace."""
+    if out is None or sel_idx is None or sel_cnt is None:
+        out, sel_idx, sel_cnt = alloc_outputs(q, k, block, rho_min, tau, k_min)
+    B, Hq, Hkv, S, D = _shape(q, k)
+    _check(_lib.stem_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, S, D, block,
+                             rho_min, tau, k_min, out.data_ptr(), sel_idx.data_ptr(),
+                             sel_cnt.data_ptr()), "stem_prefill")
+    return out, sel_idx, sel_cnt
+
+
+def stem_prefill_host(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt) -> None:
+    """Whole path on HOST tensors (pinned for speed); synchronous."""
+    a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt)
+    _check(_lib.stem_prefill_host(ctypes.byref(a)), "stem_prefill_host")
+
+
+def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None):
+    B, Hq, Hkv, S, D = _shape(q, k)
+    nb = S // block
+    dev = q.device
+    if qbar is None:
+        qbar = torch.empty((B, Hq, nb, D), dtype=torch.float32, device=dev)
+        kbar = torch.empty((B, Hkv, nb, D), dtype=torch.float32, device=dev)
+        vnorm = torch.empty((B, Hkv, nb), dtype=torch.float32, device=dev)
+    _check(_lib.stem_pool(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq, Hkv,
+                          S, D, block, qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(),
+                          _stream(stream)), "stem_pool")
+    return qbar, kbar, vnorm
+
+
+def stem_select(qbar, kbar, vnorm, rho_min, tau, k_min, with_metric=False, workspace=None,
+                sel_idx=None, sel_cnt=None, stream=None):
+    """CSR selection from pooled summaries (float32 device tensors). Returns (sel_idx, sel_cnt,
+    m or None)."""
+    B, Hq, nb, D = qbar.shape
+    Hkv = kbar.shape[1]
+    dev = qbar.device
+    cap = stem_sel_capacity(nb, rho_min, tau, k_min)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=dev)
+        sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=dev)
+    m = (torch.empty((B, Hq, nb * (nb + 1) // 2), dtype=torch.float32, device=dev)
+         if with_metric else None)
+    if workspace is None:
+        workspace = torch.empty(max(stem_workspace_size(B, Hq, Hkv, nb * 64, D, 64), 256),
+                                dtype=torch.uint8, device=dev)
+    _check(_lib.stem_select(qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(), B, Hq, Hkv, nb,
+                            D, rho_min, tau, k_min, sel_idx.data_ptr(), sel_cnt.data_ptr(),
+                            _ptr(m), workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "stem_select")
+    return sel_idx, sel_cnt, m
+
+
+def stem_sparse_attn(q, k, v, block, rho_min, tau, k_min, sel_idx, sel_cnt, out=None,
+                     workspace=None, status=None, stream=None):
+    B, Hq, Hkv, S, D = _shape(q, k)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(q, k, block)
+    _check(_lib.stem_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq,
+                                 Hkv, S, D, block, rho_min, tau, k_min, sel_idx.data_ptr(),
+                                 sel_cnt.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                 workspace.numel(), _ptr(status), _stream(stream)),
+           "stem_sparse_attn")
+    return out

@@ -1,0 +1,184 @@
+/*
+ * stem.h: C ABI of the B200 (sm_100a) library for Stem block-sparse causal prefill.
+ *
+ * The method: "Stem: Rethinking Causal Information Flow in Sparse Attention"
+ * (arXiv 2603.06274). Passages are cited by page and section:
+ *   [es] gist.science/es, "Resumen tecnico"        [it] gist.science/it, "Sommario tecnico"
+ *   [nl] gist.science/nl, "Technische samenvatting" [fr] gist.science/fr, "Resume technique"
+ *   [zh] shd-paper.top index page (English abstract, "key design" paragraph)
+ *
+ * Problem ([es] 1, [it] 1, [nl] Probleemstelling, [zh] abstract): causal prefill
+ * attention over Q, K, V in which each query block attends only to a kept set of
+ * key blocks. The pages leave the budget schedule and the pooling open; this
+ * library fixes them as parameters:
+ *   nb = S / block, query block i in [0, nb);
+ *   rho(i) = rho_min + (1 - rho_min) * exp(-i / tau);
+ *   k(i)   = min(i+1, max(k_min, ceil(rho(i) * (i+1)))), raised to 2 for i >= 1, k(0) = 1;
+ *   pooled qbar_i, kbar_j = mean of the block's rows; n_j = mean of the block's V-row L2 norms;
+ *   m_ij   = softmax_{j<=i}(qbar_i . kbar_j / sqrt(D)) * n_j;
+ *   kept(i) = {0, i} plus the k(i)-2 best j in [1, i-1] by (m_ij descending, j ascending);
+ *   out[r] = softmax attention of query token r over every token of kept(i), token-causal
+ *            inside block i, logits scaled by 1/sqrt(D).
+ *
+ * Conventions shared by every call:
+ *   - Tensors are contiguous [B, H, S, D] (row-major, D fastest). Q and out have Hq heads, K and
+ *     V have Hkv heads; query head h reads key/value head h / (Hq / Hkv).
+ *   - dtype: STEM_BF16 (bfloat16) or STEM_F32 (float32); out has the input dtype.
+ *   - Device pointers must be 16-byte aligned (int32 arrays: 4-byte aligned). All buffers are
+ *     owned by the caller; the library never frees or retains them past the call.
+ *   - CSR layout of the kept blocks: row (b, h, i) occupies
+ *       sel_idx[(b*Hq + h)*cap + off(i) .. + k(i)), ascending block indices,
+ *     with off(i) = k(0) + ... + k(i-1) and cap = off(nb) (stem_sel_capacity); sel_cnt[b,h,i] = k(i).
+ *   - Supported shapes: D in {64, 128}; block in {64, 128}; S % block == 0; Hq % Hkv == 0;
+ *     nb <= STEM_MAX_NB. B == 0 or S == 0 is an empty problem: success, nothing launched.
+ *   - Device calls are asynchronous on the given stream: a 0 return means the work was enqueued.
+ *     Faults surface at the caller's next synchronisation. The library never prints or aborts.
+ *   - Arguments are validated before anything is enqueued; on a negative return nothing was
+ *     launched and no buffer was written.
+ */
+#ifndef STEM_H
+#define STEM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define STEM_OK 0
+#define STEM_ERR_ARG (-1)         /* bad argument: null/misaligned pointer, bad shape or parameter */
+#define STEM_ERR_WORKSPACE (-2)   /* workspace missing or smaller than stem_workspace_size() */
+#define STEM_ERR_CUDA (-3)        /* a CUDA call failed (launch error, no device, no sm_100a) */
+#define STEM_ERR_TIMEOUT (-4)     /* a device-side wait exceeded its bound (reported via status) */
+#define STEM_ERR_UNSUPPORTED (-5) /* valid request beyond this build's limits (e.g. nb > STEM_MAX_NB) */
+
+/* Element types. */
+#define STEM_BF16 0
+#define STEM_F32 1
+
+/* Largest number of blocks per sequence (the selection kernel keeps one score row per
+ * query block in shared memory). */
+#define STEM_MAX_NB 4096
+
+/*
+ * Full argument set of one prefill. Sizes are element counts.
+ *   q   [B,Hq,S,D], k, v [B,Hkv,S,D]      inputs (device, or host for stem_prefill_host)
+ *   out [B,Hq,S,D]                         output, same dtype as the inputs
+ *   sel_idx [B,Hq,cap] int32, sel_cnt [B,Hq,nb] int32   kept blocks (CSR, see above)
+ *   workspace / workspace_bytes            device scratch of at least stem_workspace_size() bytes,
+ *                                          256-byte aligned; ignored by stem_prefill_host
+ *   status                                 optional device int32: set to 0 when the call is
+ *                                          enqueued, to a negative STEM_ERR_* by a kernel that
+ *                                          fails a bounded device-side wait; NULL to skip
+ *   events                                 optional: 4 cudaEvent_t (as void*) recorded on the
+ *                                          stream before pooling, before selection, before
+ *                                          attention and after attention (per-stage timing);
+ *                                          NULL to skip
+ */
+typedef struct stem_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  int32_t B, Hq, Hkv, S, D, block;
+  float rho_min; /* in (0, 1] */
+  float tau;     /* decay length in blocks, > 0 and finite */
+  int32_t k_min; /* >= 1 */
+  int32_t dtype; /* STEM_BF16 or STEM_F32 */
+  void* out;
+  int32_t* sel_idx;
+  int32_t* sel_cnt;
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* status;
+  void* const* events;
+} stem_args_t;
+
+/*
+ * The whole hot path ([es] 2 "Implementacion" steps 1-3, [it] 2.C, [nl] Implementatie,
+ * [fr] 2.C): block pooling, budget, metric and selection, block-sparse attention.
+ * bfloat16 device tensors, the default stream, and a workspace the library allocates on first
+ * use and keeps per device (grow-only, freed at process exit). Returns STEM_OK or STEM_ERR_*.
+ */
+int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int S,
+                 int D, int block, float rho_min, float tau, int k_min, void* out,
+                 int32_t* sel_idx, int32_t* sel_cnt);
+
+/* Same as stem_prefill with every argument explicit: dtype, caller workspace, status word, and
+ * the CUDA stream (a cudaStream_t passed as void*; NULL = legacy default stream). */
+int stem_prefill_ex(const stem_args_t* a, void* stream);
+
+/* stem_prefill_ex for HOST buffers (q, k, v, out, sel_idx, sel_cnt in host memory; pinned
+ * memory gives the fastest copies). Copies inputs to the device, runs the path on an internal
+ * stream and workspace, copies out, sel_idx and sel_cnt back, and returns after they have
+ * arrived. a->workspace and a->status are ignored. */
+int stem_prefill_host(const stem_args_t* a);
+
+/*
+ * Token Position-Decay budget ([es] 2.A, [it] 2.A, [nl] TPD, [fr] 2.A; exponential decay:
+ * [zh] key design). Host only. Writes k_out[nb] = k(i) and off_out[nb+1] = prefix sums into
+ * host arrays (either may be NULL). Returns 0, or STEM_ERR_ARG for nb < 0, rho_min outside (0, 1],
+ * tau <= 0 or not finite, k_min < 1, or a total that overflows int32.
+ */
+int stem_budget(int nb, float rho_min, float tau, int k_min, int32_t* k_out, int32_t* off_out);
+
+/* cap = sum_i k(i): the per-(b, h) stride of sel_idx. Host only. Negative STEM_ERR_ARG on bad
+ * parameters. */
+int64_t stem_sel_capacity(int nb, float rho_min, float tau, int k_min);
+
+/* Bytes of device workspace stem_prefill_ex needs for this shape (pooled summaries, the budget
+ * plan and the status word). 0 for an invalid or empty shape. Host only. */
+size_t stem_workspace_size(int B, int Hq, int Hkv, int S, int D, int block);
+
+/* Static description of a return code. Never NULL. */
+const char* stem_strerror(int code);
+
+/* ---------------------------------------------------------------------------------------
+ * Stage entry points: the same kernels the full path launches, one at a time. They exist so
+ * each stage can be checked on its own; the device layout of every intermediate is fixed here.
+ * --------------------------------------------------------------------------------------- */
+
+/*
+ * Block downsampling ([es] 2 "Implementacion" step 1, [it] 2.C step 1, [nl] Implementatie
+ * step 1, [fr] 2.C step 1), mean pooling. Writes (device, float32):
+ *   qbar [B,Hq,nb,D]  = mean of the block's Q rows,
+ *   kbar [B,Hkv,nb,D] = mean of the block's K rows,
+ *   vnorm [B,Hkv,nb]  = mean over the block's rows of ||V row||_2.
+ * Accumulation is float32 in a fixed tree order (deterministic).
+ */
+int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+              int S, int D, int block, float* qbar, float* kbar, float* vnorm, void* stream);
+
+/*
+ * Output-Aware Metric and variable-k selection ([es] 2.B and 2 "Implementacion" step 3,
+ * [it] 2.B, [nl] OAM, [fr] 2.B; sink retention: [es] 1, [zh] abstract). From pooled summaries
+ * (device float32, layouts of stem_pool) writes the CSR kept-block lists sel_idx / sel_cnt.
+ * Ranking uses log m_ij + const = s_ij + ln n_j with s_ij from a float32 dot product, compared
+ * in double; ties go to the lower block index.
+ * m_out: optional (NULL to skip) float32 [B,Hq,nb*(nb+1)/2], row i at offset i*(i+1)/2, the
+ * metric m_ij for j <= i (softmax over j <= i in float32).
+ * workspace: as for stem_prefill_ex (only the plan region is used).
+ */
+int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
+                int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/*
+ * Exact attention over the kept blocks ([es] 2 "Implementacion" step 3, [it] 2.C step 3,
+ * [nl] Implementatie step 3, [fr] 2.C step 3). Reads any valid CSR with the budget's layout
+ * (sel_cnt[b,h,i] must equal k(i); each row ascending, in [0, i], containing i). bfloat16 runs
+ * on the tensor cores with float32 accumulation and float32 online softmax; float32 runs on the
+ * CUDA cores in float32.
+ */
+int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                     int Hkv, int S, int D, int block, float rho_min, float tau, int k_min,
+                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
+                     size_t workspace_bytes, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STEM_H */

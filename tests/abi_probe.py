@@ -1,0 +1,93 @@
+"""Invalid-argument probes of the C ABI, run in a subprocess with CUDA_VISIBLE_DEVICES=''.
+
+Every call here must be rejected by host-side validation before anything touches CUDA; with
+the devices hidden, a validation bug could not launch a kernel anyway. Prints one JSON object
+{case: return code}.
+"""
+
+import ctypes
+import json
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+assert os.environ.get("CUDA_VISIBLE_DEVICES") == "", "run with CUDA_VISIBLE_DEVICES=''"
+
+from block_sparse_causal_pooling_b200 import stem as S  # noqa: E402
+
+L = S.lib()
+FAKE = 0x7F0000000000  # 256-byte aligned, never dereferenced
+
+
+def base(**kw):
+    a = S.stem_args_t()
+    a.q = a.k = a.v = FAKE
+    a.out = FAKE + 0x100
+    a.sel_idx = FAKE + 0x200
+    a.sel_cnt = FAKE + 0x300
+    a.B, a.Hq, a.Hkv, a.S, a.D, a.block = 1, 4, 2, 1024, 128, 128
+    a.rho_min, a.tau, a.k_min, a.dtype = 0.25, 4.0, 2, 0
+    a.workspace = FAKE + 0x1000
+    a.workspace_bytes = 1 << 30
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def ex(**kw):
+    return L.stem_prefill_ex(ctypes.byref(base(**kw)), None)
+
+
+res = {
+    "hq_not_multiple": ex(Hq=3),
+    "hkv_zero": ex(Hkv=0),
+    "d_96": ex(D=96),
+    "block_32": ex(block=32),
+    "ragged_S": ex(S=1000),
+    "negative_B": ex(B=-1),
+    "dtype_7": ex(dtype=7),
+    "rho_zero": ex(rho_min=0.0),
+    "rho_above_one": ex(rho_min=1.5),
+    "rho_nan": ex(rho_min=float("nan")),
+    "tau_zero": ex(tau=0.0),
+    "tau_inf": ex(tau=float("inf")),
+    "kmin_zero": ex(k_min=0),
+    "q_null": ex(q=None),
+    "out_null": ex(out=None),
+    "q_misaligned": ex(q=FAKE + 8),
+    "sel_idx_misaligned": ex(sel_idx=FAKE + 2),
+    "status_misaligned": ex(status=FAKE + 2),
+    "workspace_null": ex(workspace=None),
+    "workspace_small": ex(workspace_bytes=1024),
+    "workspace_misaligned": ex(workspace=FAKE + 16),
+    "nb_too_large": ex(S=(S.STEM_MAX_NB + 1) * 128),
+    "empty_B": ex(B=0, q=None, k=None, v=None, out=None, sel_idx=None, sel_cnt=None),
+    "empty_S": ex(S=0, q=None, k=None, v=None, out=None, sel_idx=None, sel_cnt=None),
+    "ex_null_args": L.stem_prefill_ex(None, None),
+    "host_null_args": L.stem_prefill_host(None),
+    "host_ragged": L.stem_prefill_host(ctypes.byref(base(S=1000))),
+    "simple_bad_block": L.stem_prefill(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 96, 0.25, 4.0, 2,
+                                       FAKE, FAKE, FAKE),
+    "simple_bad_rho": L.stem_prefill(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 128, -0.1, 4.0, 2,
+                                     FAKE, FAKE, FAKE),
+    "pool_bad_dtype": L.stem_pool(FAKE, FAKE, FAKE, 5, 1, 4, 2, 1024, 128, 128, FAKE, FAKE,
+                                  FAKE, None),
+    "pool_null_out": L.stem_pool(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, None, FAKE,
+                                 FAKE, None),
+    "pool_misaligned_qbar": L.stem_pool(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, FAKE + 4,
+                                        FAKE, FAKE, None),
+    "select_bad_kmin": L.stem_select(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, 0.25, 4.0, 0, FAKE,
+                                     FAKE, None, FAKE, 1 << 20, None),
+    "select_nb_too_large": L.stem_select(FAKE, FAKE, FAKE, 1, 4, 2, S.STEM_MAX_NB + 1, 128,
+                                         0.25, 4.0, 2, FAKE, FAKE, None, FAKE, 1 << 30, None),
+    "select_no_workspace": L.stem_select(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, 0.25, 4.0, 2, FAKE,
+                                         FAKE, None, None, 0, None),
+    "attn_bad_hq": L.stem_sparse_attn(FAKE, FAKE, FAKE, 0, 1, 5, 2, 1024, 128, 128, 0.25, 4.0,
+                                      2, FAKE, FAKE, FAKE, FAKE, 1 << 20, None, None),
+    "attn_small_workspace": L.stem_sparse_attn(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128,
+                                               0.25, 4.0, 2, FAKE, FAKE, FAKE, FAKE, 16, None,
+                                               None),
+    "budget_bad_tau": L.stem_budget(8, 0.5, -1.0, 2, None, None),
+    "capacity_bad_rho": L.stem_sel_capacity(8, 0.0, 4.0, 2),
+}
+print(json.dumps(res))

@@ -1,0 +1,186 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+Stage by stage (each stage fed the oracle's own upstream values, so a mismatch points at one
+kernel) and end to end, on seeded inputs at sizes the oracle finishes in seconds that span
+several tiles and ragged tile tails, plus the degenerate cases of the method.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_causal_pooling_b200 import stem as S
+from block_sparse_causal_pooling_b200 import workloads as wl
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+# (workload, note). Small shapes with the named workloads' value recipes.
+CASES = {
+    "tiny": wl.TINY,
+    "llama-4k": wl.LLAMA_32K.replace(name="llama-4k", Hq=8, Hkv=2, S=4096),
+    "llama-b2-2k": wl.LLAMA_32K.replace(name="llama-b2-2k", B=2, Hq=4, Hkv=1, S=2048,
+                                        rho_min=0.2, tau=4.0, k_min=3),
+    "qwen-3k": wl.QWEN_64K.replace(name="qwen-3k", Hq=7, Hkv=1, S=3072, tau=6.0),
+    "bf16-d64-blk64": wl.LLAMA_32K.replace(name="bf16-d64-blk64", Hq=4, Hkv=2, S=2560, D=64,
+                                           block=64, tau=8.0),
+    "bf16-d128-blk64": wl.LLAMA_32K.replace(name="bf16-d128-blk64", Hq=2, Hkv=2, S=2048,
+                                            block=64, tau=8.0),
+    "f32-d128-blk128": wl.TINY.replace(name="f32-d128-blk128", Hq=4, Hkv=2, S=2048, D=128,
+                                       block=128),
+    "kmin1": wl.LLAMA_32K.replace(name="kmin1", Hq=2, Hkv=1, S=4096, rho_min=0.01, tau=1.0,
+                                  k_min=1),
+    "dense": wl.LLAMA_32K.replace(name="dense", Hq=4, Hkv=2, S=2048, rho_min=1.0),
+    "nb37": wl.LLAMA_32K.replace(name="nb37", Hq=2, Hkv=2, S=37 * 128, tau=5.0),
+}
+
+
+def inputs(w, device=DEV):
+    q, k, v = wl.make_inputs(w, "cpu")
+    return (q, k, v), (q.to(device), k.to(device), v.to(device))
+
+
+def _oracle(w, cpu):
+    return oracle.prefill(*cpu, w.block, w.rho_min, w.tau, w.k_min)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_pool_parity(name):
+    w = CASES[name]
+    cpu, dev = inputs(w)
+    qbar, kbar, vnorm = S.stem_pool(*dev, w.block)
+    torch.cuda.synchronize()
+    rq, rk, rn = oracle.pool(*cpu, w.block)
+    # float32 pairwise sums of `block` rows: |error of a mean| <= log2(block)*u*max|x|
+    for got, ref, x in ((qbar, rq, cpu[0]), (kbar, rk, cpu[1])):
+        atol = 1e-6 * float(x.float().abs().max())
+        np.testing.assert_allclose(got.double().cpu().numpy(), ref, rtol=0, atol=atol)
+    np.testing.assert_allclose(vnorm.double().cpu().numpy(), rn, rtol=2e-6)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_select_parity_from_oracle_pooling(name):
+    """The selection kernel on the oracle's pooled values (rounded to float32) against the
+    oracle's selection from the same float32 values."""
+    w = CASES[name]
+    cpu, _ = inputs(w)
+    rq, rk, rn = oracle.pool(*cpu, w.block)
+    q32, k32, n32 = (torch.from_numpy(x).float() for x in (rq, rk, rn))
+    m = oracle.metric(q32.double().numpy(), k32.double().numpy(), n32.double().numpy())
+    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+    ref_idx, ref_cnt = oracle.select(m, kk, off)
+    sel_idx, sel_cnt, m_gpu = S.stem_select(q32.to(DEV), k32.to(DEV), n32.to(DEV), w.rho_min,
+                                            w.tau, w.k_min, with_metric=True)
+    torch.cuda.synchronize()
+    res = parity.compare_selection(sel_idx, sel_cnt, ref_idx, ref_cnt, m, kk, off)
+    assert not res["violations"], res["violations"][:5]
+    assert res["tie_swaps"] <= max(1, res["rows"] // 100), res
+    np.testing.assert_allclose(m_gpu.double().cpu().numpy(), m, rtol=2e-5, atol=1e-30)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attention_parity_on_oracle_selection(name):
+    w = CASES[name]
+    cpu, dev = inputs(w)
+    ref = _oracle(w, cpu)
+    sel_idx = torch.from_numpy(ref["sel_idx"]).to(DEV)
+    sel_cnt = torch.from_numpy(ref["sel_cnt"]).to(DEV)
+    out = S.stem_sparse_attn(*dev, w.block, w.rho_min, w.tau, w.k_min, sel_idx, sel_cnt)
+    torch.cuda.synchronize()
+    rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
+    parity.assert_out_close(parity.out_rows(out, rows, w.block), ref["out"], w.torch_dtype, name)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_end_to_end(name):
+    w = CASES[name]
+    cpu, dev = inputs(w)
+    ref = _oracle(w, cpu)
+    status = torch.full((1,), 7, dtype=torch.int32, device=DEV)
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(*dev, w.block, w.rho_min, w.tau, w.k_min,
+                                              status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    res = parity.compare_selection(sel_idx, sel_cnt, ref["sel_idx"], ref["sel_cnt"], ref["m"],
+                                   ref["k"], ref["off"])
+    assert not res["violations"], res["violations"][:5]
+    assert res["tie_swaps"] <= max(1, res["rows"] // 100), res
+    swapped = set(res["rows_bad"])
+    rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
+    keep = [t for t, r in enumerate(rows) if r not in swapped]
+    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
+    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, name)
+
+
+def test_dense_budget_matches_torch_sdpa():
+    """rho_min = 1 keeps every causal block: the path is dense causal attention."""
+    w = wl.LLAMA_32K.replace(Hq=8, Hkv=2, S=8192, rho_min=1.0)
+    _, (q, k, v) = inputs(w)
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(q, k, v, w.block, w.rho_min, w.tau, w.k_min)
+    G = w.Hq // w.Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.float(), k.float().repeat_interleave(G, 1), v.float().repeat_interleave(G, 1),
+        is_causal=True)
+    d = (out.float() - ref).abs()
+    assert float(d.max()) <= 2e-2 and float(d.mean()) <= 1e-3
+    kk, off = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
+    assert torch.equal(sel_cnt.cpu()[0, 0], kk)
+
+
+def test_deterministic_and_host_api():
+    w = CASES["llama-4k"]
+    cpu, dev = inputs(w)
+    a = S.stem_prefill_ex(*dev, w.block, w.rho_min, w.tau, w.k_min)
+    b = S.stem_prefill_ex(*dev, w.block, w.rho_min, w.tau, w.k_min)
+    c = S.stem_prefill(*dev, w.block, w.rho_min, w.tau, w.k_min)
+    torch.cuda.synchronize()
+    for x, y, z in zip(a, b, c):
+        assert torch.equal(x, y) and torch.equal(x, z)
+    hq, hk, hv = (t.pin_memory() for t in cpu)
+    out = torch.empty_like(hq).pin_memory()
+    si = torch.empty(a[1].shape, dtype=torch.int32).pin_memory()
+    sc = torch.empty(a[2].shape, dtype=torch.int32).pin_memory()
+    S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, out, si, sc)
+    assert torch.equal(out, a[0].cpu()) and torch.equal(si, a[1].cpu())
+    assert torch.equal(sc, a[2].cpu())
+
+
+def test_empty_and_single_block():
+    w = wl.LLAMA_32K.replace(Hq=2, Hkv=1, S=128)
+    cpu, dev = inputs(w)
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(*dev, w.block, w.rho_min, w.tau, w.k_min)
+    torch.cuda.synchronize()
+    ref = _oracle(w, cpu)
+    assert sel_idx.cpu()[:, :, :1].eq(0).all() and sel_cnt.cpu().eq(1).all()
+    parity.assert_out_close(parity.out_rows(out, [(0, 0, 0), (0, 1, 0)], 128), ref["out"],
+                            torch.bfloat16)
+    # empty problems: nothing to do, success
+    z = torch.empty((0, 2, 128, 128), dtype=torch.bfloat16, device=DEV)
+    lib = S.lib()
+    a = S.stem_args_t()
+    a.B, a.Hq, a.Hkv, a.S, a.D, a.block = 0, 2, 1, 128, 128, 128
+    a.rho_min, a.tau, a.k_min = 0.5, 4.0, 2
+    assert lib.stem_prefill_ex(S.ctypes.byref(a), None) == 0
+    a.B, a.S = 1, 0
+    assert lib.stem_prefill_ex(S.ctypes.byref(a), None) == 0
+    del z
+
+
+def test_all_equal_metric_takes_lowest_blocks():
+    """Q = 0 and every V row of norm 1: all metrics tie, the lowest block indices win."""
+    w = wl.LLAMA_32K.replace(Hq=4, Hkv=2, S=8192, rho_min=0.1, tau=8.0, k_min=4)
+    _, (q, k, v) = inputs(w)
+    q = torch.zeros_like(q)
+    v = torch.zeros_like(v)
+    v[..., 5] = 1.0
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(q, k, v, w.block, w.rho_min, w.tau, w.k_min)
+    torch.cuda.synchronize()
+    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+    si = sel_idx.cpu().numpy()
+    for h in range(w.Hq):
+        for i in range(w.nb):
+            want = [0] if i == 0 else sorted(set([0, i] + list(range(1, kk[i] - 1))))
+            assert si[0, h, off[i]:off[i + 1]].tolist() == want
