@@ -206,6 +206,39 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ GPU path
 
 
+class RawEvents:
+    """cudaEvent_t handles through the CUDA runtime torch already loaded. The library records
+    them itself (inside stem_prefill_ex), which torch.cuda.Event does not track."""
+
+    def __init__(self):
+        import ctypes
+
+        self.ct = ctypes
+        self.rt = ctypes.CDLL("libcudart.so.12")
+        self.made = []
+
+    def create(self) -> int:
+        ev = self.ct.c_void_p()
+        rc = self.rt.cudaEventCreate(self.ct.byref(ev))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventCreate failed ({rc})")
+        self.made.append(ev.value)
+        return ev.value
+
+    def elapsed_ms(self, a: int, b: int) -> float:
+        ms = self.ct.c_float()
+        rc = self.rt.cudaEventElapsedTime(self.ct.byref(ms), self.ct.c_void_p(a),
+                                          self.ct.c_void_p(b))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+        return ms.value
+
+    def destroy(self):
+        for e in self.made:
+            self.rt.cudaEventDestroy(self.ct.c_void_p(e))
+        self.made = []
+
+
 def config_of(w):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
             "block": w.block, "rho_min": w.rho_min, "tau": w.tau, "k_min": w.k_min,
@@ -228,7 +261,8 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     K, W = args.steps, args.warmup
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    raw = RawEvents()
+    ev = [[raw.create() for _ in range(4)] for _ in range(K)]
     args_warm = S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
                             ws)
     call_args = [S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
@@ -261,9 +295,10 @@ def run_ours(args, world, rank, local):
     stage_ms = {"pool": [], "select": [], "attn": []}
     for s in range(K):
         e = ev[s]
-        stage_ms["pool"].append(e[0].elapsed_time(e[1]))
-        stage_ms["select"].append(e[1].elapsed_time(e[2]))
-        stage_ms["attn"].append(e[2].elapsed_time(e[3]))
+        stage_ms["pool"].append(raw.elapsed_ms(e[0], e[1]))
+        stage_ms["select"].append(raw.elapsed_ms(e[1], e[2]))
+        stage_ms["attn"].append(raw.elapsed_ms(e[2], e[3]))
+    raw.destroy()
     ms = total_ms / K
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)

@@ -175,8 +175,9 @@ def make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, worksp
         a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
     if status is not None:
         a.status = status.data_ptr()
-    if events is not None:  # 4 torch.cuda.Event (already created with timing enabled)
-        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    if events is not None:  # 4 cudaEvent_t handles (ints) or torch.cuda.Event objects
+        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(getattr(e, "cuda_event", e))
+                                      for e in events])
         a._events_keepalive = arr
         a.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
     return a
