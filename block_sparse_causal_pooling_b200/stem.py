@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "stem_pool": (I, [P, P, P, I, I, I, I, I, I, I, P, P, P, P]),
         "stem_select": (I, [P, P, P, I, I, I, I, I, F, F, I, P, P, P, P, Z, P]),
         "stem_sparse_attn": (I, [P, P, P, I, I, I, I, I, I, I, F, F, I, P, P, P, P, Z, P, P]),
+        "stem_select_static": (I, [P, P, P, I, I, I, I, I, F, F, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -80,7 +81,7 @@ _lib = _load()
 # Every symbol include/stem.h declares.
 EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget",
             "stem_sel_capacity", "stem_workspace_size", "stem_strerror", "stem_pool",
-            "stem_select", "stem_sparse_attn")
+            "stem_select", "stem_sparse_attn", "stem_select_static")
 
 
 def lib() -> ctypes.CDLL:
@@ -265,3 +266,20 @@ def stem_sparse_attn(q, k, v, block, rho_min, tau, k_min, sel_idx, sel_cnt, out=
                                  workspace.numel(), _ptr(status), _stream(stream)),
            "stem_sparse_attn")
     return out
+
+
+def stem_select_static(qbar, kbar, vnorm, rho_min, tau, k_min, sel_idx=None, sel_cnt=None,
+                       stream=None):
+    """stem_select without a workspace or any device allocation by the library: its scratch
+    (the budget plan) sits in a fixed device array inside libstem.so. For callers that cannot
+    allocate device memory. Calls that overlap on the GPU race on that array."""
+    B, Hq, nb, D = qbar.shape
+    Hkv = kbar.shape[1]
+    if sel_idx is None:
+        cap = stem_sel_capacity(nb, rho_min, tau, k_min)
+        sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=qbar.device)
+        sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=qbar.device)
+    _check(_lib.stem_select_static(qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(), B, Hq,
+                                   Hkv, nb, D, rho_min, tau, k_min, sel_idx.data_ptr(),
+                                   sel_cnt.data_ptr(), _stream(stream)), "stem_select_static")
+    return sel_idx, sel_cnt

@@ -177,6 +177,24 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
                      const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
                      size_t workspace_bytes, int32_t* status, void* stream);
 
+/*
+ * stem_select_static: stem_select for callers that cannot allocate device memory. The paper
+ * has no counterpart; this is an interface addition.
+ *
+ * Some callers cannot call cudaMalloc or hand this library a workspace (a host application
+ * that owns every device allocation through its own budgeted allocator, a plugin that may not
+ * allocate behind that allocator's back). This entry point allocates nothing: the selection
+ * kernel's scratch, the budget plan (3*nb+1 int32), lives in a 64 KiB file-scope device array
+ * that every GPU loading the library holds until the process exits. Inputs and outputs are
+ * those of stem_select (no m_out). nb beyond STEM_MAX_NB returns STEM_ERR_UNSUPPORTED.
+ * The first call on a device looks the array up (with that device current); make it before
+ * any stream capture. All calls share the array: calls whose kernels overlap on the GPU race,
+ * so issue them in stream order. Same errors as stem_select, except that there is no workspace.
+ */
+int stem_select_static(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                       int Hkv, int nb, int D, float rho_min, float tau, int k_min,
+                       int32_t* sel_idx, int32_t* sel_cnt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -88,6 +88,12 @@ res = {
                                                0.25, 4.0, 2, FAKE, FAKE, FAKE, FAKE, 16, None,
                                                None),
     "budget_bad_tau": L.stem_budget(8, 0.5, -1.0, 2, None, None),
+    "static_bad_kmin": L.stem_select_static(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, 0.25, 4.0, 0,
+                                            FAKE, FAKE, None),
+    "static_nb_too_large": L.stem_select_static(FAKE, FAKE, FAKE, 1, 4, 2, S.STEM_MAX_NB + 1,
+                                                128, 0.25, 4.0, 2, FAKE, FAKE, None),
+    "static_null_out": L.stem_select_static(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, 0.25, 4.0, 2,
+                                            None, FAKE, None),
     "capacity_bad_rho": L.stem_sel_capacity(8, 0.0, 4.0, 2),
 }
 print(json.dumps(res))

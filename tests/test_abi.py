@@ -81,6 +81,7 @@ def test_argument_validation_rejects_before_any_device_work():
         "attn_small_workspace": S.STEM_ERR_WORKSPACE,
         "nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "select_nb_too_large": S.STEM_ERR_UNSUPPORTED,
+        "static_nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "empty_B": S.STEM_OK,
         "empty_S": S.STEM_OK,
     })
