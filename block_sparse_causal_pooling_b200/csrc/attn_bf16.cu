@@ -274,10 +274,10 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, int B, int
 
 }  // namespace
 
-cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
-                             int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
-                             const int32_t* sel_idx, const int32_t*, void* out, int32_t*,
-                             cudaStream_t st) {
+// mma.sync path: block = 64 (the tcgen05 kernel in attn_sm100.cu covers block = 128).
+cudaError_t launch_attn_bf16_mma(const void* q, const void* k, const void* v, int B, int Hq,
+                                 int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
+                                 const int32_t* sel_idx, void* out, cudaStream_t st) {
   if (D == 128 && block == 128)
     return launch_typed<128, 128>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, out, st);
   if (D == 128 && block == 64)

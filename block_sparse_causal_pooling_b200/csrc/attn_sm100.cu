@@ -1,0 +1,599 @@
+// Block-sparse causal attention on the Blackwell tensor cores (tcgen05 + TMEM + TMA), bf16 in,
+// fp32 accumulation, block = 128.
+//
+// Computes, for every query token of query block i, exact softmax attention over every token of
+// the kept key blocks of row (b, h, i), token-causal inside block i ("Stem: Rethinking Causal
+// Information Flow in Sparse Attention", gist.science/es "Resumen tecnico" 2 "Implementacion"
+// step 3; gist.science/it 2.C step 3; gist.science/nl "Implementatie" step 3; gist.science/fr
+// 2.C step 3).
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: Q tile (double-buffered) and K/V tiles of the kept blocks into a
+//               4-slot ring of 32 KB shared-memory tiles (128B-swizzled boxes of 128 x 64).
+//   warp 1      allocates 512 TMEM columns; lane 0 issues every tcgen05.mma:
+//                 S[g%2] = Q K^T           (M 128, N 128, K = D; A and B K-major in smem)
+//                 O[n%2] += P V            (A = P read from TMEM, B = V MN-major in smem)
+//               S is double-buffered so S of the next key block runs while the softmax works on
+//               the current one; O is double-buffered across work items so the epilogue of one
+//               item overlaps the next item's products.
+//   warps 2-5   softmax, one query row per thread (tcgen05.ld 32x32b): row max, exp2 with the
+//               1/sqrt(D) scale folded in, row sum in fp32; P packed to bf16 and stored over the
+//               first half of its S buffer (tcgen05.st); O rescaled in TMEM only when the running
+//               max grows by more than 2^8 (exact: the final 1/l uses the same reference max).
+//               Then the epilogue: O * (1/l) -> bf16 -> global.
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+//
+// Synchronisation is by mbarriers only. Every wait is bounded by the global nanosecond timer: on
+// expiry the CTA records STEM_ERR_TIMEOUT in the status word, every role leaves its loop, the
+// MMA thread drains its issued products, the producer drains its issued copies (both bounded),
+// TMEM is freed and the kernel returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "stem.h"
+#include "stem_internal.h"
+
+namespace stem {
+
+cudaError_t launch_attn_bf16_mma(const void* q, const void* k, const void* v, int B, int Hq,
+                                 int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
+                                 const int32_t* sel_idx, void* out, cudaStream_t st);
+
+namespace {
+
+constexpr int kM = 128;             // query rows per tile (= block)
+constexpr int kN = 128;             // keys per kept block
+constexpr int kSlots = 4;           // K/V ring slots
+constexpr int kThreads = 192;       // 6 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+
+template <int D>
+struct Cfg {
+  static constexpr uint32_t kTile = kM * D * 2;  // bytes of a 128 x D bf16 tile
+  static constexpr int kBoxes = D / 64;          // 128B-swizzled boxes of 64 columns
+  static constexpr int kKSteps = D / 16;         // MMA k-steps of QK^T
+};
+
+struct __align__(8) Bars {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[kSlots], kv_empty[kSlots];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full[2], o_empty[2];
+  uint64_t pv_done, drain;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity` of barrier b. Returns false (after recording
+// the timeout) if it expired or another role already aborted.
+__device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bars, int32_t* status) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = gtimer();
+  while (true) {
+    if (mbar_try(b, parity)) return true;
+    if (bars->abort) return false;
+    if (gtimer() - t0 > kWaitNs) {
+      bars->abort = 1;
+      if (status) atomicExch(status, STEM_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Bounded drain wait used on the abort path only (ignores the abort flag).
+__device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = gtimer();
+  while (!mbar_try(b, parity) && gtimer() - t0 < kWaitNs) {
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* b) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          su32(b))
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+#define TC_LD32(taddr, r)                                                                     \
+  asm volatile(                                                                               \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13," \
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"      \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),   \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),            \
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),         \
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),         \
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),         \
+        "=r"(r[31])                                                                           \
+      : "r"(taddr))
+
+#define TC_ST32(taddr, r)                                                                     \
+  asm volatile(                                                                               \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12," \
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"     \
+      ::"r"(taddr),                                                                           \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),       \
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),     \
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),     \
+      "r"(r[29]), "r"(r[30]), "r"(r[31])                                                      \
+      : "memory")
+
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Shared-memory matrix descriptor, 128B swizzle (sm_100 format: version 1 at bits 46-47,
+// layout type 2 at bits 61-63). Offsets in bytes.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3fff);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3fff) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, A K-major, B K- or MN-major.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(b_mn_major) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Work item t -> (b, g, h, i): kv-head-group-major, query blocks in the plan's heavy-first
+// order, the G heads of a group adjacent.
+struct Item {
+  int b, g, h, i;
+};
+__device__ __forceinline__ Item decode(int64_t t, int G, int nb, int Hkv, const int32_t* order) {
+  const int64_t per_group = static_cast<int64_t>(G) * nb;
+  const int64_t bg = t / per_group;
+  const int rem = static_cast<int>(t % per_group);
+  Item it;
+  it.i = order[rem / G];
+  it.b = static_cast<int>(bg / Hkv);
+  it.g = static_cast<int>(bg % Hkv);
+  it.h = it.g * G + rem % G;
+  return it;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, int Hq, int Hkv, int S, int nb,
+                      int64_t items, PlanDev plan, int64_t cap,
+                      const int32_t* __restrict__ sel_idx, __nv_bfloat16* __restrict__ out,
+                      int32_t* status) {
+  using C = Cfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* q_tiles = smem;                       // [2][kTile]
+  unsigned char* kv_tiles = smem + 2 * C::kTile;       // [kSlots][kTile]
+  Bars* bars = reinterpret_cast<Bars*>(kv_tiles + kSlots * C::kTile);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = Hq / Hkv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->o_full[s], 1);
+      mbar_init(&bars->o_empty[s], 128);
+    }
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // TMEM allocation (warp-wide)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(&bars->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)));
+      int64_t f = 0;  // K/V fills issued
+      int n = 0;      // items of this CTA
+      int64_t slot_round[kSlots];
+      for (int s = 0; s < kSlots; ++s) slot_round[s] = -1;
+      int64_t q_round[2] = {-1, -1};
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
+        const Item it = decode(t, G, nb, Hkv, plan.order);
+        const int64_t bh = static_cast<int64_t>(it.b) * Hq + it.h;
+        const int qs = n & 1;
+        if (!(ok = wait_bar(&bars->q_empty[qs], ((n >> 1) & 1) ^ 1, bars, status))) break;
+        mbar_expect_tx(&bars->q_full[qs], C::kTile);
+        const int qrow = static_cast<int>(bh * S + static_cast<int64_t>(it.i) * kM);
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_2d(q_tiles + qs * C::kTile + x * (kM * 128), &tm_q, x * 64, qrow,
+                      &bars->q_full[qs]);
+        q_round[qs] = n >> 1;
+        const int cnt = plan.k[it.i];
+        const int32_t* list = sel_idx + bh * cap + plan.off[it.i];
+        const int kvrow0 = static_cast<int>((static_cast<int64_t>(it.b) * Hkv + it.g) * S);
+        for (int j = 0; j < cnt && ok; ++j) {
+          const int blk = min(max(list[j], 0), it.i);
+          for (int which = 0; which < 2; ++which, ++f) {
+            const int s = static_cast<int>(f % kSlots);
+            const int64_t r = f / kSlots;
+            if (!(ok = wait_bar(&bars->kv_empty[s], static_cast<uint32_t>((r & 1) ^ 1), bars,
+                                status)))
+              break;
+            mbar_expect_tx(&bars->kv_full[s], C::kTile);
+            const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_2d(kv_tiles + s * C::kTile + x * (kN * 128), map, x * 64,
+                          kvrow0 + blk * kN, &bars->kv_full[s]);
+            slot_round[s] = r;
+          }
+        }
+      }
+      if (!ok) {  // abort: let issued copies land before the CTA can exit
+        for (int s = 0; s < kSlots; ++s)
+          if (slot_round[s] >= 0) drain_bar(&bars->kv_full[s], slot_round[s] & 1);
+        for (int s = 0; s < 2; ++s)
+          if (q_round[s] >= 0) drain_bar(&bars->q_full[s], q_round[s] & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = instr_desc(kM, kN, false);
+      constexpr uint32_t idesc_o = instr_desc(kM, D, true);
+      const uint32_t tm_s[2] = {tmem, tmem + 128};
+      const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
+      const uint32_t q_base = su32(q_tiles), kv_base = su32(kv_tiles);
+      struct Pv {
+        int64_t g, fv;
+        int n;
+        bool first, last;
+      } prev{-1, 0, 0, false, false};
+      bool have_prev = false, ok = true;
+      int64_t g = 0, fbase = 0;
+      int n = 0;
+      auto issue_pv = [&](const Pv& p) -> bool {
+        const int ob = p.n & 1;
+        if (p.first && !wait_bar(&bars->o_empty[ob], ((p.n >> 1) & 1) ^ 1, bars, status))
+          return false;
+        if (!wait_bar(&bars->p_full[p.g & 1], static_cast<uint32_t>((p.g >> 1) & 1), bars,
+                      status))
+          return false;
+        const int sv = static_cast<int>(p.fv % kSlots);
+        if (!wait_bar(&bars->kv_full[sv], static_cast<uint32_t>((p.fv / kSlots) & 1), bars,
+                      status))
+          return false;
+        tc_fence_after();
+        const uint32_t vaddr = kv_base + sv * C::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          // B = V rows kk*16 .. +15 (keys), MN-major: 64-column boxes kN*128 bytes apart
+          const uint64_t bd = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
+          mma_ts(tm_o[ob], tm_s[p.g & 1] + kk * 8, bd, idesc_o, (p.first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(&bars->kv_empty[sv]);
+        tc_commit(&bars->pv_done);
+        if (p.last) tc_commit(&bars->o_full[ob]);
+        return true;
+      };
+      for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
+        const Item it = decode(t, G, nb, Hkv, plan.order);
+        const int qs = n & 1;
+        const int cnt = plan.k[it.i];
+        if (!(ok = wait_bar(&bars->q_full[qs], (n >> 1) & 1, bars, status))) break;
+        for (int j = 0; j < cnt; ++j, ++g) {
+          const int64_t fk = fbase + 2 * j;
+          const int sk = static_cast<int>(fk % kSlots);
+          if (!(ok = wait_bar(&bars->kv_full[sk], static_cast<uint32_t>((fk / kSlots) & 1), bars,
+                              status)))
+            break;
+          tc_fence_after();
+          const uint32_t qa = q_base + qs * C::kTile, ka = kv_base + sk * C::kTile;
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
+            mma_ss(tm_s[g & 1], smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
+                   idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars->kv_empty[sk]);
+          tc_commit(&bars->s_full[g & 1]);
+          if (j == cnt - 1) tc_commit(&bars->q_empty[qs]);
+          if (have_prev && !(ok = issue_pv(prev))) break;
+          prev = Pv{g, fk + 1, n, j == 0, j == cnt - 1};
+          have_prev = true;
+        }
+        fbase += 2 * static_cast<int64_t>(cnt);
+      }
+      if (ok && have_prev) ok = issue_pv(prev);
+      // make sure every issued product has completed before TMEM is released
+      tc_commit(&bars->drain);
+      drain_bar(&bars->drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int sub = warp & 3;           // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;    // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(D));
+    int64_t g = 0;
+    int n = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
+      const Item it = decode(t, G, nb, Hkv, plan.order);
+      const int64_t bh = static_cast<int64_t>(it.b) * Hq + it.h;
+      const int cnt = plan.k[it.i];
+      const int32_t* list = sel_idx + bh * cap + plan.off[it.i];
+      const int ob = n & 1;
+      const uint32_t o_addr = tmem + 256 + ob * 128 + lane_off;
+      float m_run = 0.f, l = 0.f;
+      for (int j = 0; j < cnt; ++j, ++g) {
+        const int sb = static_cast<int>(g & 1);
+        ok = wait_bar(&bars->s_full[sb], static_cast<uint32_t>((g >> 1) & 1), bars, status);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before tcgen05.ld
+        tc_fence_after();
+        const uint32_t s_addr = tmem + sb * 128 + lane_off;
+        uint32_t sr[kN];
+#pragma unroll
+        for (int c = 0; c < kN / 32; ++c) TC_LD32(s_addr + 32 * c, (sr + 32 * c));
+        tc_wait_ld();
+        const bool diag = min(max(list[j], 0), it.i) == it.i;
+        if (diag) {  // token-causal inside the query's own block
+#pragma unroll
+          for (int c = 0; c < kN; ++c)
+            if (c > row) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
+#pragma unroll
+        for (int c = 8; c < kN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
+        const float mt =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+        if (j == 0) {
+          m_run = mt;
+        } else if (__any_sync(0xffffffffu, mt > m_run + 8.0f)) {
+          // some row's max grew by more than 2^8: the whole warp rescales its rows of O (each
+          // by its own factor, 1 where the max did not grow); PV of the previous block first
+          const float m_new = fmaxf(m_run, mt);
+          const float alpha = ex2(m_run - m_new);
+          m_run = m_new;
+          l *= alpha;
+          ok = wait_bar(&bars->pv_done, static_cast<uint32_t>((g - 1) & 1), bars, status);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            TC_LD32(o_addr + 32 * c, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            TC_ST32(o_addr + 32 * c, o);
+          }
+          tc_wait_st();
+        }
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t p[kN / 2];
+#pragma unroll
+        for (int c = 0; c < kN / 2; ++c) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_run));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_run));
+          sum[c & 3] += p0 + p1;
+          p[c] = pack_bf16(p0, p1);
+        }
+        l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        TC_ST32(s_addr, p);
+        TC_ST32(s_addr + 32, (p + 32));
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[sb]);
+      }
+      if (!ok) break;
+      // epilogue
+      ok = wait_bar(&bars->o_full[ob], (n >> 1) & 1, bars, status);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      __nv_bfloat16* dst = out + (bh * S + static_cast<int64_t>(it.i) * kM + row) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        TC_LD32(o_addr + 32 * c, o);
+        tc_wait_ld();
+        uint4 pk[4];
+        uint32_t* w = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d4[e] = pk[e];
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty[ob]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D view [rows, D] of a bf16 tensor, boxes of 64 columns x 128 rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                         int S, PlanDev plan, int64_t cap, const int32_t* sel_idx, void* out,
+                         int32_t* status, cudaStream_t st) {
+  const int nb = S / kM;
+  const int64_t items = static_cast<int64_t>(B) * Hq * nb;
+  if (items == 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, static_cast<uint64_t>(B) * Hq * S, D) ||
+      !make_map(&tk, k, static_cast<uint64_t>(B) * Hkv * S, D) ||
+      !make_map(&tv, v, static_cast<uint64_t>(B) * Hkv * S, D))
+    return cudaErrorInvalidValue;
+  // one CTA per SM: each CTA takes all 512 TMEM columns
+  const size_t smem = std::max<size_t>(1024 + (2 + kSlots) * Cfg<D>::kTile + sizeof(Bars),
+                                       120 * 1024);
+  auto kern = attn_sm100_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(items, sm_count());
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, Hq, Hkv, S, nb, items,
+                                                           plan, cap, sel_idx,
+                                                           static_cast<__nv_bfloat16*>(out),
+                                                           status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
+                             int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
+                             const int32_t* sel_idx, const int32_t*, void* out, int32_t* status,
+                             cudaStream_t st) {
+  if (block == 128 && D == 128)
+    return launch_sm100<128>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, out, status, st);
+  if (block == 128 && D == 64)
+    return launch_sm100<64>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, out, status, st);
+  return launch_attn_bf16_mma(q, k, v, B, Hq, Hkv, S, D, block, plan, cap, sel_idx, out, st);
+}
+
+}  // namespace stem
