@@ -98,7 +98,8 @@ const Plan* get_plan(int nb, float rho_min, float tau, int k_min) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Layout {
-  size_t status = 0, plan = 0, qbar = 0, kbar = 0, vnorm = 0, total = 0;
+  size_t status = 0, plan = 0, sched = 0, sched_end = 0, qbar = 0, kbar = 0, vnorm = 0,
+         total = 0;
 };
 
 Layout layout(int B, int Hq, int Hkv, int nb, int D) {
@@ -108,6 +109,9 @@ Layout layout(int B, int Hq, int Hkv, int nb, int D) {
   o += kAlign;
   L.plan = o;
   o += plan_bytes(nb);
+  L.sched = o;
+  o += align_up(pairs_bytes(B, Hq, Hkv, nb));
+  L.sched_end = o;
   L.qbar = o;
   o += align_up(sizeof(float) * static_cast<size_t>(B) * Hq * nb * D);
   L.kbar = o;
@@ -210,7 +214,9 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   if ((rc = mark(2)) != STEM_OK) return rc;
   if (a->dtype == STEM_BF16) {
     rc = cuda_err(launch_attn_bf16(a->q, a->k, a->v, a->B, a->Hq, a->Hkv, a->S, a->D, a->block,
-                                   pd, plan->cap, a->sel_idx, a->sel_cnt, a->out, a->status, st));
+                                   pd, plan->cap, a->sel_idx, a->sel_cnt,
+                                   reinterpret_cast<uint32_t*>(ws + L.sched), a->out, a->status,
+                                   st));
   } else {
     rc = cuda_err(launch_attn_f32(static_cast<const float*>(a->q),
                                   static_cast<const float*>(a->k),
@@ -467,7 +473,7 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
       !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) || !aligned(status, 4))
     return STEM_ERR_ARG;
   const Layout L = layout(B, Hq, Hkv, nb, D);
-  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.plan + plan_bytes(nb))
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.sched_end)
     return STEM_ERR_WORKSPACE;
   const Plan* plan = get_plan(nb, rho_min, tau, k_min);
   if (plan == nullptr) return STEM_ERR_CUDA;
@@ -481,7 +487,10 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
   if (rc != STEM_OK) return rc;
   if (dtype == STEM_BF16)
     return cuda_err(launch_attn_bf16(q, k, v, B, Hq, Hkv, S, D, block, pd, plan->cap, sel_idx,
-                                     sel_cnt, out, status, st));
+                                     sel_cnt,
+                                     reinterpret_cast<uint32_t*>(
+                                         static_cast<unsigned char*>(workspace) + L.sched),
+                                     out, status, st));
   return cuda_err(launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                   static_cast<const float*>(v), B, Hq, Hkv, S, D, block, pd,
                                   plan->cap, sel_idx, sel_cnt, static_cast<float*>(out), st));

@@ -7,7 +7,7 @@
 // step 3; gist.science/it 2.C step 3; gist.science/nl "Implementatie" step 3; gist.science/fr
 // 2.C step 3).
 //
-// Persistent kernel, one CTA per SM, 6 warps:
+// Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: Q tile (double-buffered) and K/V tiles of the kept blocks into a
 //               4-slot ring of 32 KB shared-memory tiles (128B-swizzled boxes of 128 x 64).
 //   warp 1      allocates 512 TMEM columns; lane 0 issues every tcgen05.mma:
@@ -16,11 +16,13 @@
 //               S is double-buffered so S of the next key block runs while the softmax works on
 //               the current one; O is double-buffered across work items so the epilogue of one
 //               item overlaps the next item's products.
-//   warps 2-5   softmax, one query row per thread (tcgen05.ld 32x32b): row max, exp2 with the
-//               1/sqrt(D) scale folded in, row sum in fp32; P packed to bf16 and stored over the
-//               first half of its S buffer (tcgen05.st); O rescaled in TMEM only when the running
-//               max grows by more than 2^8 (exact: the final 1/l uses the same reference max).
-//               Then the epilogue: O * (1/l) -> bf16 -> global.
+//   warps 2-9   softmax, two threads per query row (warps w and w+4 share TMEM lanes
+//               32*(w%4).. and take 64 columns each; tcgen05.ld 32x32b): row max (halves
+//               exchanged through shared memory under a per-pair named barrier), exp2 with the
+//               1/sqrt(D) scale folded in, per-thread partial row sums in fp32; P packed to bf16
+//               and stored over the first half of its S buffer (tcgen05.st); O rescaled in TMEM
+//               only when the running max grows by more than 2^8 (exact: the final 1/l uses the
+//               same reference max). Then the epilogue: O * (1/l) -> bf16 -> global.
 // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 //
 // Synchronisation is by mbarriers only. Every wait is bounded by the global nanosecond timer: on
@@ -49,7 +51,8 @@ namespace {
 constexpr int kM = 128;             // query rows per tile (= block)
 constexpr int kN = 128;             // keys per kept block
 constexpr int kSlots = 4;           // K/V ring slots
-constexpr int kThreads = 192;       // 6 warps
+constexpr int kThreads = 320;       // 10 warps
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
@@ -61,13 +64,15 @@ struct Cfg {
 };
 
 struct __align__(8) Bars {
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2];            // per tile (A, B)
   uint64_t kv_full[kSlots], kv_empty[kSlots];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_full[2], o_empty[2];
-  uint64_t pv_done, drain;
+  uint64_t s_full[2], p_full[2];             // per tile
+  uint64_t o_full[2], o_empty[2];            // per tile
+  uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
+  float xch[2][2][kM];  // [parity][half][row] partial row maxima of the two halves
+  float xl[2][2][kM];   // [tile][half][row] partial row sums (epilogue)
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -105,8 +110,8 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 
 // Bounded wait for the phase of parity `parity` of barrier b. Returns false (after recording
 // the timeout) if it expired or another role already aborted.
-__device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bars, int32_t* status) {
-  if (mbar_try(b, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, Bars* bars,
+                                           int32_t* status) {
   const uint64_t t0 = gtimer();
   while (true) {
     if (mbar_try(b, parity)) return true;
@@ -118,6 +123,13 @@ __device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bars, 
     }
   }
 }
+__device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bars,
+                                         int32_t* status) {
+  return mbar_try(b, parity) || wait_bar_slow(b, parity, bars, status);
+}
+__device__ __forceinline__ void pair_sync(int id) {  // the two warps that share TMEM lanes
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
 // Bounded drain wait used on the abort path only (ignores the abort flag).
 __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
   const uint64_t t0 = gtimer();
@@ -126,12 +138,22 @@ __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar)), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -222,22 +244,90 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major)
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Work item t -> (b, g, h, i): kv-head-group-major, query blocks in the plan's heavy-first
-// order, the G heads of a group adjacent.
+// Work item t -> (b, g, i, head pair): kv-head-group-major, query blocks in the plan's
+// heavy-first order, the ceil(G/2) head pairs of a group adjacent. Tile A is head g*G + 2p,
+// tile B head g*G + 2p + 1 (absent when G is odd and this is the group's last pair).
 struct Item {
-  int b, g, h, i;
+  int b, g, p, i, hA, hB;  // hB < 0: single tile
 };
 __device__ __forceinline__ Item decode(int64_t t, int G, int nb, int Hkv, const int32_t* order) {
-  const int64_t per_group = static_cast<int64_t>(G) * nb;
+  const int P = (G + 1) >> 1;
+  const int64_t per_group = static_cast<int64_t>(P) * nb;
   const int64_t bg = t / per_group;
   const int rem = static_cast<int>(t % per_group);
   Item it;
-  it.i = order[rem / G];
+  it.i = order[rem / P];
   it.b = static_cast<int>(bg / Hkv);
   it.g = static_cast<int>(bg % Hkv);
-  it.h = it.g * G + rem % G;
+  it.p = rem % P;
+  it.hA = it.g * G + 2 * it.p;
+  it.hB = (2 * it.p + 1 < G) ? it.hA + 1 : -1;
   return it;
 }
+
+// The k(i) steps of a head pair come from the schedule written by the pairing kernel: entry t
+// is blockA | blockB << 16 (blockB 0xFFFF: no head B). Shared blocks first, then lone pairs;
+// online softmax does not depend on the order of a row's blocks, and the diagonal is recognised
+// by its index. Indices are clamped to [0, i], so no entry can send a load outside the head.
+__device__ __forceinline__ const uint32_t* sched_row(const uint32_t* sched, const Item& it,
+                                                     int Hkv, int G, int64_t cap,
+                                                     const PlanDev& plan) {
+  const int P = (G + 1) >> 1;
+  const int64_t gp = (static_cast<int64_t>(it.b) * Hkv + it.g) * P + it.p;
+  return sched + gp * cap + plan.off[it.i];
+}
+__device__ __forceinline__ void sched_step(uint32_t e, int i, int& ba, int& bb) {
+  ba = min(static_cast<int>(e & 0xFFFFu), i);
+  const uint32_t hb = e >> 16;
+  bb = hb == 0xFFFFu ? -1 : min(static_cast<int>(hb), i);
+}
+
+// Global step sequence of one CTA: its work items (stride gridDim.x) and, inside each, the k(i)
+// steps of the head pair's schedule. Producer and MMA thread walk the same sequence with one step of
+// lookahead; the softmax warps walk it item by item.
+struct Step {
+  int n;  // item count of this CTA so far
+  bool first, last;
+  Item it;
+  int ba, bb;  // key blocks of tiles A and B (bb < 0: no tile B)
+  __device__ __forceinline__ bool has_b() const { return it.hB >= 0; }
+  __device__ __forceinline__ bool shared() const { return bb == ba; }
+};
+struct Seq {
+  int64_t t, items;
+  int G, nb, Hkv, Hq;
+  int64_t cap;
+  PlanDev plan;
+  const uint32_t* sched;
+  int n, j, cnt;
+  Item it;
+  const uint32_t* row;
+  __device__ __forceinline__ void init(int64_t items_, int G_, int nb_, int Hkv_, int Hq_,
+                                       int64_t cap_, PlanDev plan_, const uint32_t* sched_) {
+    t = blockIdx.x;
+    items = items_; G = G_; nb = nb_; Hkv = Hkv_; Hq = Hq_; cap = cap_; plan = plan_;
+    sched = sched_;
+    n = -1; j = 0; cnt = 0;
+  }
+  __device__ __forceinline__ bool next(Step& s) {
+    if (j >= cnt) {
+      if (n >= 0) t += gridDim.x;
+      if (t >= items) return false;
+      ++n;
+      it = decode(t, G, nb, Hkv, plan.order);
+      cnt = plan.k[it.i];
+      j = 0;
+      row = sched_row(sched, it, Hkv, G, cap, plan);
+    }
+    s.n = n;
+    s.first = (j == 0);
+    s.last = (j == cnt - 1);
+    s.it = it;
+    sched_step(row[j], it.i, s.ba, s.bb);
+    ++j;
+    return true;
+  }
+};
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -245,14 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, int Hq, int Hkv, int S, int nb,
                       int64_t items, PlanDev plan, int64_t cap,
-                      const int32_t* __restrict__ sel_idx, __nv_bfloat16* __restrict__ out,
+                      const uint32_t* __restrict__ sched, __nv_bfloat16* __restrict__ out,
                       int32_t* status) {
   using C = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* q_tiles = smem;                       // [2][kTile]
-  unsigned char* kv_tiles = smem + 2 * C::kTile;       // [kSlots][kTile]
+  unsigned char* q_tiles = smem;                   // [tile A, tile B][kTile]
+  unsigned char* kv_tiles = smem + 2 * C::kTile;   // [kSlots][kTile]
   Bars* bars = reinterpret_cast<Bars*>(kv_tiles + kSlots * C::kTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,15 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->p_full[s], kSoftmaxThreads);
       mbar_init(&bars->o_full[s], 1);
-      mbar_init(&bars->o_empty[s], 128);
+      mbar_init(&bars->o_empty[s], kSoftmaxThreads);
     }
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -293,48 +382,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)));
-      int64_t f = 0;  // K/V fills issued
-      int n = 0;      // items of this CTA
+      const uint64_t pol_kv = policy_evict_last(), pol_q = policy_evict_first();
+      // The ring is filled in the order the MMA thread first uses tiles: for step c with
+      // lookahead x: V(c, A), K(x, A), V(c, B), K(x, B); a block both heads keep is one tile.
+      int64_t f = 0;
       int64_t slot_round[kSlots];
       for (int s = 0; s < kSlots; ++s) slot_round[s] = -1;
-      int64_t q_round[2] = {-1, -1};
+      int64_t q_loads[2] = {0, 0};
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
-        const Item it = decode(t, G, nb, Hkv, plan.order);
-        const int64_t bh = static_cast<int64_t>(it.b) * Hq + it.h;
-        const int qs = n & 1;
-        if (!(ok = wait_bar(&bars->q_empty[qs], ((n >> 1) & 1) ^ 1, bars, status))) break;
-        mbar_expect_tx(&bars->q_full[qs], C::kTile);
-        const int qrow = static_cast<int>(bh * S + static_cast<int64_t>(it.i) * kM);
+      auto fill = [&](const CUtensorMap* map, const Step& st, int blk) -> bool {
+        const int s = static_cast<int>(f % kSlots);
+        const int64_t r = f / kSlots;
+        if (!wait_bar(&bars->kv_empty[s], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
+          return false;
+        mbar_expect_tx(&bars->kv_full[s], C::kTile);
+        const int row =
+            static_cast<int>((static_cast<int64_t>(st.it.b) * Hkv + st.it.g) * S) + blk * kN;
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_2d(q_tiles + qs * C::kTile + x * (kM * 128), &tm_q, x * 64, qrow,
-                      &bars->q_full[qs]);
-        q_round[qs] = n >> 1;
-        const int cnt = plan.k[it.i];
-        const int32_t* list = sel_idx + bh * cap + plan.off[it.i];
-        const int kvrow0 = static_cast<int>((static_cast<int64_t>(it.b) * Hkv + it.g) * S);
-        for (int j = 0; j < cnt && ok; ++j) {
-          const int blk = min(max(list[j], 0), it.i);
-          for (int which = 0; which < 2; ++which, ++f) {
-            const int s = static_cast<int>(f % kSlots);
-            const int64_t r = f / kSlots;
-            if (!(ok = wait_bar(&bars->kv_empty[s], static_cast<uint32_t>((r & 1) ^ 1), bars,
-                                status)))
-              break;
-            mbar_expect_tx(&bars->kv_full[s], C::kTile);
-            const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
-            for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_2d(kv_tiles + s * C::kTile + x * (kN * 128), map, x * 64,
-                          kvrow0 + blk * kN, &bars->kv_full[s]);
-            slot_round[s] = r;
-          }
+          tma_load_2d(kv_tiles + s * C::kTile + x * (kN * 128), map, x * 64, row,
+                      &bars->kv_full[s], pol_kv);
+        slot_round[s] = r;
+        ++f;
+        return true;
+      };
+      auto load_q = [&](const Step& st, int tile) -> bool {
+        const int64_t r = q_loads[tile];
+        if (!wait_bar(&bars->q_empty[tile], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
+          return false;
+        mbar_expect_tx(&bars->q_full[tile], C::kTile);
+        const int h = tile == 0 ? st.it.hA : st.it.hB;
+        const int qrow = static_cast<int>((static_cast<int64_t>(st.it.b) * Hq + h) * S +
+                                          static_cast<int64_t>(st.it.i) * kM);
+        for (int x = 0; x < C::kBoxes; ++x)
+          tma_load_2d(q_tiles + tile * C::kTile + x * (kM * 128), &tm_q, x * 64, qrow,
+                      &bars->q_full[tile], pol_q);
+        ++q_loads[tile];
+        return true;
+      };
+      auto start_step = [&](const Step& st) -> bool {  // Q at item start, then K of tile A
+        if (st.first) {
+          if (!load_q(st, 0)) return false;
+          if (st.has_b() && !load_q(st, 1)) return false;
         }
+        return fill(&tm_k, st, st.ba);
+      };
+      Seq seq;
+      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched);
+      Step x;
+      bool have = seq.next(x);
+      if (have) {
+        ok = start_step(x);
+        if (ok && x.has_b() && !x.shared()) ok = fill(&tm_k, x, x.bb);
+      }
+      while (have && ok) {
+        const Step c = x;
+        have = seq.next(x);
+        if (!(ok = fill(&tm_v, c, c.ba))) break;
+        if (have && !(ok = start_step(x))) break;
+        if (c.has_b() && !c.shared() && !(ok = fill(&tm_v, c, c.bb))) break;
+        if (have && x.has_b() && !x.shared() && !(ok = fill(&tm_k, x, x.bb))) break;
       }
       if (!ok) {  // abort: let issued copies land before the CTA can exit
         for (int s = 0; s < kSlots; ++s)
           if (slot_round[s] >= 0) drain_bar(&bars->kv_full[s], slot_round[s] & 1);
-        for (int s = 0; s < 2; ++s)
-          if (q_round[s] >= 0) drain_bar(&bars->q_full[s], q_round[s] & 1);
+        for (int tl = 0; tl < 2; ++tl)
+          if (q_loads[tl] > 0) drain_bar(&bars->q_full[tl], (q_loads[tl] - 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -342,177 +454,217 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = instr_desc(kM, kN, false);
       constexpr uint32_t idesc_o = instr_desc(kM, D, true);
-      const uint32_t tm_s[2] = {tmem, tmem + 128};
-      const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
       const uint32_t q_base = su32(q_tiles), kv_base = su32(kv_tiles);
-      struct Pv {
-        int64_t g, fv;
-        int n;
-        bool first, last;
-      } prev{-1, 0, 0, false, false};
-      bool have_prev = false, ok = true;
-      int64_t g = 0, fbase = 0;
-      int n = 0;
-      auto issue_pv = [&](const Pv& p) -> bool {
-        const int ob = p.n & 1;
-        if (p.first && !wait_bar(&bars->o_empty[ob], ((p.n >> 1) & 1) ^ 1, bars, status))
-          return false;
-        if (!wait_bar(&bars->p_full[p.g & 1], static_cast<uint32_t>((p.g >> 1) & 1), bars,
-                      status))
-          return false;
-        const int sv = static_cast<int>(p.fv % kSlots);
-        if (!wait_bar(&bars->kv_full[sv], static_cast<uint32_t>((p.fv / kSlots) & 1), bars,
-                      status))
-          return false;
+      int64_t tiles = 0;           // ring tiles taken, in the producer's fill order
+      int64_t q_uses[2] = {0, 0};  // Q tiles consumed per tile
+      int64_t steps[2] = {0, 0};   // PV issued per tile (p_full parity)
+      int64_t outs[2] = {0, 0};    // items finished per tile (o_empty parity)
+      int k_slot = 0, v_slot = 0;  // slots of the current step's K and V (shared blocks)
+      bool ok = true;
+      auto take = [&](int& slot) -> bool {
+        const int64_t fidx = tiles++;
+        slot = static_cast<int>(fidx % kSlots);
+        return wait_bar(&bars->kv_full[slot], static_cast<uint32_t>((fidx / kSlots) & 1), bars,
+                        status);
+      };
+      // S_T(x) = Q_T K^T into S_T; releases what it is the last user of
+      auto issue_s = [&](const Step& st, int tl) -> bool {
+        if (st.first) {
+          const int64_t r = q_uses[tl]++;
+          if (!wait_bar(&bars->q_full[tl], static_cast<uint32_t>(r & 1), bars, status))
+            return false;
+        }
+        const bool reuse = (tl == 1 && st.shared());
+        if (!reuse && !take(k_slot)) return false;
         tc_fence_after();
-        const uint32_t vaddr = kv_base + sv * C::kTile;
+        const uint32_t qa = q_base + tl * C::kTile, ka = kv_base + k_slot * C::kTile;
+#pragma unroll
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+          const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
+          mma_ss(tmem + tl * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+        if (tl == 1 || !st.has_b() || !st.shared()) tc_commit(&bars->kv_empty[k_slot]);
+        tc_commit(&bars->s_full[tl]);
+        if (st.last) tc_commit(&bars->q_empty[tl]);
+        return true;
+      };
+      // O_T += P_T V (P from TMEM over the first half of S_T)
+      auto issue_pv = [&](const Step& st, int tl) -> bool {
+        if (st.first) {
+          const int64_t r = outs[tl];
+          if (!wait_bar(&bars->o_empty[tl], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
+            return false;
+        }
+        const int64_t r = steps[tl]++;
+        if (!wait_bar(&bars->p_full[tl], static_cast<uint32_t>(r & 1), bars, status))
+          return false;
+        const bool reuse = (tl == 1 && st.shared());
+        if (!reuse && !take(v_slot)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = kv_base + v_slot * C::kTile;
+        const uint32_t o_tm = tmem + 256 + tl * 128, p_tm = tmem + tl * 128;
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk) {
           // B = V rows kk*16 .. +15 (keys), MN-major: 64-column boxes kN*128 bytes apart
           const uint64_t bd = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
-          mma_ts(tm_o[ob], tm_s[p.g & 1] + kk * 8, bd, idesc_o, (p.first && kk == 0) ? 0u : 1u);
+          mma_ts(o_tm, p_tm + kk * 8, bd, idesc_o, (st.first && kk == 0) ? 0u : 1u);
         }
-        tc_commit(&bars->kv_empty[sv]);
-        tc_commit(&bars->pv_done);
-        if (p.last) tc_commit(&bars->o_full[ob]);
+        if (tl == 1 || !st.has_b() || !st.shared()) tc_commit(&bars->kv_empty[v_slot]);
+        if (st.last) {
+          tc_commit(&bars->o_full[tl]);
+          ++outs[tl];
+        }
         return true;
       };
-      for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
-        const Item it = decode(t, G, nb, Hkv, plan.order);
-        const int qs = n & 1;
-        const int cnt = plan.k[it.i];
-        if (!(ok = wait_bar(&bars->q_full[qs], (n >> 1) & 1, bars, status))) break;
-        for (int j = 0; j < cnt; ++j, ++g) {
-          const int64_t fk = fbase + 2 * j;
-          const int sk = static_cast<int>(fk % kSlots);
-          if (!(ok = wait_bar(&bars->kv_full[sk], static_cast<uint32_t>((fk / kSlots) & 1), bars,
-                              status)))
-            break;
-          tc_fence_after();
-          const uint32_t qa = q_base + qs * C::kTile, ka = kv_base + sk * C::kTile;
-#pragma unroll
-          for (int kk = 0; kk < C::kKSteps; ++kk) {
-            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
-            mma_ss(tm_s[g & 1], smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
-                   idesc_s, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars->kv_empty[sk]);
-          tc_commit(&bars->s_full[g & 1]);
-          if (j == cnt - 1) tc_commit(&bars->q_empty[qs]);
-          if (have_prev && !(ok = issue_pv(prev))) break;
-          prev = Pv{g, fk + 1, n, j == 0, j == cnt - 1};
-          have_prev = true;
-        }
-        fbase += 2 * static_cast<int64_t>(cnt);
+      Seq seq;
+      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched);
+      Step x;
+      bool have = seq.next(x);
+      if (have) {
+        ok = issue_s(x, 0);
+        if (ok && x.has_b()) ok = issue_s(x, 1);
       }
-      if (ok && have_prev) ok = issue_pv(prev);
+      while (have && ok) {
+        const Step c = x;
+        have = seq.next(x);
+        if (!(ok = issue_pv(c, 0))) break;
+        if (have && !(ok = issue_s(x, 0))) break;
+        if (c.has_b() && !(ok = issue_pv(c, 1))) break;
+        if (have && x.has_b() && !(ok = issue_s(x, 1))) break;
+      }
       // make sure every issued product has completed before TMEM is released
       tc_commit(&bars->drain);
       drain_bar(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    constexpr int kH = kN / 2;          // key columns per thread
+    constexpr int kDH = D / 2;          // output columns per thread
     const int sub = warp & 3;           // TMEM sub-partition of this warp
+    const int half = (warp - 2) >> 2;   // 0: columns [0, 64), 1: [64, 128)
     const int row = sub * 32 + lane;    // query row within the tile
+    const int bar_id = 1 + sub;         // named barrier of the warp pair (sub, sub + 4)
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(D));
-    int64_t g = 0;
-    int n = 0;
+    // per-tile state lives in scalars (passed by reference) so it stays in registers
+    int64_t steps_a = 0, steps_b = 0, outs_a = 0, outs_b = 0;
+    int xp = 0;  // exchange-slot parity
+    float m_a = 0.f, m_b = 0.f, l_a = 0.f, l_b = 0.f;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x, ++n) {
-      const Item it = decode(t, G, nb, Hkv, plan.order);
-      const int64_t bh = static_cast<int64_t>(it.b) * Hq + it.h;
-      const int cnt = plan.k[it.i];
-      const int32_t* list = sel_idx + bh * cap + plan.off[it.i];
-      const int ob = n & 1;
-      const uint32_t o_addr = tmem + 256 + ob * 128 + lane_off;
-      float m_run = 0.f, l = 0.f;
-      for (int j = 0; j < cnt; ++j, ++g) {
-        const int sb = static_cast<int>(g & 1);
-        ok = wait_bar(&bars->s_full[sb], static_cast<uint32_t>((g >> 1) & 1), bars, status);
-        if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before tcgen05.ld
-        tc_fence_after();
-        const uint32_t s_addr = tmem + sb * 128 + lane_off;
-        uint32_t sr[kN];
-#pragma unroll
-        for (int c = 0; c < kN / 32; ++c) TC_LD32(s_addr + 32 * c, (sr + 32 * c));
-        tc_wait_ld();
-        const bool diag = min(max(list[j], 0), it.i) == it.i;
-        if (diag) {  // token-causal inside the query's own block
-#pragma unroll
-          for (int c = 0; c < kN; ++c)
-            if (c > row) sr[c] = __float_as_uint(-INFINITY);
-        }
-        float mx[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
-#pragma unroll
-        for (int c = 8; c < kN; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-        const float mt =
-            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-        if (j == 0) {
-          m_run = mt;
-        } else if (__any_sync(0xffffffffu, mt > m_run + 8.0f)) {
-          // some row's max grew by more than 2^8: the whole warp rescales its rows of O (each
-          // by its own factor, 1 where the max did not grow); PV of the previous block first
-          const float m_new = fmaxf(m_run, mt);
-          const float alpha = ex2(m_run - m_new);
-          m_run = m_new;
-          l *= alpha;
-          ok = wait_bar(&bars->pv_done, static_cast<uint32_t>((g - 1) & 1), bars, status);
-          if (!(ok = __all_sync(0xffffffffu, ok))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            TC_LD32(o_addr + 32 * c, o);
-            tc_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            TC_ST32(o_addr + 32 * c, o);
-          }
-          tc_wait_st();
-        }
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t p[kN / 2];
-#pragma unroll
-        for (int c = 0; c < kN / 2; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_run));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_run));
-          sum[c & 3] += p0 + p1;
-          p[c] = pack_bf16(p0, p1);
-        }
-        l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
-        TC_ST32(s_addr, p);
-        TC_ST32(s_addr + 32, (p + 32));
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[sb]);
-      }
-      if (!ok) break;
-      // epilogue
-      ok = wait_bar(&bars->o_full[ob], (n >> 1) & 1, bars, status);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+    // one step of tile tl on key block blk; returns false on abort
+    auto step = [&](int tl, int blk, int qi, bool first, int64_t& nsteps, float& m_run,
+                    float& lsum) -> bool {
+      const int64_t r = nsteps++;
+      bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(r & 1), bars, status);
+      if (!__all_sync(0xffffffffu, w)) return false;  // warp-uniform before tcgen05.ld
       tc_fence_after();
-      const float inv = 1.0f / l;
-      __nv_bfloat16* dst = out + (bh * S + static_cast<int64_t>(it.i) * kM + row) * D;
+      const uint32_t s_addr = tmem + tl * 128 + lane_off;
+      uint32_t sr[kH];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < kH / 32; ++c) TC_LD32(s_addr + half * kH + 32 * c, (sr + 32 * c));
+      tc_wait_ld();
+      if (blk == qi) {  // the diagonal block: token-causal
+#pragma unroll
+        for (int c = 0; c < kH; ++c)
+          if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
+#pragma unroll
+      for (int c = 8; c < kH; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      bars->xch[xp][half][row] = mt;
+      pair_sync(bar_id);
+      mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // row max, both halves alike
+      xp ^= 1;
+      if (first) {
+        m_run = mt;
+        lsum = 0.f;
+      } else if (__any_sync(0xffffffffu, mt > m_run + 8.0f)) {
+        // a row's max grew by more than 2^8: the warp rescales its part of O_T (each row by
+        // its own factor, 1 where the max did not grow). The previous P V of this tile is
+        // complete: this S was issued after it and s_full tracks every earlier product.
+        const float m_new = fmaxf(m_run, mt);
+        const float alpha = ex2(m_run - m_new);
+        m_run = m_new;
+        lsum *= alpha;
+        const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
+#pragma unroll
+        for (int c = 0; c < kDH / 32; ++c) {
+          uint32_t o[32];
+          TC_LD32(o_addr + 32 * c, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          TC_ST32(o_addr + 32 * c, o);
+        }
+        tc_wait_st();
+      }
+      const float mr = m_run;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t p[kH / 2];
+#pragma unroll
+      for (int c = 0; c < kH / 2; ++c) {
+        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mr));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mr));
+        sum[c & 3] += p0 + p1;
+        p[c] = pack_bf16(p0, p1);
+      }
+      lsum += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      // P over S_T columns [0, 64): this half's keys go to columns half*32 .. +32 (both halves
+      // finished reading S before the pair barrier above)
+      TC_ST32(s_addr + half * (kH / 2), p);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[tl]);
+      return true;
+    };
+    auto epilogue = [&](int tl, const Item& it, int64_t& nouts, float lsum) -> bool {
+      bars->xl[tl][half][row] = lsum;
+      pair_sync(bar_id);
+      const float inv = 1.0f / (lsum + bars->xl[tl][half ^ 1][row]);
+      const int64_t r = nouts++;
+      bool w = wait_bar(&bars->o_full[tl], static_cast<uint32_t>(r & 1), bars, status);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      const int h = tl == 0 ? it.hA : it.hB;
+      __nv_bfloat16* dst = out + ((static_cast<int64_t>(it.b) * Hq + h) * S +
+                                  static_cast<int64_t>(it.i) * kM + row) * D + half * kDH;
+      const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
+#pragma unroll
+      for (int c = 0; c < kDH / 32; ++c) {
         uint32_t o[32];
         TC_LD32(o_addr + 32 * c, o);
         tc_wait_ld();
         uint4 pk[4];
-        uint32_t* w = reinterpret_cast<uint32_t*>(pk);
+        uint32_t* wv = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d4[e] = pk[e];
+        for (int e = 0; e < 4; ++e) __stcs(d4 + e, pk[e]);  // evict-first: keep K/V in L2
       }
       tc_fence_before();
-      mbar_arrive(&bars->o_empty[ob]);
+      mbar_arrive(&bars->o_empty[tl]);
+      return true;
+    };
+    for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x) {
+      const Item it = decode(t, G, nb, Hkv, plan.order);
+      const int cnt = plan.k[it.i];
+      const uint32_t* srow = sched_row(sched, it, Hkv, G, cap, plan);
+      for (int j = 0; j < cnt && ok; ++j) {
+        int ba, bb;
+        sched_step(srow[j], it.i, ba, bb);
+        ok = step(0, ba, it.i, j == 0, steps_a, m_a, l_a);
+        if (ok && it.hB >= 0) ok = step(1, bb, it.i, j == 0, steps_b, m_b, l_b);
+      }
+      if (!ok) break;
+      ok = epilogue(0, it, outs_a, l_a);
+      if (ok && it.hB >= 0) ok = epilogue(1, it, outs_b, l_b);
     }
   }
 
@@ -558,10 +710,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
 
 template <int D>
 cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                         int S, PlanDev plan, int64_t cap, const int32_t* sel_idx, void* out,
-                         int32_t* status, cudaStream_t st) {
+                         int S, PlanDev plan, int64_t cap, const int32_t* sel_idx,
+                         uint32_t* sched, void* out, int32_t* status, cudaStream_t st) {
   const int nb = S / kM;
-  const int64_t items = static_cast<int64_t>(B) * Hq * nb;
+  const int G = Hq / Hkv;
+  const int64_t items = static_cast<int64_t>(B) * Hkv * nb * ((G + 1) / 2);  // head pairs
   if (items == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, static_cast<uint64_t>(B) * Hq * S, D) ||
@@ -575,9 +728,11 @@ cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  e = launch_pairs(sel_idx, B, Hq, Hkv, nb, plan, cap, sched, st);
+  if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(items, sm_count());
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, Hq, Hkv, S, nb, items,
-                                                           plan, cap, sel_idx,
+                                                           plan, cap, sched,
                                                            static_cast<__nv_bfloat16*>(out),
                                                            status);
   return cudaGetLastError();
@@ -587,12 +742,12 @@ cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int
 
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
                              int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
-                             const int32_t* sel_idx, const int32_t*, void* out, int32_t* status,
-                             cudaStream_t st) {
+                             const int32_t* sel_idx, const int32_t*, uint32_t* sched, void* out,
+                             int32_t* status, cudaStream_t st) {
   if (block == 128 && D == 128)
-    return launch_sm100<128>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, out, status, st);
+    return launch_sm100<128>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, sched, out, status, st);
   if (block == 128 && D == 64)
-    return launch_sm100<64>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, out, status, st);
+    return launch_sm100<64>(q, k, v, B, Hq, Hkv, S, plan, cap, sel_idx, sched, out, status, st);
   return launch_attn_bf16_mma(q, k, v, B, Hq, Hkv, S, D, block, plan, cap, sel_idx, out, st);
 }
 

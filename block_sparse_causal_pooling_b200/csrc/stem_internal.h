@@ -23,11 +23,19 @@ cudaError_t launch_select(const float* qbar, const float* kbar, const float* vno
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
                           int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st);
 
-// Block-sparse attention, bfloat16 inputs on the tensor cores (attn_bf16.cu).
+// Block-sparse attention, bfloat16 inputs on the tensor cores (attn_sm100.cu; block 64 falls to
+// the mma.sync kernel of attn_bf16.cu). `sched` is workspace of pairs_bytes() for the head-pair
+// step schedule (pairs.cu).
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
                              int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
-                             const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
-                             int32_t* status, cudaStream_t st);
+                             const int32_t* sel_idx, const int32_t* sel_cnt, uint32_t* sched,
+                             void* out, int32_t* status, cudaStream_t st);
+
+// Head-pair step schedules from the CSR lists (pairs.cu).
+cudaError_t launch_pairs(const int32_t* sel_idx, int B, int Hq, int Hkv, int nb, PlanDev plan,
+                         int64_t cap, uint32_t* sched, cudaStream_t st);
+// Workspace bytes of the schedule for any budget of this shape.
+size_t pairs_bytes(int B, int Hq, int Hkv, int nb);
 
 // Block-sparse attention, float32 inputs on the CUDA cores (attn_f32.cu).
 cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, int B, int Hq,
