@@ -1,0 +1,81 @@
+"""Full-size parity: every named workload at its real shape, through the same C-ABI call and
+launch configuration the benchmark times (stem_prefill_ex, caller workspace, torch's stream).
+
+Selection is compared with the oracle on every (b, head, query block) row (ties within 1e-6
+relative allowed). Attention is compared on a deterministic sample of query blocks that the
+fp64 oracle computes one by one (bounded to a few tens of GFLOP per workload), and, for the
+dense budget rho_min = 1, on the whole output against torch's scaled_dot_product_attention.
+"""
+
+import random
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_causal_pooling_b200 import stem as S
+from block_sparse_causal_pooling_b200 import workloads as wl
+from tests import parity
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+DEV = "cuda:0"
+FULL = [wl.LLAMA_32K, wl.LLAMA_128K, wl.QWEN_64K] + list(wl.SWEEP_128K[1:]) + list(wl.SWEEP_B4_16K)
+ORACLE_GFLOP_BUDGET = 40.0
+
+
+def sample(w, kk, seed=7):
+    """Blocks 0, 1, nb-1 of heads 0 and Hq-1, then random (b, h, i) rows while the oracle's
+    effective work stays within the budget."""
+    rng = random.Random(seed)
+    rows, total = [], 0.0
+    for (b, h, i) in [(0, 0, 0), (0, 0, 1), (0, w.Hq - 1, 0), (0, w.Hq - 1, w.nb - 1),
+                      (w.B - 1, 0, w.nb - 1)]:
+        rows.append((b, h, i))
+        total += wl.effective_flops(int(kk[i]), w.block, w.D)
+    tries = 0
+    while tries < 500:
+        tries += 1
+        r = (rng.randrange(w.B), rng.randrange(w.Hq), rng.randrange(w.nb))
+        f = wl.effective_flops(int(kk[r[2]]), w.block, w.D)
+        if r in rows or total + f > ORACLE_GFLOP_BUDGET * 1e9:
+            continue
+        rows.append(r)
+        total += f
+    return sorted(set(rows))
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_full_size_selection_and_sampled_attention(w):
+    q, k, v = wl.make_inputs(w, DEV)
+    out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min)
+    ws = S.alloc_workspace(q, k, w.block)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S.stem_prefill_ex(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt, ws,
+                      status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+    qb, kb, vn = oracle.pool(qc, kc, vc, w.block)
+    m = oracle.metric(qb, kb, vn)
+    ref_idx, ref_cnt = oracle.select(m, kk, off)
+    res = parity.compare_selection(sel_idx, sel_cnt, ref_idx, ref_cnt, m, kk, off)
+    assert not res["violations"], res["violations"][:5]
+    assert res["tie_swaps"] <= max(1, res["rows"] // 100), res
+    swapped = set(res["rows_bad"])
+    rows = [r for r in sample(w, kk) if r not in swapped]
+    ref = oracle.attention(qc, kc, vc, w.block, ref_idx, ref_cnt, off, rows)
+    parity.assert_out_close(parity.out_rows(out, rows, w.block), ref, w.torch_dtype, w.name)
+    if w.rho_min == 1.0:  # dense: the whole output against the library routine
+        G = w.Hq // w.Hkv
+        k_rep = k.repeat_interleave(G, 1)
+        v_rep = v.repeat_interleave(G, 1)
+        for b in range(w.B):
+            for h0 in range(0, w.Hq, 8):
+                sl = (slice(b, b + 1), slice(h0, min(w.Hq, h0 + 8)))
+                ref_d = torch.nn.functional.scaled_dot_product_attention(
+                    q[sl], k_rep[sl], v_rep[sl], is_causal=True)
+                d = (out[sl].float() - ref_d.float()).abs()
+                assert float(d.max()) <= 2e-2 and float(d.mean()) <= 1e-3, (b, h0)
