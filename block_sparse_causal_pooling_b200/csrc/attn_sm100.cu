@@ -222,6 +222,33 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Two fp32 lanes per instruction (sm_100 f32x2 arithmetic).
+struct f2 {
+  float x, y;
+};
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -327,6 +354,20 @@ struct Seq {
     ++j;
     return true;
   }
+};
+
+// Fill indices of the K/V tiles each step's products take, in the MMA thread's issue order:
+// S_A(0), S_B(0), then for every step c with successor x: P V_A(c), S_A(x), P V_B(c), S_B(x).
+// A block both heads keep is one tile. The MMA thread (which takes the tiles) and the release
+// thread (which frees them) run this same recurrence, so both agree on every slot.
+struct TileOrder {
+  int64_t next = 0;
+  int64_t kA = 0, kB = 0, vA = 0, vB = 0;  // tiles of the latest S_A, S_B, PV_A, PV_B
+  // call in issue order: k_a(x0), k_b(x0); then per step c: v_a(), k_a(x), v_b(c), k_b(x)
+  __device__ __forceinline__ void k_a() { kA = next++; }
+  __device__ __forceinline__ void k_b(bool shared) { kB = shared ? kA : next++; }
+  __device__ __forceinline__ void v_a() { vA = next++; }
+  __device__ __forceinline__ void v_b(bool shared) { vB = shared ? vA : next++; }
 };
 
 template <int D>
@@ -455,42 +496,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = instr_desc(kM, kN, false);
       constexpr uint32_t idesc_o = instr_desc(kM, D, true);
       const uint32_t q_base = su32(q_tiles), kv_base = su32(kv_tiles);
-      int64_t tiles = 0;           // ring tiles taken, in the producer's fill order
       int64_t q_uses[2] = {0, 0};  // Q tiles consumed per tile
       int64_t steps[2] = {0, 0};   // PV issued per tile (p_full parity)
       int64_t outs[2] = {0, 0};    // items finished per tile (o_empty parity)
-      int k_slot = 0, v_slot = 0;  // slots of the current step's K and V (shared blocks)
       bool ok = true;
-      auto take = [&](int& slot) -> bool {
-        const int64_t fidx = tiles++;
-        slot = static_cast<int>(fidx % kSlots);
-        return wait_bar(&bars->kv_full[slot], static_cast<uint32_t>((fidx / kSlots) & 1), bars,
+      TileOrder order;
+      auto wait_tile = [&](int64_t f) -> bool {
+        return wait_bar(&bars->kv_full[f % kSlots], static_cast<uint32_t>((f / kSlots) & 1), bars,
                         status);
       };
-      // S_T(x) = Q_T K^T into S_T; releases what it is the last user of
+      // S_T(x) = Q_T K^T into S_T; one commit, to s_full[T]. Every release (K and V slots, Q)
+      // is done by the softmax release thread when it sees that commit: a commit covers every
+      // earlier product of this thread.
       auto issue_s = [&](const Step& st, int tl) -> bool {
         if (st.first) {
           const int64_t r = q_uses[tl]++;
           if (!wait_bar(&bars->q_full[tl], static_cast<uint32_t>(r & 1), bars, status))
             return false;
         }
-        const bool reuse = (tl == 1 && st.shared());
-        if (!reuse && !take(k_slot)) return false;
+        const int64_t f = tl == 0 ? order.kA : order.kB;
+        if (!(tl == 1 && st.shared()) && !wait_tile(f)) return false;
         tc_fence_after();
-        const uint32_t qa = q_base + tl * C::kTile, ka = kv_base + k_slot * C::kTile;
+        const uint32_t qa = q_base + tl * C::kTile;
+        const uint32_t ka = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
 #pragma unroll
         for (int kk = 0; kk < C::kKSteps; ++kk) {
           const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
           mma_ss(tmem + tl * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
                  idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (tl == 1 || !st.has_b() || !st.shared()) tc_commit(&bars->kv_empty[k_slot]);
         tc_commit(&bars->s_full[tl]);
-        if (st.last) tc_commit(&bars->q_empty[tl]);
         return true;
       };
-      // O_T += P_T V (P from TMEM over the first half of S_T)
-      auto issue_pv = [&](const Step& st, int tl) -> bool {
+      // O_T += P_T V (P from TMEM over the first half of S_T). No commit: the next S_T commit
+      // covers it; o_full at the item's end; and when head B has no next step (the next item
+      // has a single head, or the sequence ends), its V slot is released here.
+      auto issue_pv = [&](const Step& st, int tl, bool next_has_b) -> bool {
         if (st.first) {
           const int64_t r = outs[tl];
           if (!wait_bar(&bars->o_empty[tl], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
@@ -499,10 +540,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t r = steps[tl]++;
         if (!wait_bar(&bars->p_full[tl], static_cast<uint32_t>(r & 1), bars, status))
           return false;
-        const bool reuse = (tl == 1 && st.shared());
-        if (!reuse && !take(v_slot)) return false;
+        const int64_t f = tl == 0 ? order.vA : order.vB;
+        if (!(tl == 1 && st.shared()) && !wait_tile(f)) return false;
         tc_fence_after();
-        const uint32_t vaddr = kv_base + v_slot * C::kTile;
+        const uint32_t vaddr = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
         const uint32_t o_tm = tmem + 256 + tl * 128, p_tm = tmem + tl * 128;
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk) {
@@ -510,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
           mma_ts(o_tm, p_tm + kk * 8, bd, idesc_o, (st.first && kk == 0) ? 0u : 1u);
         }
-        if (tl == 1 || !st.has_b() || !st.shared()) tc_commit(&bars->kv_empty[v_slot]);
+        if (tl == 1 && !next_has_b) tc_commit(&bars->kv_empty[f % kSlots]);
         if (st.last) {
           tc_commit(&bars->o_full[tl]);
           ++outs[tl];
@@ -522,16 +563,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       Step x;
       bool have = seq.next(x);
       if (have) {
+        order.k_a();
         ok = issue_s(x, 0);
-        if (ok && x.has_b()) ok = issue_s(x, 1);
+        if (ok && x.has_b()) {
+          order.k_b(x.shared());
+          ok = issue_s(x, 1);
+        }
       }
       while (have && ok) {
         const Step c = x;
         have = seq.next(x);
-        if (!(ok = issue_pv(c, 0))) break;
-        if (have && !(ok = issue_s(x, 0))) break;
-        if (c.has_b() && !(ok = issue_pv(c, 1))) break;
-        if (have && x.has_b() && !(ok = issue_s(x, 1))) break;
+        order.v_a();
+        if (!(ok = issue_pv(c, 0, false))) break;
+        if (have) {
+          order.k_a();
+          if (!(ok = issue_s(x, 0))) break;
+        }
+        if (c.has_b()) {
+          order.v_b(c.shared());
+          if (!(ok = issue_pv(c, 1, have && x.has_b()))) break;
+        }
+        if (have && x.has_b()) {
+          order.k_b(x.shared());
+          if (!(ok = issue_s(x, 1))) break;
+        }
       }
       // make sure every issued product has completed before TMEM is released
       tc_commit(&bars->drain);
@@ -552,12 +607,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     int xp = 0;  // exchange-slot parity
     float m_a = 0.f, m_b = 0.f, l_a = 0.f, l_b = 0.f;
     bool ok = true;
+    // The release thread frees ring slots and Q tiles: when S_T of a step is complete, so is
+    // every product issued before it (K of this step unless head B still needs it, V of the
+    // previous step, Q after the item's last S).
+    const bool releaser = (warp == 2 && lane == 0);
+    auto release = [&](int64_t tile) {
+      if (tile >= 0) mbar_arrive(&bars->kv_empty[tile % kSlots]);
+    };
     // one step of tile tl on key block blk; returns false on abort
     auto step = [&](int tl, int blk, int qi, bool first, int64_t& nsteps, float& m_run,
-                    float& lsum) -> bool {
+                    float& lsum, int64_t rel_k, int64_t rel_v, bool rel_q) -> bool {
       const int64_t r = nsteps++;
       bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(r & 1), bars, status);
       if (!__all_sync(0xffffffffu, w)) return false;  // warp-uniform before tcgen05.ld
+      if (releaser) {
+        release(rel_k);
+        release(rel_v);
+        if (rel_q) mbar_arrive(&bars->q_empty[tl]);
+      }
       tc_fence_after();
       const uint32_t s_addr = tmem + tl * 128 + lane_off;
       uint32_t sr[kH];
@@ -569,13 +636,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kH; ++c)
           if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx[8];
+      float mx[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
+      for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
 #pragma unroll
-      for (int c = 8; c < kH; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 4; c < kH; c += 2)
+        mx[(c >> 1) & 3] =
+            max3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       bars->xch[xp][half][row] = mt;
       pair_sync(bar_id);
       mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // row max, both halves alike
@@ -603,17 +671,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_wait_st();
       }
-      const float mr = m_run;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
+      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
       uint32_t p[kH / 2];
 #pragma unroll
       for (int c = 0; c < kH / 2; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mr));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mr));
-        sum[c & 3] += p0 + p1;
-        p[c] = pack_bf16(p0, p1);
+        const f2 x = fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
+        const f2 e{ex2(x.x), ex2(x.y)};
+        sum[c & 1] = add2(sum[c & 1], e);
+        p[c] = pack_bf16(e.x, e.y);
       }
-      lsum += (sum[0] + sum[1]) + (sum[2] + sum[3]);
+      lsum += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
       // P over S_T columns [0, 64): this half's keys go to columns half*32 .. +32 (both halves
       // finished reading S before the pair barrier above)
       TC_ST32(s_addr + half * (kH / 2), p);
@@ -652,15 +720,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->o_empty[tl]);
       return true;
     };
+    TileOrder order;  // replica of the MMA thread's tile numbering
+    bool have_prev = false, prev_has_b = false, prev_shared = false;
     for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x) {
       const Item it = decode(t, G, nb, Hkv, plan.order);
       const int cnt = plan.k[it.i];
       const uint32_t* srow = sched_row(sched, it, Hkv, G, cap, plan);
       for (int j = 0; j < cnt && ok; ++j) {
-        int ba, bb;
-        sched_step(srow[j], it.i, ba, bb);
-        ok = step(0, ba, it.i, j == 0, steps_a, m_a, l_a);
-        if (ok && it.hB >= 0) ok = step(1, bb, it.i, j == 0, steps_b, m_b, l_b);
+        Step x;
+        x.it = it;
+        sched_step(srow[j], it.i, x.ba, x.bb);
+        const bool has_b = x.has_b(), shared = x.shared();
+        if (have_prev) order.v_a();
+        order.k_a();
+        if (have_prev && prev_has_b) order.v_b(prev_shared);
+        if (has_b) order.k_b(shared);
+        const int64_t rka = (has_b && shared) ? -1 : order.kA;
+        const int64_t rva = (have_prev && !(prev_has_b && prev_shared)) ? order.vA : -1;
+        ok = step(0, x.ba, it.i, j == 0, steps_a, m_a, l_a, rka, rva, j == cnt - 1);
+        if (ok && has_b) {
+          const int64_t rvb = (have_prev && prev_has_b) ? order.vB : -1;
+          ok = step(1, x.bb, it.i, j == 0, steps_b, m_b, l_b, order.kB, rvb, j == cnt - 1);
+        }
+        have_prev = true;
+        prev_has_b = has_b;
+        prev_shared = shared;
       }
       if (!ok) break;
       ok = epilogue(0, it, outs_a, l_a);
