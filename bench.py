@@ -41,6 +41,11 @@ from block_sparse_causal_pooling_b200 import workloads as wl  # noqa: E402
 METRIC = "Stem prefill attention latency (ms) & effective TFLOP/s at S=128K, % of BF16 peak"
 # library kernels per step: pooling, metric + selection, head-pair schedule, attention
 KERNELS_PER_STEP = 4
+# DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
+# profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
+# to the revision that capture measured.
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1.61e9 + 1.02e9,
+                "sources_sha256": "8739a962b45f0028ef68ca8c219bf2de73c48dc5dfcbfcd2bf56e46834b5ebe0"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -54,6 +59,18 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
+
+
+def attn_traffic(workload_name):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("attn_sm100.cu", "pairs.cu"):
+        with open(os.path.join(ROOT, "block_sparse_causal_pooling_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if workload_name == ATTN_TRAFFIC["workload"] and h.hexdigest() == ATTN_TRAFFIC["sources_sha256"]:
+        return ATTN_TRAFFIC["bytes"]
+    return None
 
 
 def peaks():
@@ -368,7 +385,7 @@ def run_ours(args, world, rank, local):
                        causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                     "traffic": None,
+                     "traffic": attn_traffic(w.name),
                      "peak_source": f"{pk_kind} {'sustained' if long_region else 'burst'} "
                                     "bf16 dense"},
         "kernels": {
