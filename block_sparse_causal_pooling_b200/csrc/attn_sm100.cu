@@ -7,28 +7,34 @@
 // step 3; gist.science/it 2.C step 3; gist.science/nl "Implementatie" step 3; gist.science/fr
 // 2.C step 3).
 //
+// Work item: two GQA sibling heads A and B at one query block, which keep the same number of key
+// blocks; a step schedule (pairs.cu) pairs their lists so a block both keep is one K/V tile.
+//
 // Persistent kernel, one CTA per SM, 10 warps:
-//   warp 0      TMA producer: Q tile (double-buffered) and K/V tiles of the kept blocks into a
-//               4-slot ring of 32 KB shared-memory tiles (128B-swizzled boxes of 128 x 64).
-//   warp 1      allocates 512 TMEM columns; lane 0 issues every tcgen05.mma:
-//                 S[g%2] = Q K^T           (M 128, N 128, K = D; A and B K-major in smem)
-//                 O[n%2] += P V            (A = P read from TMEM, B = V MN-major in smem)
-//               S is double-buffered so S of the next key block runs while the softmax works on
-//               the current one; O is double-buffered across work items so the epilogue of one
-//               item overlaps the next item's products.
+//   warp 0      TMA producer: Q_A, Q_B (one tile each) and K/V tiles into a 4-slot ring of
+//               128B-swizzled shared-memory tiles (boxes of 128 rows x 64 columns), filled in the
+//               order the products first use them.
+//   warp 1      allocates the 512 TMEM columns; lane 0 issues every tcgen05.mma:
+//                 S_T = Q_T K^T     (M 128, N 128, K = D; A and B K-major in shared memory)
+//                 O_T += P_T V      (A = P read from TMEM over the first half of S_T, B = V
+//                                    MN-major in shared memory)
+//               in the order P V_A(c), S_A(c+1), P V_B(c), S_B(c+1), so one head's products run
+//               while the softmax works on the other head; one commit per S, none per P V.
 //   warps 2-9   softmax, two threads per query row (warps w and w+4 share TMEM lanes
 //               32*(w%4).. and take 64 columns each; tcgen05.ld 32x32b): row max (halves
-//               exchanged through shared memory under a per-pair named barrier), exp2 with the
-//               1/sqrt(D) scale folded in, per-thread partial row sums in fp32; P packed to bf16
-//               and stored over the first half of its S buffer (tcgen05.st); O rescaled in TMEM
-//               only when the running max grows by more than 2^8 (exact: the final 1/l uses the
-//               same reference max). Then the epilogue: O * (1/l) -> bf16 -> global.
-// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+//               exchanged through shared memory at a barrier of the warp pair that also makes
+//               both warps agree on going on, so an abort cannot strand one), exp2 with the
+//               1/sqrt(D) scale folded in, per-thread partial row sums in fp32 (f32x2
+//               arithmetic); P packed to bf16 and stored over the first half of S_T
+//               (tcgen05.st); O rescaled in TMEM only when the running max grows by more than
+//               2^8 (exact: the final 1/l uses the same reference max). At an item's end:
+//               O * (1/l) -> bf16 -> global (streaming stores).
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).
 //
-// Synchronisation is by mbarriers only. Every wait is bounded by the global nanosecond timer: on
-// expiry the CTA records STEM_ERR_TIMEOUT in the status word, every role leaves its loop, the
-// MMA thread drains its issued products, the producer drains its issued copies (both bounded),
-// TMEM is freed and the kernel returns.
+// Synchronisation is by mbarriers, plus the warp-pair barrier above. Every mbarrier wait is
+// bounded by the global nanosecond timer: on expiry the CTA records STEM_ERR_TIMEOUT in the
+// status word, every role leaves its loop, the MMA thread drains its issued products, the
+// producer drains its issued copies (both bounded), TMEM is freed and the kernel returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -127,8 +133,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bar
                                          int32_t* status) {
   return mbar_try(b, parity) || wait_bar_slow(b, parity, bars, status);
 }
-__device__ __forceinline__ void pair_sync(int id) {  // the two warps that share TMEM lanes
-  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+// Barrier of the two warps that share TMEM lanes, which also agree on whether to go on: both
+// get the AND of their flags, so a warp that gave up (a timed-out wait) takes its partner with
+// it instead of leaving it at the barrier. Both warps make the same sequence of these calls.
+__device__ __forceinline__ bool pair_and(int id, bool go) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "barrier.cta.red.and.pred b, %2, 64, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(go)), "r"(id)
+      : "memory");
+  return r != 0;
 }
 // Bounded drain wait used on the abort path only (ignores the abort flag).
 __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
@@ -619,7 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float& lsum, int64_t rel_k, int64_t rel_v, bool rel_q) -> bool {
       const int64_t r = nsteps++;
       bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(r & 1), bars, status);
-      if (!__all_sync(0xffffffffu, w)) return false;  // warp-uniform before tcgen05.ld
+      if (!__all_sync(0xffffffffu, w)) {
+        pair_and(bar_id, false);
+        return false;
+      }
       if (releaser) {
         release(rel_k);
         release(rel_v);
@@ -645,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             max3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
       float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       bars->xch[xp][half][row] = mt;
-      pair_sync(bar_id);
+      if (!pair_and(bar_id, true)) return false;
       mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // row max, both halves alike
       xp ^= 1;
       if (first) {
@@ -691,12 +712,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     auto epilogue = [&](int tl, const Item& it, int64_t& nouts, float lsum) -> bool {
-      bars->xl[tl][half][row] = lsum;
-      pair_sync(bar_id);
-      const float inv = 1.0f / (lsum + bars->xl[tl][half ^ 1][row]);
       const int64_t r = nouts++;
       bool w = wait_bar(&bars->o_full[tl], static_cast<uint32_t>(r & 1), bars, status);
-      if (!__all_sync(0xffffffffu, w)) return false;
+      w = __all_sync(0xffffffffu, w);
+      bars->xl[tl][half][row] = lsum;
+      if (!pair_and(bar_id, w)) return false;
+      const float inv = 1.0f / (lsum + bars->xl[tl][half ^ 1][row]);
       tc_fence_after();
       const int h = tl == 0 ? it.hA : it.hB;
       __nv_bfloat16* dst = out + ((static_cast<int64_t>(it.b) * Hq + h) * S +
