@@ -9,9 +9,11 @@ boundary as single-precision floats, so the oracle rounds rho_min and tau to
 float32 first and then widens them to double, exactly as the product does.
 
 Parity status: every function here is pinned by the CPU test suite (budget:
-arbitrary-precision recomputation, closed forms; pooling, metric, selection,
+arbitrary-precision recomputation, closed forms; linear budget: cases worked by
+hand, closed forms, exact rational recomputation; pooling, metric, selection,
 attention: brute force from token-level definitions, the additive-metric
-equivalence, dense attention via a library routine). See the tests for the pins.
+equivalence and closed forms, dense attention via a library routine). See the
+tests for the pins.
 """
 
 from __future__ import annotations
@@ -43,10 +45,16 @@ def _load():
         lib.stem_oracle_budget.restype = ctypes.c_int64
         lib.stem_oracle_budget.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                            ctypes.c_int, _c_i32p, _c_i64p]
+        lib.stem_oracle_budget_linear.restype = ctypes.c_int64
+        lib.stem_oracle_budget_linear.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                                  ctypes.c_int, _c_i32p, _c_i64p]
         lib.stem_oracle_pool.restype = None
-        lib.stem_oracle_pool.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 + [_c_f64p] * 3
+        lib.stem_oracle_pool.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 8 + [_c_f64p] * 3
         lib.stem_oracle_metric.restype = None
         lib.stem_oracle_metric.argtypes = [_c_f64p] * 3 + [ctypes.c_int] * 5 + [_c_f64p]
+        lib.stem_oracle_metric_additive.restype = None
+        lib.stem_oracle_metric_additive.argtypes = ([_c_f64p] * 3 + [ctypes.c_int] * 5 +
+                                                    [ctypes.c_double, ctypes.c_int, _c_f64p])
         lib.stem_oracle_select.restype = None
         lib.stem_oracle_select.argtypes = [_c_f64p, _c_i32p, _c_i64p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int64, _c_i32p, _c_i32p]
@@ -96,8 +104,21 @@ def budget(nb: int, rho_min: float, tau: float, k_min: int):
     return k[:nb].copy(), off
 
 
-def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int):
-    """Pooled block summaries in double: qbar [B,Hq,nb,D], kbar [B,Hkv,nb,D], vnorm [B,Hkv,nb]."""
+def budget_linear(nb: int, k_start: float, mu: float, k_min: int):
+    """k[nb] (int32) and off[nb+1] (int64) of the linear position-decay budget (k_start at
+    block 0 down to mu*k_start at block nb-1)."""
+    k = np.zeros(max(nb, 1), dtype=np.int32)
+    off = np.zeros(nb + 1, dtype=np.int64)
+    _load().stem_oracle_budget_linear(nb, f32(k_start), f32(mu), int(k_min), _ptr(k, _c_i32p),
+                                      _ptr(off, _c_i64p))
+    return k[:nb].copy(), off
+
+
+def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, vsum: str = "mean"):
+    """Pooled block summaries in double: qbar [B,Hq,nb,D], kbar [B,Hkv,nb,D], vnorm [B,Hkv,nb].
+    vsum: "mean" (mean row norm of V per block) or "max" (largest row norm)."""
+    if vsum not in ("mean", "max"):
+        raise ValueError(vsum)
     q, k, v = _host(q), _host(k), _host(v)
     B, Hq, S, D = q.shape
     Hkv = k.shape[1]
@@ -106,8 +127,8 @@ def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int):
     kbar = np.zeros((B, Hkv, nb, D))
     vnorm = np.zeros((B, Hkv, nb))
     _load().stem_oracle_pool(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq,
-                             Hkv, S, D, block, _ptr(qbar, _c_f64p), _ptr(kbar, _c_f64p),
-                             _ptr(vnorm, _c_f64p))
+                             Hkv, S, D, block, int(vsum == "max"), _ptr(qbar, _c_f64p),
+                             _ptr(kbar, _c_f64p), _ptr(vnorm, _c_f64p))
     return qbar, kbar, vnorm
 
 
@@ -121,6 +142,22 @@ def metric(qbar: np.ndarray, kbar: np.ndarray, vnorm: np.ndarray) -> np.ndarray:
     m = np.zeros((B, Hq, nb * (nb + 1) // 2))
     _load().stem_oracle_metric(_ptr(qbar, _c_f64p), _ptr(kbar, _c_f64p), _ptr(vnorm, _c_f64p),
                                B, Hq, Hkv, nb, D, _ptr(m, _c_f64p))
+    return m
+
+
+def metric_additive(qbar: np.ndarray, kbar: np.ndarray, vnorm: np.ndarray, beta: float,
+                    clamp: bool = True) -> np.ndarray:
+    """The pages' additive output-aware metric s_ij + beta * max(0, log n_j^2), packed like
+    metric(); beta is rounded to float32 as the C boundary does."""
+    qbar = np.ascontiguousarray(qbar, dtype=np.float64)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float64)
+    vnorm = np.ascontiguousarray(vnorm, dtype=np.float64)
+    B, Hq, nb, D = qbar.shape
+    Hkv = kbar.shape[1]
+    m = np.zeros((B, Hq, nb * (nb + 1) // 2))
+    _load().stem_oracle_metric_additive(_ptr(qbar, _c_f64p), _ptr(kbar, _c_f64p),
+                                        _ptr(vnorm, _c_f64p), B, Hq, Hkv, nb, D, f32(beta),
+                                        int(bool(clamp)), _ptr(m, _c_f64p))
     return m
 
 
@@ -175,14 +212,29 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
 
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_min: float,
-            tau: float, k_min: int, rows: Optional[Sequence] = None, with_metric: bool = True):
+            tau: float, k_min: int, rows: Optional[Sequence] = None, with_metric: bool = True,
+            schedule: str = "exp", k_start: float = 0.0, mu: float = 1.0,
+            metric_form: str = "product", beta: float = 0.0, clamp: bool = True,
+            vsum: str = "mean"):
     """All stages. Returns a dict with k, off, qbar, kbar, vnorm, m, sel_idx, sel_cnt and
-    out ([len(rows), block, D] for the listed query blocks; all blocks when rows is None)."""
+    out ([len(rows), block, D] for the listed query blocks; all blocks when rows is None).
+    schedule "exp" uses rho_min, tau; "linear" uses k_start, mu. metric_form "product" is
+    softmax(s) * n, "additive" is s + beta * max(0, log n^2) (clamp=False drops the max)."""
     B, Hq, S, D = q.shape
     nb = S // block
-    kk, off = budget(nb, rho_min, tau, k_min)
-    qbar, kbar, vnorm = pool(q, k, v, block)
-    m = metric(qbar, kbar, vnorm)
+    if schedule == "exp":
+        kk, off = budget(nb, rho_min, tau, k_min)
+    elif schedule == "linear":
+        kk, off = budget_linear(nb, k_start, mu, k_min)
+    else:
+        raise ValueError(schedule)
+    qbar, kbar, vnorm = pool(q, k, v, block, vsum)
+    if metric_form == "product":
+        m = metric(qbar, kbar, vnorm)
+    elif metric_form == "additive":
+        m = metric_additive(qbar, kbar, vnorm, beta, clamp)
+    else:
+        raise ValueError(metric_form)
     sel_idx, sel_cnt = select(m, kk, off)
     out = attention(q, k, v, block, sel_idx, sel_cnt, off, rows)
     res = dict(k=kk, off=off, qbar=qbar, kbar=kbar, vnorm=vnorm, sel_idx=sel_idx,

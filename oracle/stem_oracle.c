@@ -21,10 +21,15 @@
  * parameterised reading used here is:
  *   budget   k(i) = min(i+1, max(k_min, ceil(rho(i)*(i+1)))),
  *            rho(i) = rho_min + (1-rho_min)*exp(-i/tau), i = query-block index;
+ *            or the pages' linear form ([es] 2.A, [it] 2.A, [nl] TPD, [fr] 2.A)
+ *            k(i) = min(i+1, max(k_min, ceil(k_start*(1 - (1-mu)*i/(nb-1)))));
  *            for i >= 1 at least 2 blocks (sink and diagonal); k(0) = 1;
  *   pooling  arithmetic mean of Q rows and of K rows per block; mean of the
- *            per-row L2 norms of V per block;
+ *            per-row L2 norms of V per block (or their maximum: the "maximised
+ *            magnitudes of V" of [nl] Implementatie step 1);
  *   metric   m_ij = softmax_{j<=i}(qbar_i . kbar_j / sqrt(D)) * n_j;
+ *            or the pages' additive form ([es] 2.B, [it] 2.B, [nl] OAM, [fr] 2.B)
+ *            M_ij = qbar_i . kbar_j / sqrt(D) + beta * max(0, log(n_j^2));
  *   keep     block 0, block i, and the k(i)-2 best other blocks j in [1, i-1]
  *            by (m descending, j ascending);
  *   attend   exact softmax attention of each query token over all tokens of
@@ -89,13 +94,48 @@ int64_t stem_oracle_budget(int nb, double rho_min, double tau, int k_min,
 }
 
 /*
+ * Token Position-Decay budget, linear form ([es] 2.A: a high budget k_start for
+ * the first tokens that decays linearly to k_end = mu * k_start for the last
+ * ones, by linear interpolation; [it] 2.A and [nl] TPD: mu in (0, 1]; [fr] 2.A).
+ * Reading: positions are query blocks, k_start is in blocks, the interpolation
+ * runs from block 0 (k_start) to block nb-1 (k_end), and the interpolated
+ * budget is rounded up, floored by k_min and capped by the i+1 causal blocks as
+ * in the exponential form. Returns sum_i k(i); writes k[nb] and off[nb+1].
+ */
+int64_t stem_oracle_budget_linear(int nb, double k_start, double mu, int k_min,
+                                  int32_t* k_out, int64_t* off_out) {
+  int64_t total = 0;
+  for (int i = 0; i < nb; ++i) {
+    /* fraction of the way from the first block to the last */
+    double t = nb > 1 ? (double)i / (double)(nb - 1) : 0.0;
+    double k_lin = k_start * (1.0 - (1.0 - mu) * t);
+    double want = ceil(k_lin);
+    double kk = want > (double)k_min ? want : (double)k_min;
+    if (kk > (double)(i + 1)) kk = (double)(i + 1);
+    int k = (int)kk;
+    if (i == 0) {
+      k = 1;
+    } else if (k < 2) {
+      k = 2;
+    }
+    if (off_out) off_out[i] = total;
+    if (k_out) k_out[i] = k;
+    total += k;
+  }
+  if (off_out) off_out[nb] = total;
+  return total;
+}
+
+/*
  * Block downsampling ([es] 2 "Implementacion" step 1: block-level Q, K and V
  * magnitude; [it] 2.C step 1; [nl] Implementatie step 1; [fr] 2.C step 1).
  * qbar [B,Hq,nb,D], kbar [B,Hkv,nb,D]: mean over the block's rows.
- * vnorm [B,Hkv,nb]: mean over the block's rows of the row's Euclidean norm.
+ * vnorm [B,Hkv,nb]: vmax == 0: mean over the block's rows of the row's
+ * Euclidean norm; vmax == 1: the largest row norm of the block ([nl]
+ * Implementatie step 1: maximised magnitudes of V).
  */
 void stem_oracle_pool(const void* q, const void* k, const void* v, int dtype, int B,
-                      int Hq, int Hkv, int S, int D, int block, double* qbar,
+                      int Hq, int Hkv, int S, int D, int block, int vmax, double* qbar,
                       double* kbar, double* vnorm) {
   const int nb = S / block;
   const int64_t nq = (int64_t)B * Hq * nb;
@@ -119,16 +159,18 @@ void stem_oracle_pool(const void* q, const void* k, const void* v, int dtype, in
       for (int r = 0; r < block; ++r) acc += elem(k, dtype, (row0 + r) * D + d);
       kbar[u * D + d] = acc / block;
     }
-    double nacc = 0.0;
+    double nacc = 0.0, nmax = 0.0;
     for (int r = 0; r < block; ++r) {
       double sq = 0.0;
       for (int d = 0; d < D; ++d) {
         double x = elem(v, dtype, (row0 + r) * D + d);
         sq += x * x;
       }
-      nacc += sqrt(sq);
+      const double norm = sqrt(sq);
+      nacc += norm;
+      if (norm > nmax) nmax = norm;
     }
-    vnorm[u] = nacc / block;
+    vnorm[u] = vmax ? nmax : nacc / block;
   }
 }
 
@@ -169,6 +211,41 @@ void stem_oracle_metric(const double* qbar, const double* kbar, const double* vn
     for (int j = 0; j <= i; ++j) {
       double p = exp(mrow[j] - mx) / z;
       mrow[j] = p * vnorm[bg * nb + j];
+    }
+  }
+}
+
+/*
+ * Output-Aware Metric, the pages' additive form ([es] 2.B, [it] 2.B, [nl] OAM,
+ * [fr] 2.B): routing score plus a weighted, clamped log energy of the value,
+ *   M_ij = qbar_i . kbar_j / sqrt(D) + beta * max(0, log(n_j^2)),   j = 0..i,
+ * with n_j the block's V magnitude (pooled as above) standing for ||V_j||.
+ * clamp == 0 drops the max(0, .). beta == 0 gives M = s (the magnitude term is
+ * taken as 0 even where n_j = 0). Same packed layout as stem_oracle_metric.
+ */
+void stem_oracle_metric_additive(const double* qbar, const double* kbar,
+                                 const double* vnorm, int B, int Hq, int Hkv, int nb,
+                                 int D, double beta, int clamp, double* m) {
+  const int G = Hq / Hkv;
+  const int64_t T = (int64_t)nb * (nb + 1) / 2;
+  const double scale = 1.0 / sqrt((double)D);
+  const int64_t rows = (int64_t)B * Hq * nb;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t u = 0; u < rows; ++u) {
+    const int64_t bh = u / nb;
+    const int i = (int)(u % nb);
+    const int64_t b = bh / Hq, h = bh % Hq;
+    const int64_t bg = b * Hkv + h / G;
+    const double* qi = qbar + u * D;
+    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;
+    for (int j = 0; j <= i; ++j) {
+      const double* kj = kbar + (bg * nb + j) * D;
+      double dot = 0.0;
+      for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+      const double n = vnorm[bg * nb + j];
+      double energy = log(n * n);
+      if (clamp && energy < 0.0) energy = 0.0;
+      mrow[j] = dot * scale + (beta == 0.0 ? 0.0 : beta * energy);
     }
   }
 }

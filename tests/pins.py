@@ -9,13 +9,20 @@ What pins what:
   budget     arbitrary-precision (decimal, 60 digits) recomputation of the
              exponential-ratio schedule; closed forms at rho_min = 1 and tau -> 0;
              the invariants k <= i+1, k >= min(i+1, k_min), k(0) = 1, k(i >= 1) >= 2.
+             Linear schedule: two cases worked by hand (tests/golden/
+             budget_linear_hand.txt); mu = 1 is a constant budget; the last block
+             gets ceil(mu * k_start); the unclamped budget never grows with i;
+             exact rational recomputation.
   pooling    closed forms: constant blocks, +x/-x alternating rows (mean of norms
              is not the norm of the mean), arithmetic-progression rows; numpy
-             brute force on random tensors.
+             brute force on random tensors. Max-pooled V: rows of norm r give
+             block-1; numpy brute force.
   metric     Q = 0 gives m_ij = n_j/(i+1); two-block logistic closed form; each
              row of m/n sums to 1; the ranking equals that of the pages' printed
              additive score s_ij + beta*log(n_j^2) at beta = 1/2, no clamp; numpy
-             brute force.
+             brute force. Additive metric: beta = 0 gives the numpy scores; at
+             beta = 1/2 without the clamp, M_ij - log m_ij equals the row's
+             logsumexp (scipy); constant-norm blocks give the clamp's known values.
   selection  all-equal metric keeps {0, 1, ..., k-2, i} (ties to the lower
              index); Q = 0 keeps the top norms; full-sort brute force; structural
              invariants.
@@ -28,7 +35,9 @@ What pins what:
 from __future__ import annotations
 
 import math
+import os
 from decimal import ROUND_CEILING, Decimal, getcontext
+from fractions import Fraction
 
 import numpy as np
 import torch
@@ -146,7 +155,89 @@ def pin_budget_closed_forms():
         assert np.all(k[1:] >= 2)
 
 
+def _hand_linear_cases():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                        "budget_linear_hand.txt")
+    cases = []
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        head, ks = line.split(":")
+        nb, ks0, mu, km = head.split()
+        cases.append((int(nb), float(ks0), float(mu), int(km), [int(x) for x in ks.split()]))
+    return cases
+
+
+def budget_linear_exact(nb, k_start, mu, k_min):
+    """Exact rational k(i) of the linear schedule from the float32-rounded parameters, and the
+    blocks whose unrounded budget lies within 1e-9 of an integer (where double rounding
+    could fall either way)."""
+    ksf = Fraction(float(np.float32(k_start)))
+    muf = Fraction(float(np.float32(mu)))
+    ks, amb = [], set()
+    for i in range(nb):
+        t = Fraction(i, nb - 1) if nb > 1 else Fraction(0)
+        lin = ksf * (1 - (1 - muf) * t)
+        c = math.ceil(lin)
+        if abs(lin - round(lin)) < Fraction(1, 10 ** 9):
+            amb.add(i)
+        kk = min(i + 1, max(k_min, c))
+        ks.append(1 if i == 0 else max(2, kk))
+    return ks, amb
+
+
+def pin_budget_linear():
+    for nb, ks0, mu, km, want in _hand_linear_cases():
+        k, off = oracle.budget_linear(nb, ks0, mu, km)
+        assert list(k) == want, (nb, ks0, mu, km, list(k), want)
+        assert off[nb] == sum(want)
+    # mu = 1: a constant budget ceil(k_start), floored and capped as usual
+    for nb, ks0, km in ((64, 9.5, 1), (300, 40.0, 8), (17, 3.2, 5)):
+        k, _ = oracle.budget_linear(nb, ks0, 1.0, km)
+        for i in range(1, nb):
+            assert k[i] == max(2, min(i + 1, max(km, math.ceil(ks0)))), (nb, ks0, km, i)
+    # the last block gets ceil(mu * k_start) (values chosen away from integers)
+    for nb, ks0, mu in ((1024, 36.0, 0.7), (512, 50.0, 0.35), (100, 90.0, 0.123)):
+        k, _ = oracle.budget_linear(nb, ks0, mu, 1)
+        assert k[nb - 1] == max(2, math.ceil(ks0 * mu)), (nb, ks0, mu, k[nb - 1])
+    # exact recomputation and the invariants
+    for nb, ks0, mu, km in ((1024, 36.0, 0.7, 8), (256, 20.0, 0.5, 4), (1000, 700.0, 0.05, 1),
+                            (2, 5.0, 0.2, 1), (1, 4.0, 0.7, 1)):
+        k, off = oracle.budget_linear(nb, ks0, mu, km)
+        ref, amb = budget_linear_exact(nb, ks0, mu, km)
+        for i in range(nb):
+            if i not in amb:
+                assert k[i] == ref[i], (nb, ks0, mu, km, i, k[i], ref[i])
+        i = np.arange(nb)
+        assert k[0] == 1 and np.all(k <= i + 1) and np.all(k >= np.minimum(i + 1, km))
+        assert np.all(k[1:] >= 2) and off[0] == 0 and np.all(np.diff(off) == k)
+        # where neither the floor nor the cap binds, the budget never grows with i
+        free = [j for j in range(1, nb) if k[j] < j + 1 and k[j] > max(km, 2)]
+        for a_, b_ in zip(free, free[1:]):
+            assert k[b_] <= k[a_], (nb, ks0, mu, km, a_, b_)
+
+
 # --------------------------------------------------------------------------- pooling
+
+
+def pin_pool_max():
+    B, Hkv, S, D, block = 1, 2, 64, 8, 16
+    # row r of each block is r * e_3: largest norm block - 1
+    z = torch.zeros(B, Hkv, S, D)
+    vap = torch.zeros(B, Hkv, S, D)
+    vap[..., 3] = torch.arange(S, dtype=torch.float32) % block
+    _, _, vn = oracle.pool(z, z, vap, block, "max")
+    np.testing.assert_allclose(vn, block - 1.0, rtol=0, atol=1e-12)
+    # random rows against numpy; pooled Q and K do not depend on the V summary
+    for dtype in (torch.float32, torch.bfloat16):
+        q, k, v = _tiny_inputs(13, dtype=dtype)
+        qb1, kb1, _ = oracle.pool(q, k, v, 16)
+        qb2, kb2, vn2 = oracle.pool(q, k, v, 16, "max")
+        V = brute.f64(v)
+        B_, Hkv_, S_, D_ = V.shape
+        want = np.linalg.norm(V, axis=-1).reshape(B_, Hkv_, S_ // 16, 16).max(axis=3)
+        np.testing.assert_allclose(vn2, want, rtol=1e-13)
+        assert np.array_equal(qb1, qb2) and np.array_equal(kb1, kb2)
 
 
 def pin_pool_closed_forms():
@@ -264,6 +355,47 @@ def pin_metric_brute():
                                            rtol=1e-11, atol=1e-15)
 
 
+def pin_metric_additive_closed_forms():
+    from scipy.special import logsumexp
+    q, k, v = _tiny_inputs(31, Hq=4, Hkv=2, S=512, D=32, block=16)
+    qbar, kbar, vnorm = oracle.pool(q, k, v, 16)
+    B, Hq, nb, D = qbar.shape
+    G = Hq // kbar.shape[1]
+    # beta = 0: the routing score alone, from numpy
+    m0 = oracle.metric_additive(qbar, kbar, vnorm, 0.0, True)
+    for h in range(Hq):
+        for i in range(nb):
+            s = qbar[0, h, i] @ kbar[0, h // G, : i + 1].T / math.sqrt(D)
+            np.testing.assert_allclose(oracle.metric_row(m0, 0, h, i), s, rtol=1e-12, atol=1e-14)
+    # beta = 1/2, no clamp: M_ij - log(m_ij) is the row's logsumexp of s (product metric pinned
+    # above; logsumexp from scipy)
+    mh = oracle.metric_additive(qbar, kbar, vnorm, 0.5, False)
+    mp = oracle.metric(qbar, kbar, vnorm)
+    for h in range(Hq):
+        for i in range(nb):
+            s = qbar[0, h, i] @ kbar[0, h // G, : i + 1].T / math.sqrt(D)
+            diff = oracle.metric_row(mh, 0, h, i) - np.log(oracle.metric_row(mp, 0, h, i))
+            np.testing.assert_allclose(diff, logsumexp(s), rtol=1e-11, atol=1e-11)
+    # clamp: V blocks of constant rows with norm 3 (odd blocks) and 0.5 (even blocks); Q = 0
+    # so M = beta * max(0, log n^2): 0.2 * 2 ln 3 and 0 (clamped) or 0.2 * 2 ln 0.5 (not)
+    S, block, Dv = 128, 16, 8
+    nbv = S // block
+    vv = torch.zeros(1, 1, S, Dv)
+    for j in range(nbv):
+        vv[0, 0, j * block:(j + 1) * block, 0] = 3.0 if j % 2 else 0.5
+    z = torch.zeros(1, 1, S, Dv)
+    qb, kb, vn = oracle.pool(z, z, vv, block)
+    beta = float(np.float32(0.2))
+    mc = oracle.metric_additive(qb, kb, vn, 0.2, True)
+    mu_ = oracle.metric_additive(qb, kb, vn, 0.2, False)
+    row_c = oracle.metric_row(mc, 0, 0, nbv - 1)
+    row_u = oracle.metric_row(mu_, 0, 0, nbv - 1)
+    for j in range(nbv):
+        want_c = beta * 2 * math.log(3.0) if j % 2 else 0.0
+        want_u = beta * 2 * math.log(3.0 if j % 2 else 0.5)
+        assert abs(row_c[j] - want_c) < 1e-13 and abs(row_u[j] - want_u) < 1e-13, (j, row_c[j], row_u[j])
+
+
 # --------------------------------------------------------------------------- selection
 
 
@@ -368,8 +500,11 @@ PINS = [
     pin_budget_closed_forms,
     pin_pool_closed_forms,
     pin_pool_brute,
+    pin_pool_max,
+    pin_budget_linear,
     pin_metric_closed_forms,
     pin_metric_additive_equivalence,
+    pin_metric_additive_closed_forms,
     pin_metric_brute,
     pin_select_ties_and_special_cases,
     pin_select_brute_and_invariants,

@@ -20,20 +20,45 @@ SRC = os.path.join(ROOT, "oracle", "stem_oracle.c")
 MUTANTS = [
     ("budget-sign", "exp(-(double)i / tau)", "exp((double)i / tau)"),
     ("budget-index", "ceil(rho * (double)(i + 1))", "ceil(rho * (double)(i))"),
-    ("budget-no-clamp", "if (kk > (double)(i + 1)) kk = (double)(i + 1);", ""),
+    ("budget-no-clamp",
+     "ceil(rho * (double)(i + 1));\n    double kk = want > (double)k_min ? want : (double)k_min;\n"
+     "    if (kk > (double)(i + 1)) kk = (double)(i + 1);",
+     "ceil(rho * (double)(i + 1));\n    double kk = want > (double)k_min ? want : (double)k_min;\n"),
+    ("linear-no-cap",
+     "ceil(k_lin);\n    double kk = want > (double)k_min ? want : (double)k_min;\n"
+     "    if (kk > (double)(i + 1)) kk = (double)(i + 1);",
+     "ceil(k_lin);\n    double kk = want > (double)k_min ? want : (double)k_min;\n"),
+    ("linear-no-floor", "double want = ceil(k_lin);\n    double kk = want > (double)k_min ? want : (double)k_min;",
+     "double want = ceil(k_lin);\n    double kk = want;"),
     ("pool-divisor", "qbar[u * D + d] = acc / block;", "qbar[u * D + d] = acc / (block - 1);"),
-    ("pool-no-sqrt", "nacc += sqrt(sq);", "nacc += sq;"),
+    ("pool-no-sqrt", "const double norm = sqrt(sq);", "const double norm = sq;"),
     ("pool-norm-of-mean", "sq += x * x;", "sq += x;"),
     ("metric-no-scale", "mrow[j] = dot * scale; /* s_ij", "mrow[j] = dot; /* s_ij"),
     ("metric-no-vnorm", "mrow[j] = p * vnorm[bg * nb + j];", "mrow[j] = p;"),
     ("metric-softmax-sign", "z += exp(mrow[j] - mx);", "z += exp(mx - mrow[j]);"),
-    ("metric-gqa", "const int64_t bg = b * Hkv + h / G;", "const int64_t bg = b * Hkv + h % Hkv;"),
+    ("metric-gqa",
+     "const int64_t bg = b * Hkv + h / G;\n    const double* qi = qbar + u * D;\n"
+     "    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;\n    double mx",
+     "const int64_t bg = b * Hkv + h % Hkv;\n    const double* qi = qbar + u * D;\n"
+     "    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;\n    double mx"),
+    ("additive-gqa",
+     "const int64_t bg = b * Hkv + h / G;\n    const double* qi = qbar + u * D;\n"
+     "    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;\n    for",
+     "const int64_t bg = b * Hkv + h % Hkv;\n    const double* qi = qbar + u * D;\n"
+     "    double* mrow = m + bh * T + (int64_t)i * (i + 1) / 2;\n    for"),
     ("select-tie-order", "return (a->j > b->j) - (a->j < b->j);", "return (a->j < b->j) - (a->j > b->j);"),
     ("select-shift", "c[j - 1].m = mrow[j];", "c[j - 1].m = mrow[j - 1];"),
     ("select-no-sink", "chosen[n++] = 0;\n", "chosen[n++] = 1;\n"),
     ("attn-no-causal", "const int last = (j == i) ? r : block - 1;", "const int last = block - 1;"),
     ("attn-no-scale", "logit[nkeys] = dot * scale;", "logit[nkeys] = dot;"),
     ("attn-no-normalise", "const double w = logit[c] / z;", "const double w = logit[c];"),
+    ("linear-denominator", "(double)i / (double)(nb - 1)", "(double)i / (double)nb"),
+    ("linear-direction", "k_start * (1.0 - (1.0 - mu) * t)", "k_start * (mu + (1.0 - mu) * t)"),
+    ("linear-floor", "double want = ceil(k_lin);", "double want = floor(k_lin);"),
+    ("pool-max-is-mean", "vnorm[u] = vmax ? nmax : nacc / block;", "vnorm[u] = nacc / block;"),
+    ("additive-no-clamp", "if (clamp && energy < 0.0) energy = 0.0;", ""),
+    ("additive-no-square", "double energy = log(n * n);", "double energy = log(n);"),
+    ("additive-no-scale", "mrow[j] = dot * scale + (beta", "mrow[j] = dot + (beta"),
 ]
 
 
