@@ -2,9 +2,10 @@
 //
 // Host responsibilities: argument validation (before anything is enqueued), the Token
 // Position-Decay budget in double precision ("Stem: Rethinking Causal Information Flow in
-// Sparse Attention", gist.science/es "Resumen tecnico" 2.A; gist.science/it 2.A; exponential
-// decay per the shd-paper.top "key design" paragraph), a per-parameter plan cache, the
-// workspace carve-up, and the launch sequence pool -> select -> sparse attention.
+// Sparse Attention", gist.science/es "Resumen tecnico" 2.A; gist.science/it 2.A: linear
+// interpolation from k_start to mu * k_start; exponential decay per the shd-paper.top "key
+// design" paragraph), a per-parameter plan cache, the workspace carve-up, and the launch
+// sequence pool -> select -> sparse attention.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -27,18 +28,61 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ budget
 
-bool budget_params_ok(int nb, float rho_min, float tau, int k_min) {
-  return nb >= 0 && std::isfinite(rho_min) && rho_min > 0.0f && rho_min <= 1.0f &&
-         std::isfinite(tau) && tau > 0.0f && k_min >= 1;
+stem_method_t default_method(float rho_min, float tau, int k_min) {
+  stem_method_t m;
+  std::memset(&m, 0, sizeof m);
+  m.schedule = STEM_SCHED_EXP;
+  m.rho_min = rho_min;
+  m.tau = tau;
+  m.mu = 1.0f;
+  m.k_min = k_min;
+  m.metric = STEM_METRIC_PRODUCT;
+  m.clamp = 1;
+  m.vsum = STEM_VSUM_MEAN;
+  return m;
 }
 
-// k(i) = min(i+1, max(k_min, ceil(rho(i) (i+1)))), rho(i) = rho_min + (1-rho_min) e^{-i/tau};
-// block 0 alone at i = 0, at least the sink and the diagonal for i >= 1.
-int budget_k(int i, double rho_min, double tau, int k_min) {
+bool method_ok(int nb, const stem_method_t& m) {
+  if (nb < 0 || m.k_min < 1) return false;
+  if (m.schedule == STEM_SCHED_EXP) {
+    if (!(std::isfinite(m.rho_min) && m.rho_min > 0.0f && m.rho_min <= 1.0f &&
+          std::isfinite(m.tau) && m.tau > 0.0f))
+      return false;
+  } else if (m.schedule == STEM_SCHED_LINEAR) {
+    if (!(std::isfinite(m.k_start) && m.k_start > 0.0f && std::isfinite(m.mu) && m.mu > 0.0f &&
+          m.mu <= 1.0f))
+      return false;
+  } else {
+    return false;
+  }
+  if (m.metric == STEM_METRIC_ADDITIVE) {
+    if (!(std::isfinite(m.beta) && m.beta >= 0.0f) || (m.clamp != 0 && m.clamp != 1))
+      return false;
+  } else if (m.metric != STEM_METRIC_PRODUCT) {
+    return false;
+  }
+  return m.vsum == STEM_VSUM_MEAN || m.vsum == STEM_VSUM_MAX;
+}
+
+// Exponential: k(i) = min(i+1, max(k_min, ceil(rho(i) (i+1)))), rho(i) = rho_min + (1-rho_min)
+// e^{-i/tau}. Linear: k(i) = min(i+1, max(k_min, ceil(k_start (1 - (1-mu) i/(nb-1))))), the
+// interpolation from k_start at the first query block to mu * k_start at the last. Block 0
+// alone at i = 0, at least the sink and the diagonal for i >= 1.
+int budget_k(int i, int nb, const stem_method_t& m) {
   if (i == 0) return 1;
-  const double rho = rho_min + (1.0 - rho_min) * std::exp(-static_cast<double>(i) / tau);
-  const double want = std::ceil(rho * static_cast<double>(i + 1));
-  double kk = std::max(want, static_cast<double>(k_min));
+  double want;
+  if (m.schedule == STEM_SCHED_LINEAR) {
+    const double t = nb > 1 ? static_cast<double>(i) / static_cast<double>(nb - 1) : 0.0;
+    const double k_lin =
+        static_cast<double>(m.k_start) * (1.0 - (1.0 - static_cast<double>(m.mu)) * t);
+    want = std::ceil(k_lin);
+  } else {
+    const double rho_min = m.rho_min;
+    const double rho =
+        rho_min + (1.0 - rho_min) * std::exp(-static_cast<double>(i) / static_cast<double>(m.tau));
+    want = std::ceil(rho * static_cast<double>(i + 1));
+  }
+  double kk = std::max(want, static_cast<double>(m.k_min));
   kk = std::min(kk, static_cast<double>(i + 1));
   return std::max(2, static_cast<int>(kk));
 }
@@ -50,7 +94,7 @@ struct Plan {
   size_t bytes = 0;
 };
 
-using PlanKey = std::tuple<int, uint32_t, uint32_t, int>;
+using PlanKey = std::tuple<int, int, uint32_t, uint32_t, int>;
 std::mutex g_plan_mu;
 std::map<PlanKey, Plan> g_plans;
 
@@ -63,9 +107,11 @@ uint32_t fbits(float f) {
 size_t plan_bytes(int nb) { return align_up(sizeof(int32_t) * (3 * static_cast<size_t>(nb) + 1)); }
 
 // Returns the cached plan (building it on first use), or nullptr on a pinned-allocation failure.
-const Plan* get_plan(int nb, float rho_min, float tau, int k_min) {
+const Plan* get_plan(int nb, const stem_method_t& m) {
   std::lock_guard<std::mutex> lock(g_plan_mu);
-  const PlanKey key{nb, fbits(rho_min), fbits(tau), k_min};
+  const bool lin = m.schedule == STEM_SCHED_LINEAR;
+  const PlanKey key{nb, m.schedule, fbits(lin ? m.k_start : m.rho_min), fbits(lin ? m.mu : m.tau),
+                    m.k_min};
   auto it = g_plans.find(key);
   if (it != g_plans.end()) return &it->second;
   Plan p;
@@ -81,7 +127,7 @@ const Plan* get_plan(int nb, float rho_min, float tau, int k_min) {
   int32_t* order = off + nb + 1;
   int64_t tot = 0;
   for (int i = 0; i < nb; ++i) {
-    k[i] = budget_k(i, rho_min, tau, k_min);
+    k[i] = budget_k(i, nb, m);
     off[i] = static_cast<int32_t>(tot);
     tot += k[i];
   }
@@ -141,12 +187,26 @@ int check_shape(int B, int Hq, int Hkv, int S, int D, int block, int dtype) {
 
 bool is_empty(int B, int S) { return B == 0 || S == 0; }
 
-int check_params(int nb, float rho_min, float tau, int k_min) {
-  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
+int64_t capacity(int nb, const stem_method_t& m) {
+  int64_t tot = 0;
+  for (int i = 0; i < nb; ++i) tot += budget_k(i, nb, m);
+  return tot;
+}
+
+int check_params(int nb, const stem_method_t& m) {
+  if (!method_ok(nb, m)) return STEM_ERR_ARG;
   // off[] is int32: the capacity must fit
-  const int64_t cap = stem_sel_capacity(nb, rho_min, tau, k_min);
-  if (cap < 0 || cap > 0x7fffffffLL) return STEM_ERR_UNSUPPORTED;
+  const int64_t cap = capacity(nb, m);
+  if (cap > 0x7fffffffLL) return STEM_ERR_UNSUPPORTED;
   return STEM_OK;
+}
+
+SelMetric sel_metric(const stem_method_t& m) {
+  SelMetric s;
+  s.additive = m.metric == STEM_METRIC_ADDITIVE;
+  s.beta = m.beta;
+  s.clamp = m.clamp != 0;
+  return s;
 }
 
 int cuda_err(cudaError_t e) {
@@ -170,12 +230,17 @@ int elem_size(int dtype) { return dtype == STEM_BF16 ? 2 : 4; }
 
 // ------------------------------------------------------------------ the path
 
+stem_method_t args_method(const stem_args_t* a) {
+  return a->method ? *a->method : default_method(a->rho_min, a->tau, a->k_min);
+}
+
 int run_prefill(const stem_args_t* a, cudaStream_t st) {
   if (a == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(a->B, a->Hq, a->Hkv, a->S, a->D, a->block, a->dtype);
   if (rc != STEM_OK) return rc;
   const int nb = a->S / a->block;
-  rc = check_params(nb, a->rho_min, a->tau, a->k_min);
+  const stem_method_t m = args_method(a);
+  rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
   if (is_empty(a->B, a->S)) return STEM_OK;
   if (!a->q || !a->k || !a->v || !a->out || !a->sel_idx || !a->sel_cnt) return STEM_ERR_ARG;
@@ -185,7 +250,7 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D);
   if (a->workspace == nullptr || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total)
     return STEM_ERR_WORKSPACE;
-  const Plan* plan = get_plan(nb, a->rho_min, a->tau, a->k_min);
+  const Plan* plan = get_plan(nb, m);
   if (plan == nullptr) return STEM_ERR_CUDA;
 
   auto* ws = static_cast<unsigned char*>(a->workspace);
@@ -205,11 +270,11 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   };
   if ((rc = mark(0)) != STEM_OK) return rc;
   rc = cuda_err(launch_pool(a->q, a->k, a->v, a->dtype, a->B, a->Hq, a->Hkv, a->S, a->D,
-                            a->block, qbar, kbar, vnorm, st));
+                            a->block, m.vsum == STEM_VSUM_MAX, qbar, kbar, vnorm, st));
   if (rc != STEM_OK) return rc;
   if ((rc = mark(1)) != STEM_OK) return rc;
   rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, plan->cap,
-                              a->sel_idx, a->sel_cnt, nullptr, st));
+                              sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st));
   if (rc != STEM_OK) return rc;
   if ((rc = mark(2)) != STEM_OK) return rc;
   if (a->dtype == STEM_BF16) {
@@ -281,11 +346,11 @@ using namespace stem;
 
 extern "C" {
 
-int stem_budget(int nb, float rho_min, float tau, int k_min, int32_t* k_out, int32_t* off_out) {
-  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
+int stem_budget_m(int nb, const stem_method_t* m, int32_t* k_out, int32_t* off_out) {
+  if (m == nullptr || !method_ok(nb, *m)) return STEM_ERR_ARG;
   int64_t tot = 0;
   for (int i = 0; i < nb; ++i) {
-    const int k = budget_k(i, rho_min, tau, k_min);
+    const int k = budget_k(i, nb, *m);
     if (off_out) off_out[i] = static_cast<int32_t>(tot);
     if (k_out) k_out[i] = k;
     tot += k;
@@ -295,11 +360,19 @@ int stem_budget(int nb, float rho_min, float tau, int k_min, int32_t* k_out, int
   return STEM_OK;
 }
 
+int stem_budget(int nb, float rho_min, float tau, int k_min, int32_t* k_out, int32_t* off_out) {
+  const stem_method_t m = default_method(rho_min, tau, k_min);
+  return stem_budget_m(nb, &m, k_out, off_out);
+}
+
+int64_t stem_sel_capacity_m(int nb, const stem_method_t* m) {
+  if (m == nullptr || !method_ok(nb, *m)) return STEM_ERR_ARG;
+  return capacity(nb, *m);
+}
+
 int64_t stem_sel_capacity(int nb, float rho_min, float tau, int k_min) {
-  if (!budget_params_ok(nb, rho_min, tau, k_min)) return STEM_ERR_ARG;
-  int64_t tot = 0;
-  for (int i = 0; i < nb; ++i) tot += budget_k(i, rho_min, tau, k_min);
-  return tot;
+  const stem_method_t m = default_method(rho_min, tau, k_min);
+  return stem_sel_capacity_m(nb, &m);
 }
 
 size_t stem_workspace_size(int B, int Hq, int Hkv, int S, int D, int block) {
@@ -348,7 +421,7 @@ int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int
   int rc = check_shape(B, Hq, Hkv, S, D, block, STEM_BF16);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, S)) return run_prefill(&a, nullptr);
-  rc = check_params(S / block, rho_min, tau, k_min);
+  rc = check_params(S / block, default_method(rho_min, tau, k_min));
   if (rc != STEM_OK) return rc;
   a.workspace_bytes = stem_workspace_size(B, Hq, Hkv, S, D, block);
   rc = get_scratch(a.workspace_bytes, &a.workspace, 0);
@@ -361,14 +434,15 @@ int stem_prefill_host(const stem_args_t* h) {
   int rc = check_shape(h->B, h->Hq, h->Hkv, h->S, h->D, h->block, h->dtype);
   if (rc != STEM_OK) return rc;
   const int nb = h->S / h->block;
-  rc = check_params(nb, h->rho_min, h->tau, h->k_min);
+  const stem_method_t m = args_method(h);
+  rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
   if (is_empty(h->B, h->S)) return STEM_OK;
   if (!h->q || !h->k || !h->v || !h->out || !h->sel_idx || !h->sel_cnt) return STEM_ERR_ARG;
   const size_t es = elem_size(h->dtype);
   const size_t qb = es * static_cast<size_t>(h->B) * h->Hq * h->S * h->D;
   const size_t kvb = es * static_cast<size_t>(h->B) * h->Hkv * h->S * h->D;
-  const int64_t cap = stem_sel_capacity(nb, h->rho_min, h->tau, h->k_min);
+  const int64_t cap = capacity(nb, m);
   const size_t sib = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * cap;
   const size_t scb = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * nb;
   const Layout L = layout(h->B, h->Hq, h->Hkv, nb, h->D);
@@ -416,8 +490,10 @@ int stem_prefill_host(const stem_args_t* h) {
   return status < 0 ? status : STEM_OK;
 }
 
-int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
-              int S, int D, int block, float* qbar, float* kbar, float* vnorm, void* stream) {
+int stem_pool_m(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+                int S, int D, int block, const stem_method_t* m, float* qbar, float* kbar,
+                float* vnorm, void* stream) {
+  if (m == nullptr || (m->vsum != STEM_VSUM_MEAN && m->vsum != STEM_VSUM_MAX)) return STEM_ERR_ARG;
   int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, S)) return STEM_OK;
@@ -425,20 +501,26 @@ int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(qbar, 16) ||
       !aligned(kbar, 16) || !aligned(vnorm, 4))
     return STEM_ERR_ARG;
-  return cuda_err(launch_pool(q, k, v, dtype, B, Hq, Hkv, S, D, block, qbar, kbar, vnorm,
-                              static_cast<cudaStream_t>(stream)));
+  return cuda_err(launch_pool(q, k, v, dtype, B, Hq, Hkv, S, D, block, m->vsum == STEM_VSUM_MAX,
+                              qbar, kbar, vnorm, static_cast<cudaStream_t>(stream)));
 }
 
-int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
-                int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
-                int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
-                void* stream) {
-  if (nb < 0) return STEM_ERR_ARG;
+int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+              int S, int D, int block, float* qbar, float* kbar, float* vnorm, void* stream) {
+  const stem_method_t m = default_method(1.0f, 1.0f, 1);
+  return stem_pool_m(q, k, v, dtype, B, Hq, Hkv, S, D, block, &m, qbar, kbar, vnorm, stream);
+}
+
+int stem_select_m(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                  int Hkv, int nb, int D, const stem_method_t* m, int32_t* sel_idx,
+                  int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (nb < 0 || m == nullptr) return STEM_ERR_ARG;
   if (nb > STEM_MAX_NB) return STEM_ERR_UNSUPPORTED;
   // the selection sees blocks only: validate as a shape with block 64
   int rc = check_shape(B, Hq, Hkv, nb * 64, D, 64, STEM_F32);
   if (rc != STEM_OK) return rc;
-  rc = check_params(nb, rho_min, tau, k_min);
+  rc = check_params(nb, *m);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, nb)) return STEM_OK;
   if (!qbar || !kbar || !vnorm || !sel_idx || !sel_cnt) return STEM_ERR_ARG;
@@ -448,24 +530,34 @@ int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B,
   const Layout L = layout(B, Hq, Hkv, nb, D);
   if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.plan + plan_bytes(nb))
     return STEM_ERR_WORKSPACE;
-  const Plan* plan = get_plan(nb, rho_min, tau, k_min);
+  const Plan* plan = get_plan(nb, *m);
   if (plan == nullptr) return STEM_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   PlanDev pd;
   rc = upload_plan(plan, workspace, L, st, &pd);
   if (rc != STEM_OK) return rc;
-  return cuda_err(launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, plan->cap, sel_idx,
-                                sel_cnt, m_out, st));
+  return cuda_err(launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, plan->cap,
+                                sel_metric(*m), sel_idx, sel_cnt, m_out, st));
 }
 
-int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
-                     int Hkv, int S, int D, int block, float rho_min, float tau, int k_min,
-                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
-                     size_t workspace_bytes, int32_t* status, void* stream) {
+int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
+                int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  const stem_method_t m = default_method(rho_min, tau, k_min);
+  return stem_select_m(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, &m, sel_idx, sel_cnt, m_out,
+                       workspace, workspace_bytes, stream);
+}
+
+int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                       int Hkv, int S, int D, int block, const stem_method_t* m,
+                       const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
+                       void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  if (m == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
   if (rc != STEM_OK) return rc;
   const int nb = S / block;
-  rc = check_params(nb, rho_min, tau, k_min);
+  rc = check_params(nb, *m);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, S)) return STEM_OK;
   if (!q || !k || !v || !out || !sel_idx || !sel_cnt) return STEM_ERR_ARG;
@@ -475,7 +567,7 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
   const Layout L = layout(B, Hq, Hkv, nb, D);
   if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.sched_end)
     return STEM_ERR_WORKSPACE;
-  const Plan* plan = get_plan(nb, rho_min, tau, k_min);
+  const Plan* plan = get_plan(nb, *m);
   if (plan == nullptr) return STEM_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (status) {
@@ -494,6 +586,15 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
   return cuda_err(launch_attn_f32(static_cast<const float*>(q), static_cast<const float*>(k),
                                   static_cast<const float*>(v), B, Hq, Hkv, S, D, block, pd,
                                   plan->cap, sel_idx, sel_cnt, static_cast<float*>(out), st));
+}
+
+int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                     int Hkv, int S, int D, int block, float rho_min, float tau, int k_min,
+                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
+                     size_t workspace_bytes, int32_t* status, void* stream) {
+  const stem_method_t m = default_method(rho_min, tau, k_min);
+  return stem_sparse_attn_m(q, k, v, dtype, B, Hq, Hkv, S, D, block, &m, sel_idx, sel_cnt, out,
+                            workspace, workspace_bytes, status, stream);
 }
 
 }  // extern "C"

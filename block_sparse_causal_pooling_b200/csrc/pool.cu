@@ -4,7 +4,8 @@
 // "Implementatie" step 1). Mean pooling is the reading used:
 //   qbar[b,h,i,:] = mean of Q rows i*block .. i*block+block-1,
 //   kbar[b,g,i,:] = mean of K rows of block i,
-//   vnorm[b,g,i]  = mean over the block's rows of the row's Euclidean norm.
+//   vnorm[b,g,i]  = mean over the block's rows of the row's Euclidean norm, or (vmax) the
+//                   largest row norm ("maximised magnitudes of V", gist.science/nl step 1).
 //
 // Design (HBM-bound: every input byte is read once, outputs are ~1/64 of the input):
 //   - one CTA of 256 threads per (tensor, b, head, block) unit; a unit is one contiguous
@@ -63,7 +64,7 @@ template <typename T, int D, int BLOCK>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict__ q,
                                                             const T* __restrict__ k,
                                                             const T* __restrict__ v, int nq,
-                                                            int nk, int nb, int S,
+                                                            int nk, int nb, int S, int vmax,
                                                             float* __restrict__ qbar,
                                                             float* __restrict__ kbar,
                                                             float* __restrict__ vnorm) {
@@ -141,21 +142,29 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict_
       for (int o = CPR / 2; o >= 1; o /= 2) sq += __shfl_xor_sync(0xffffffffu, sq, o, CPR);
       norms[it] = sqrtf(sq);
     }
-    const float mine = pairwise<ITERS>(norms);
+    float mine;
+    if (vmax) {
+      mine = norms[0];
+#pragma unroll
+      for (int it = 1; it < ITERS; ++it) mine = fmaxf(mine, norms[it]);
+    } else {
+      mine = pairwise<ITERS>(norms);
+    }
     if (c == 0) part[rg][0] = mine;
     __syncthreads();
 #pragma unroll
     for (int s = RPI / 2; s >= 1; s /= 2) {
-      if (t < s) part[t][0] = part[t][0] + part[t + s][0];
+      if (t < s) part[t][0] = vmax ? fmaxf(part[t][0], part[t + s][0]) : part[t][0] + part[t + s][0];
       __syncthreads();
     }
-    if (t == 0) vnorm[unit] = part[0][0] * (1.0f / BLOCK);
+    if (t == 0) vnorm[unit] = vmax ? part[0][0] : part[0][0] * (1.0f / BLOCK);
   }
 }
 
 template <typename T, int D, int BLOCK>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                         int S, float* qbar, float* kbar, float* vnorm, cudaStream_t st) {
+                         int S, bool vmax, float* qbar, float* kbar, float* vnorm,
+                         cudaStream_t st) {
   const int nb = S / BLOCK;
   const int64_t nq = static_cast<int64_t>(B) * Hq * nb;
   const int64_t nk = static_cast<int64_t>(B) * Hkv * nb;
@@ -164,34 +173,34 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, int B, int
   if (units > 0x7fffffff) return cudaErrorInvalidConfiguration;
   pool_kernel<T, D, BLOCK><<<static_cast<unsigned>(units), kPoolThreads, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-      static_cast<int>(nq), static_cast<int>(nk), nb, S, qbar, kbar, vnorm);
+      static_cast<int>(nq), static_cast<int>(nk), nb, S, vmax ? 1 : 0, qbar, kbar, vnorm);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_dispatch(const void* q, const void* k, const void* v, int B, int Hq,
-                            int Hkv, int S, int D, int block, float* qbar, float* kbar,
+                            int Hkv, int S, int D, int block, bool vmax, float* qbar, float* kbar,
                             float* vnorm, cudaStream_t st) {
   if (D == 128 && block == 128)
-    return launch_typed<T, 128, 128>(q, k, v, B, Hq, Hkv, S, qbar, kbar, vnorm, st);
+    return launch_typed<T, 128, 128>(q, k, v, B, Hq, Hkv, S, vmax, qbar, kbar, vnorm, st);
   if (D == 128 && block == 64)
-    return launch_typed<T, 128, 64>(q, k, v, B, Hq, Hkv, S, qbar, kbar, vnorm, st);
+    return launch_typed<T, 128, 64>(q, k, v, B, Hq, Hkv, S, vmax, qbar, kbar, vnorm, st);
   if (D == 64 && block == 128)
-    return launch_typed<T, 64, 128>(q, k, v, B, Hq, Hkv, S, qbar, kbar, vnorm, st);
+    return launch_typed<T, 64, 128>(q, k, v, B, Hq, Hkv, S, vmax, qbar, kbar, vnorm, st);
   if (D == 64 && block == 64)
-    return launch_typed<T, 64, 64>(q, k, v, B, Hq, Hkv, S, qbar, kbar, vnorm, st);
+    return launch_typed<T, 64, 64>(q, k, v, B, Hq, Hkv, S, vmax, qbar, kbar, vnorm, st);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 cudaError_t launch_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
-                        int Hkv, int S, int D, int block, float* qbar, float* kbar,
+                        int Hkv, int S, int D, int block, bool vmax, float* qbar, float* kbar,
                         float* vnorm, cudaStream_t st) {
   if (dtype == 0)
-    return launch_dispatch<__nv_bfloat16>(q, k, v, B, Hq, Hkv, S, D, block, qbar, kbar, vnorm,
-                                          st);
-  return launch_dispatch<float>(q, k, v, B, Hq, Hkv, S, D, block, qbar, kbar, vnorm, st);
+    return launch_dispatch<__nv_bfloat16>(q, k, v, B, Hq, Hkv, S, D, block, vmax, qbar, kbar,
+                                          vnorm, st);
+  return launch_dispatch<float>(q, k, v, B, Hq, Hkv, S, D, block, vmax, qbar, kbar, vnorm, st);
 }
 
 }  // namespace stem

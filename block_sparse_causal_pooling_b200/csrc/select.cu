@@ -12,6 +12,10 @@
 // ranks exactly like m_ij; the kernel ranks by key_ij in double (s_ij from a float32 dot
 // product, ln n_j in double) and never materialises m unless asked for it.
 //
+// The pages' additive form (es 2.B, it 2.B, nl OAM, fr 2.B) ranks by
+//   key_ij = s_ij + beta * e_j,   e_j = log(n_j^2) = 2 ln n_j, clamped at 0 (max(0, .)) on request,
+// the same machinery with another per-column term (e_j is not evaluated when beta = 0).
+//
 // Kept set of row i: {0, i} plus the k(i)-2 largest key_ij over j in [1, i-1], larger first,
 // equal keys to the lower j. Written ascending into the CSR slot of row (b, h, i).
 //
@@ -44,7 +48,7 @@ struct SelSmem {
   float* s;       // [R][ldS] scaled logits
   float* qs;      // [R][D]
   float* ks;      // [kTileJ][D+4]
-  double* lnn;    // [ldS]
+  double* lnn;    // [ldS] per-column term of the key: ln n_j, or beta * e_j (additive)
   int* hist;      // [kWarps][256]
 };
 
@@ -52,7 +56,7 @@ template <int D, int R>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(
     const float* __restrict__ qbar, const float* __restrict__ kbar,
     const float* __restrict__ vnorm, int BH, int Hq, int Hkv, int nb, int ldS, PlanDev plan,
-    int64_t cap, int32_t* __restrict__ sel_idx, int32_t* __restrict__ sel_cnt,
+    int64_t cap, SelMetric metric, int32_t* __restrict__ sel_idx, int32_t* __restrict__ sel_cnt,
     float* __restrict__ m_out) {
   constexpr int RPW = R / kWarps;  // rows per warp in phase 1
   constexpr int KLD = D + 4;       // padded kbar row (conflict-free 16-byte column reads)
@@ -85,7 +89,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     if (r < rows) val = reinterpret_cast<const float4*>(qsrc + r * D)[c4];
     reinterpret_cast<float4*>(sm.qs + r * D)[c4] = val;
   }
-  for (int j = t; j < jend; j += kSelThreads) sm.lnn[j] = log(static_cast<double>(nsrc[j]));
+  for (int j = t; j < jend; j += kSelThreads) {
+    double c;
+    if (!metric.additive) {
+      c = log(static_cast<double>(nsrc[j]));
+    } else if (metric.beta == 0.f) {
+      c = 0.0;
+    } else {
+      double e = 2.0 * log(static_cast<double>(nsrc[j]));
+      if (metric.clamp && e < 0.0) e = 0.0;
+      c = static_cast<double>(metric.beta) * e;
+    }
+    sm.lnn[j] = c;
+  }
 
   const float scale = rsqrtf(static_cast<float>(D));
   // ---- phase 1: s[r][j] for r < rows, j < jend
@@ -139,7 +155,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     int32_t* dst = sel_idx + static_cast<int64_t>(bh) * cap + plan.off[i];
     if (lane == 0) sel_cnt[static_cast<int64_t>(bh) * nb + i] = kk;
 
-    if (m_out != nullptr) {  // diagnostic metric row, float32 softmax
+    if (m_out != nullptr && metric.additive) {  // diagnostic metric row: M_ij = s_ij + beta e_j
+      float* mrow = m_out + static_cast<int64_t>(bh) * (static_cast<int64_t>(nb) * (nb + 1) / 2) +
+                    static_cast<int64_t>(i) * (i + 1) / 2;
+      for (int j = lane; j <= i; j += 32)
+        mrow[j] = static_cast<float>(static_cast<double>(srow[j]) + sm.lnn[j]);
+    } else if (m_out != nullptr) {  // diagnostic metric row, float32 softmax
       float mx = -INFINITY;
       for (int j = lane; j <= i; j += 32) mx = fmaxf(mx, srow[j]);
 #pragma unroll
@@ -282,8 +303,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 
 template <int D, int R>
 cudaError_t launch_rt(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
-                      int Hkv, int nb, PlanDev plan, int64_t cap, int32_t* sel_idx,
-                      int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+                      int Hkv, int nb, PlanDev plan, int64_t cap, SelMetric metric,
+                      int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st) {
   const int ldS = (nb + 3) & ~3;
   const size_t smem = sizeof(float) * (static_cast<size_t>(R) * ldS + R * D + kTileJ * (D + 4)) +
                       sizeof(double) * ldS + sizeof(int) * kWarps * 256;
@@ -295,37 +316,38 @@ cudaError_t launch_rt(const float* qbar, const float* kbar, const float* vnorm, 
   const int64_t grid = static_cast<int64_t>(BH) * ((nb + R - 1) / R);
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(grid), kSelThreads, smem, st>>>(qbar, kbar, vnorm, BH, Hq, Hkv,
-                                                             nb, ldS, plan, cap, sel_idx,
-                                                             sel_cnt, m_out);
+                                                             nb, ldS, plan, cap, metric,
+                                                             sel_idx, sel_cnt, m_out);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
-                     int Hkv, int nb, PlanDev plan, int64_t cap, int32_t* sel_idx,
-                     int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+                     int Hkv, int nb, PlanDev plan, int64_t cap, SelMetric metric,
+                     int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st) {
   if (nb <= 1024)
-    return launch_rt<D, 32>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt,
-                            m_out, st);
+    return launch_rt<D, 32>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                            sel_cnt, m_out, st);
   if (nb <= 2048)
-    return launch_rt<D, 16>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt,
-                            m_out, st);
-  return launch_rt<D, 8>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
-                         st);
+    return launch_rt<D, 16>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                            sel_cnt, m_out, st);
+  return launch_rt<D, 8>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt,
+                         m_out, st);
 }
 
 }  // namespace
 
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
-                          int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+                          SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
+                          cudaStream_t st) {
   if (B * Hq == 0 || nb == 0) return cudaSuccess;
   if (D == 128)
-    return launch_d<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
-                         st);
+    return launch_d<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt,
+                         m_out, st);
   if (D == 64)
-    return launch_d<64>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, sel_idx, sel_cnt, m_out,
-                        st);
+    return launch_d<64>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt,
+                        m_out, st);
   return cudaErrorInvalidValue;
 }
 

@@ -93,7 +93,7 @@ extern "C" int stem_select_static(const float* qbar, const float* kbar, const fl
   }
   const int32_t* dk = static_cast<const int32_t*>(g_static_addr[dev]);
   PlanDev pd{dk, dk + nb, dk + 2 * nb + 1};
-  const cudaError_t e = launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, cap, sel_idx,
+  const cudaError_t e = launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, cap, SelMetric{}, sel_idx,
                                       sel_cnt, nullptr, st);
   if (e != cudaSuccess) {
     cudaGetLastError();

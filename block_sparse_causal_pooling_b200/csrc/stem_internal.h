@@ -13,15 +13,25 @@ struct PlanDev {
   const int32_t* order;  // [nb]   query blocks sorted by k(i) descending (heaviest first)
 };
 
-// Block pooling (pool.cu). dtype: 0 bf16, 1 f32.
+// Block pooling (pool.cu). dtype: 0 bf16, 1 f32. vmax: vnorm is the largest V-row norm of the
+// block instead of the mean.
 cudaError_t launch_pool(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
-                        int Hkv, int S, int D, int block, float* qbar, float* kbar,
+                        int Hkv, int S, int D, int block, bool vmax, float* qbar, float* kbar,
                         float* vnorm, cudaStream_t st);
+
+// Block metric of the selection: product (rank by s + ln n) or additive (rank by
+// s + beta * e, e = 2 ln n clamped at 0 when clamp).
+struct SelMetric {
+  bool additive = false;
+  float beta = 0.f;
+  bool clamp = true;
+};
 
 // Metric + top-k selection (select.cu).
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
-                          int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st);
+                          SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
+                          cudaStream_t st);
 
 // Block-sparse attention, bfloat16 inputs on the tensor cores (attn_sm100.cu; block 64 falls to
 // the mma.sync kernel of attn_bf16.cu). `sched` is workspace of pairs_bytes() for the head-pair

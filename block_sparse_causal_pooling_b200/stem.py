@@ -27,12 +27,41 @@ STEM_ERR_UNSUPPORTED = -5
 STEM_BF16 = 0
 STEM_F32 = 1
 STEM_MAX_NB = 4096
+STEM_SCHED_EXP = 0
+STEM_SCHED_LINEAR = 1
+STEM_METRIC_PRODUCT = 0
+STEM_METRIC_ADDITIVE = 1
+STEM_VSUM_MEAN = 0
+STEM_VSUM_MAX = 1
 
 
 class StemError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
         super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+class stem_method_t(ctypes.Structure):
+    _fields_ = [
+        ("schedule", ctypes.c_int32), ("rho_min", ctypes.c_float), ("tau", ctypes.c_float),
+        ("k_start", ctypes.c_float), ("mu", ctypes.c_float), ("k_min", ctypes.c_int32),
+        ("metric", ctypes.c_int32), ("beta", ctypes.c_float), ("clamp", ctypes.c_int32),
+        ("vsum", ctypes.c_int32),
+    ]
+
+
+def make_method(schedule: str = "exp", rho_min: float = 1.0, tau: float = 1.0,
+                k_start: float = 1.0, mu: float = 1.0, k_min: int = 1, metric: str = "product",
+                beta: float = 0.0, clamp: bool = True, vsum: str = "mean") -> stem_method_t:
+    """Method parameters (stem_method_t): schedule "exp" (rho_min, tau) or "linear" (k_start,
+    mu); metric "product" or "additive" (beta, clamp); vsum "mean" or "max"."""
+    m = stem_method_t()
+    m.schedule = {"exp": STEM_SCHED_EXP, "linear": STEM_SCHED_LINEAR}[schedule]
+    m.rho_min, m.tau, m.k_start, m.mu, m.k_min = rho_min, tau, k_start, mu, k_min
+    m.metric = {"product": STEM_METRIC_PRODUCT, "additive": STEM_METRIC_ADDITIVE}[metric]
+    m.beta, m.clamp = beta, int(bool(clamp))
+    m.vsum = {"mean": STEM_VSUM_MEAN, "max": STEM_VSUM_MAX}[vsum]
+    return m
 
 
 class stem_args_t(ctypes.Structure):
@@ -46,6 +75,7 @@ class stem_args_t(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("status", ctypes.c_void_p),
         ("events", ctypes.POINTER(ctypes.c_void_p)),
+        ("method", ctypes.POINTER(stem_method_t)),
     ]
 
 
@@ -56,6 +86,7 @@ def _load() -> ctypes.CDLL:
             "`python -m block_sparse_causal_pooling_b200.build` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    M = ctypes.POINTER(stem_method_t)
     sig = {
         "stem_prefill": (I, [P, P, P, I, I, I, I, I, I, F, F, I, P, P, P]),
         "stem_prefill_ex": (I, [ctypes.POINTER(stem_args_t), P]),
@@ -68,6 +99,11 @@ def _load() -> ctypes.CDLL:
         "stem_select": (I, [P, P, P, I, I, I, I, I, F, F, I, P, P, P, P, Z, P]),
         "stem_sparse_attn": (I, [P, P, P, I, I, I, I, I, I, I, F, F, I, P, P, P, P, Z, P, P]),
         "stem_select_static": (I, [P, P, P, I, I, I, I, I, F, F, I, P, P, P]),
+        "stem_budget_m": (I, [I, M, P, P]),
+        "stem_sel_capacity_m": (ctypes.c_int64, [I, M]),
+        "stem_pool_m": (I, [P, P, P, I, I, I, I, I, I, I, M, P, P, P, P]),
+        "stem_select_m": (I, [P, P, P, I, I, I, I, I, M, P, P, P, P, Z, P]),
+        "stem_sparse_attn_m": (I, [P, P, P, I, I, I, I, I, I, I, M, P, P, P, P, Z, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -81,7 +117,8 @@ _lib = _load()
 # Every symbol include/stem.h declares.
 EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget",
             "stem_sel_capacity", "stem_workspace_size", "stem_strerror", "stem_pool",
-            "stem_select", "stem_sparse_attn", "stem_select_static")
+            "stem_select", "stem_sparse_attn", "stem_budget_m", "stem_sel_capacity_m",
+            "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_select_static")
 
 
 def lib() -> ctypes.CDLL:
@@ -126,11 +163,22 @@ def stem_budget(nb: int, rho_min: float, tau: float, k_min: int):
     return k[:nb].clone(), off
 
 
-def stem_sel_capacity(nb: int, rho_min: float, tau: float, k_min: int) -> int:
-    cap = int(_lib.stem_sel_capacity(nb, rho_min, tau, k_min))
+def stem_sel_capacity(nb: int, rho_min: float, tau: float, k_min: int, method=None) -> int:
+    if method is not None:
+        cap = int(_lib.stem_sel_capacity_m(nb, ctypes.byref(method)))
+    else:
+        cap = int(_lib.stem_sel_capacity(nb, rho_min, tau, k_min))
     if cap < 0:
         raise StemError(cap, "stem_sel_capacity")
     return cap
+
+
+def stem_budget_m(nb: int, method: stem_method_t):
+    """(k [nb] int32, off [nb+1] int32) of the budget of `method` (host)."""
+    k = torch.zeros(max(nb, 1), dtype=torch.int32)
+    off = torch.zeros(nb + 1, dtype=torch.int32)
+    _check(_lib.stem_budget_m(nb, ctypes.byref(method), _ptr(k), _ptr(off)), "stem_budget_m")
+    return k[:nb].clone(), off
 
 
 def stem_workspace_size(B: int, Hq: int, Hkv: int, S: int, D: int, block: int) -> int:
@@ -146,11 +194,11 @@ def _shape(q: torch.Tensor, k: torch.Tensor):
 
 
 def alloc_outputs(q: torch.Tensor, k: torch.Tensor, block: int, rho_min: float, tau: float,
-                  k_min: int):
+                  k_min: int, method=None):
     """(out, sel_idx, sel_cnt) allocated on q's device."""
     B, Hq, Hkv, S, D = _shape(q, k)
     nb = S // block
-    cap = stem_sel_capacity(nb, rho_min, tau, k_min)
+    cap = stem_sel_capacity(nb, rho_min, tau, k_min, method)
     out = torch.empty_like(q)
     sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=q.device)
     sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=q.device)
@@ -164,7 +212,7 @@ def alloc_workspace(q: torch.Tensor, k: torch.Tensor, block: int) -> torch.Tenso
 
 
 def make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, workspace=None,
-              status=None, events=None) -> stem_args_t:
+              status=None, events=None, method=None) -> stem_args_t:
     B, Hq, Hkv, S, D = _shape(q, k)
     a = stem_args_t()
     a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
@@ -181,20 +229,24 @@ def make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, worksp
                                       for e in events])
         a._events_keepalive = arr
         a.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    if method is not None:
+        a._method_keepalive = method
+        a.method = ctypes.pointer(method)
     return a
 
 
 def stem_prefill_ex(q, k, v, block, rho_min, tau, k_min, out=None, sel_idx=None, sel_cnt=None,
-                    workspace=None, status=None, stream=None, events=None):
+                    workspace=None, status=None, stream=None, events=None, method=None):
     """Whole path on device tensors [B,H,S,D] (bf16 or f32). Returns (out, sel_idx, sel_cnt).
     Asynchronous on `stream` (default: torch's current stream). `events`: optional four
-    torch.cuda.Event recorded before pooling, selection, attention and after attention."""
+    torch.cuda.Event recorded before pooling, selection, attention and after attention.
+    `method`: optional stem_method_t (make_method); it replaces rho_min, tau and k_min."""
     if out is None or sel_idx is None or sel_cnt is None:
-        out, sel_idx, sel_cnt = alloc_outputs(q, k, block, rho_min, tau, k_min)
+        out, sel_idx, sel_cnt = alloc_outputs(q, k, block, rho_min, tau, k_min, method)
     if workspace is None:
         workspace = alloc_workspace(q, k, block)
     a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, workspace, status,
-                  events)
+                  events, method)
     _check(_lib.stem_prefill_ex(ctypes.byref(a), _stream(stream)), "stem_prefill_ex")
     return out, sel_idx, sel_cnt
 
@@ -210,13 +262,14 @@ def stem_prefill(q, k, v, block, rho_min, tau, k_min, out=None, sel_idx=None, se
     return out, sel_idx, sel_cnt
 
 
-def stem_prefill_host(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt) -> None:
+def stem_prefill_host(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt,
+                      method=None) -> None:
     """Whole path on HOST tensors (pinned for speed); synchronous."""
-    a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt)
+    a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, method=method)
     _check(_lib.stem_prefill_host(ctypes.byref(a)), "stem_prefill_host")
 
 
-def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None):
+def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None, method=None):
     B, Hq, Hkv, S, D = _shape(q, k)
     nb = S // block
     dev = q.device
@@ -224,6 +277,11 @@ def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None):
         qbar = torch.empty((B, Hq, nb, D), dtype=torch.float32, device=dev)
         kbar = torch.empty((B, Hkv, nb, D), dtype=torch.float32, device=dev)
         vnorm = torch.empty((B, Hkv, nb), dtype=torch.float32, device=dev)
+    if method is not None:
+        _check(_lib.stem_pool_m(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq,
+                                Hkv, S, D, block, ctypes.byref(method), qbar.data_ptr(),
+                                kbar.data_ptr(), vnorm.data_ptr(), _stream(stream)), "stem_pool_m")
+        return qbar, kbar, vnorm
     _check(_lib.stem_pool(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq, Hkv,
                           S, D, block, qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(),
                           _stream(stream)), "stem_pool")
@@ -231,13 +289,13 @@ def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None):
 
 
 def stem_select(qbar, kbar, vnorm, rho_min, tau, k_min, with_metric=False, workspace=None,
-                sel_idx=None, sel_cnt=None, stream=None):
+                sel_idx=None, sel_cnt=None, stream=None, method=None):
     """CSR selection from pooled summaries (float32 device tensors). Returns (sel_idx, sel_cnt,
     m or None)."""
     B, Hq, nb, D = qbar.shape
     Hkv = kbar.shape[1]
     dev = qbar.device
-    cap = stem_sel_capacity(nb, rho_min, tau, k_min)
+    cap = stem_sel_capacity(nb, rho_min, tau, k_min, method)
     if sel_idx is None:
         sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=dev)
         sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=dev)
@@ -246,6 +304,12 @@ def stem_select(qbar, kbar, vnorm, rho_min, tau, k_min, with_metric=False, works
     if workspace is None:
         workspace = torch.empty(max(stem_workspace_size(B, Hq, Hkv, nb * 64, D, 64), 256),
                                 dtype=torch.uint8, device=dev)
+    if method is not None:
+        _check(_lib.stem_select_m(qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(), B, Hq, Hkv,
+                                  nb, D, ctypes.byref(method), sel_idx.data_ptr(),
+                                  sel_cnt.data_ptr(), _ptr(m), workspace.data_ptr(),
+                                  workspace.numel(), _stream(stream)), "stem_select_m")
+        return sel_idx, sel_cnt, m
     _check(_lib.stem_select(qbar.data_ptr(), kbar.data_ptr(), vnorm.data_ptr(), B, Hq, Hkv, nb,
                             D, rho_min, tau, k_min, sel_idx.data_ptr(), sel_cnt.data_ptr(),
                             _ptr(m), workspace.data_ptr(), workspace.numel(), _stream(stream)),
@@ -254,12 +318,19 @@ def stem_select(qbar, kbar, vnorm, rho_min, tau, k_min, with_metric=False, works
 
 
 def stem_sparse_attn(q, k, v, block, rho_min, tau, k_min, sel_idx, sel_cnt, out=None,
-                     workspace=None, status=None, stream=None):
+                     workspace=None, status=None, stream=None, method=None):
     B, Hq, Hkv, S, D = _shape(q, k)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(q, k, block)
+    if method is not None:
+        _check(_lib.stem_sparse_attn_m(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q),
+                                       B, Hq, Hkv, S, D, block, ctypes.byref(method),
+                                       sel_idx.data_ptr(), sel_cnt.data_ptr(), out.data_ptr(),
+                                       workspace.data_ptr(), workspace.numel(), _ptr(status),
+                                       _stream(stream)), "stem_sparse_attn_m")
+        return out
     _check(_lib.stem_sparse_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, Hq,
                                  Hkv, S, D, block, rho_min, tau, k_min, sel_idx.data_ptr(),
                                  sel_cnt.data_ptr(), out.data_ptr(), workspace.data_ptr(),

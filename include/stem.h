@@ -19,6 +19,10 @@
  *   kept(i) = {0, i} plus the k(i)-2 best j in [1, i-1] by (m_ij descending, j ascending);
  *   out[r] = softmax attention of query token r over every token of kept(i), token-causal
  *            inside block i, logits scaled by 1/sqrt(D).
+ * The pages' own parameterisations are selectable per call (stem_method_t below): the linear
+ * budget k(i) = ceil(k_start * (1 - (1 - mu) * i/(nb-1))) ([es] 2.A, [it] 2.A, [nl] TPD,
+ * [fr] 2.A), the additive metric s_ij + beta * max(0, log n_j^2) ([es] 2.B, [it] 2.B, [nl] OAM,
+ * [fr] 2.B) and the largest V-row norm as n_j ([nl] Implementatie step 1).
  *
  * Conventions shared by every call:
  *   - Tensors are contiguous [B, H, S, D] (row-major, D fastest). Q and out have Hq heads, K and
@@ -58,6 +62,42 @@ extern "C" {
 #define STEM_BF16 0
 #define STEM_F32 1
 
+/* Budget schedules, metrics and V summaries of stem_method_t. */
+#define STEM_SCHED_EXP 0       /* rho(i) = rho_min + (1 - rho_min) exp(-i / tau) (the default) */
+#define STEM_SCHED_LINEAR 1    /* k_start at block 0 down to mu * k_start at block nb-1 */
+#define STEM_METRIC_PRODUCT 0  /* m_ij = softmax_j(s_ij) * n_j (the default) */
+#define STEM_METRIC_ADDITIVE 1 /* M_ij = s_ij + beta * max(0, log n_j^2) */
+#define STEM_VSUM_MEAN 0       /* n_j = mean of the block's V-row L2 norms (the default) */
+#define STEM_VSUM_MAX 1        /* n_j = largest V-row L2 norm of the block */
+
+/*
+ * Method parameters: budget schedule, block metric and V summary.
+ *   STEM_SCHED_EXP:     k(i) = min(i+1, max(k_min, ceil(rho(i) * (i+1)))), rho as above;
+ *                       rho_min in (0, 1], tau > 0 and finite.
+ *   STEM_SCHED_LINEAR:  k(i) = min(i+1, max(k_min, ceil(k_start * (1 - (1 - mu) * t)))),
+ *                       t = i / (nb - 1) (0 when nb == 1), in double precision from the float
+ *                       parameters; k_start > 0 and finite (blocks), mu in (0, 1].
+ *   Both: k(0) = 1 and k(i) >= 2 for i >= 1 (sink and diagonal); k_min >= 1.
+ *   STEM_METRIC_PRODUCT:  rank by s_ij + ln n_j (= log m_ij + const).
+ *   STEM_METRIC_ADDITIVE: rank by s_ij + beta * e_j, e_j = 2 ln n_j, clamped at 0 when clamp is
+ *                         1; beta >= 0 and finite (beta == 0: e_j is not evaluated, so
+ *                         n_j = 0 is allowed); clamp in {0, 1}.
+ *   vsum: STEM_VSUM_MEAN or STEM_VSUM_MAX (pooling of ||V row|| into n_j).
+ * Fields the chosen schedule and metric do not use are ignored.
+ */
+typedef struct stem_method {
+  int32_t schedule;
+  float rho_min;
+  float tau;
+  float k_start;
+  float mu;
+  int32_t k_min;
+  int32_t metric;
+  float beta;
+  int32_t clamp;
+  int32_t vsum;
+} stem_method_t;
+
 /* Largest number of blocks per sequence (the selection kernel keeps one score row per
  * query block in shared memory). */
 #define STEM_MAX_NB 4096
@@ -76,6 +116,7 @@ extern "C" {
  *                                          stream before pooling, before selection, before
  *                                          attention and after attention (per-stage timing);
  *                                          NULL to skip
+ *   method                                 optional method parameters (stem_method_t)
  */
 typedef struct stem_args {
   const void* q;
@@ -93,6 +134,10 @@ typedef struct stem_args {
   size_t workspace_bytes;
   int32_t* status;
   void* const* events;
+  /* optional: NULL keeps the exponential schedule of rho_min, tau and k_min above, the product
+   * metric and mean-pooled V norms; otherwise it sets every method parameter and rho_min, tau
+   * and k_min above are ignored */
+  const stem_method_t* method;
 } stem_args_t;
 
 /*
@@ -176,6 +221,26 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
                      int Hkv, int S, int D, int block, float rho_min, float tau, int k_min,
                      const int32_t* sel_idx, const int32_t* sel_cnt, void* out, void* workspace,
                      size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * Method-parameterised forms of the calls above: the same behaviour, with the schedule, metric
+ * and V summary taken from m (see stem_method_t) instead of (rho_min, tau, k_min). m must not
+ * be NULL; an invalid field returns STEM_ERR_ARG. stem_pool_m reads only m->vsum.
+ */
+int stem_budget_m(int nb, const stem_method_t* m, int32_t* k_out, int32_t* off_out);
+int64_t stem_sel_capacity_m(int nb, const stem_method_t* m);
+int stem_pool_m(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
+                int S, int D, int block, const stem_method_t* m, float* qbar, float* kbar,
+                float* vnorm, void* stream);
+/* m_out holds the metric of the chosen form: m_ij (product) or M_ij (additive), float32. */
+int stem_select_m(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                  int Hkv, int nb, int D, const stem_method_t* m, int32_t* sel_idx,
+                  int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
+                  void* stream);
+int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, int B, int Hq,
+                       int Hkv, int S, int D, int block, const stem_method_t* m,
+                       const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
+                       void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
 /*
  * stem_select_static: stem_select for callers that cannot allocate device memory. The paper

@@ -96,4 +96,34 @@ res = {
                                             None, FAKE, None),
     "capacity_bad_rho": L.stem_sel_capacity(8, 0.0, 4.0, 2),
 }
+
+# method-parameterised calls: an invalid stem_method_t field is rejected the same way
+BAD_MU = S.make_method("linear", k_start=8.0, mu=0.0, k_min=2)
+BAD_BETA = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2, metric="additive", beta=-1.0)
+BAD_VSUM = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2)
+BAD_VSUM.vsum = 7
+GOOD = S.make_method("linear", k_start=8.0, mu=0.7, k_min=2, metric="additive", beta=0.2)
+M = lambda m: ctypes.byref(m)  # noqa: E731
+res.update({
+    "method_bad_mu": ex(method=ctypes.pointer(BAD_MU)),
+    "method_bad_beta": ex(method=ctypes.pointer(BAD_BETA)),
+    "method_bad_vsum": ex(method=ctypes.pointer(BAD_VSUM)),
+    "method_overrides_bad_rho": ex(rho_min=-1.0, method=ctypes.pointer(BAD_MU)),
+    "host_method_bad": L.stem_prefill_host(ctypes.byref(base(method=ctypes.pointer(BAD_BETA)))),
+    "pool_m_bad_vsum": L.stem_pool_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, M(BAD_VSUM),
+                                     FAKE, FAKE, FAKE, None),
+    "pool_m_null_method": L.stem_pool_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, None,
+                                        FAKE, FAKE, FAKE, None),
+    "select_m_bad_mu": L.stem_select_m(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, M(BAD_MU), FAKE, FAKE,
+                                       None, FAKE, 1 << 20, None),
+    "select_m_null_method": L.stem_select_m(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, None, FAKE, FAKE,
+                                            None, FAKE, 1 << 20, None),
+    "select_m_no_workspace": L.stem_select_m(FAKE, FAKE, FAKE, 1, 4, 2, 8, 128, M(GOOD), FAKE,
+                                             FAKE, None, None, 0, None),
+    "attn_m_bad_beta": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128,
+                                            M(BAD_BETA), FAKE, FAKE, FAKE, FAKE, 1 << 20, None,
+                                            None),
+    "attn_m_ragged": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1000, 128, 128, M(GOOD),
+                                          FAKE, FAKE, FAKE, FAKE, 1 << 20, None, None),
+})
 print(json.dumps(res))

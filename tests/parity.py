@@ -3,7 +3,9 @@
 Selection: counts must equal k(i) exactly and every row must be ascending, distinct, inside
 [0, i] and contain 0 and i. Kept sets must equal the oracle's, except where the two differ only
 by swapping blocks whose oracle metrics are within REL_TIE of each other (several selections
-are then equally correct).
+are then equally correct). For the product metric m = exp(key - logsumexp) that is a relative
+gap; the additive metric M is itself a key, so the same gap is taken absolutely, scaled by
+max(1, |M|): |M_a - M_b| <= REL_TIE * max(1, |M_a|, |M_b|).
 
 Attention output: max-abs error <= 2e-2 and mean-abs error <= 1e-3 against the oracle's
 double-precision result for bfloat16 inputs (float32 accumulation); tighter for float32 inputs.
@@ -25,7 +27,8 @@ def tol_for(dtype: torch.dtype):
     return TOL_BF16 if dtype == torch.bfloat16 else TOL_F32
 
 
-def compare_selection(gpu_idx, gpu_cnt, ref_idx, ref_cnt, m_ref, k, off, rel=REL_TIE):
+def compare_selection(gpu_idx, gpu_cnt, ref_idx, ref_cnt, m_ref, k, off, rel=REL_TIE,
+                      additive=False):
     """Returns dict(rows, identical, tie_swaps, violations=[...])."""
     gi = np.asarray(gpu_idx.cpu() if torch.is_tensor(gpu_idx) else gpu_idx)
     gc = np.asarray(gpu_cnt.cpu() if torch.is_tensor(gpu_cnt) else gpu_cnt)
@@ -64,11 +67,12 @@ def compare_selection(gpu_idx, gpu_cnt, ref_idx, ref_cnt, m_ref, k, off, rel=REL
         mrow = oracle.metric_row(m_ref, b, h, i)
         hi = mrow[missing].max()
         lo = mrow[extra].min()
-        if hi - lo <= rel * hi:
+        scale = max(1.0, abs(hi), abs(lo)) if additive else hi
+        if hi - lo <= rel * scale:
             tie_swaps += 1
         else:
             violations.append(f"row {(b, h, i)}: kept {extra.tolist()} over {missing.tolist()} "
-                              f"(rel gap {(hi - lo) / hi:.3e})")
+                              f"(rel gap {(hi - lo) / scale:.3e})")
     return dict(rows=B * Hq * nb, identical=B * Hq * nb - len(rows_bad), tie_swaps=tie_swaps,
                 violations=violations, rows_bad=sorted(rows_bad))
 

@@ -1,5 +1,6 @@
 """The C ABI on the CPU: exports, host-only functions, argument validation (no GPU needed)."""
 
+import ctypes
 import json
 import os
 import re
@@ -49,6 +50,56 @@ def test_budget_matches_oracle(case):
     assert S.stem_sel_capacity(nb, r, t, km) == int(offo[-1])
 
 
+LINEAR_CASES = [(8, 8.0, 0.5, 1), (6, 10.0, 0.35, 3), (1024, 36.0, 0.7, 8), (512, 40.0, 0.7, 4),
+                (128, 12.0, 0.7, 8), (1000, 700.0, 0.05, 1), (1, 4.0, 0.7, 1), (0, 4.0, 0.7, 1),
+                (4096, 64.0, 0.3, 2)]
+
+
+@pytest.mark.parametrize("case", LINEAR_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_linear_budget_matches_oracle(case):
+    nb, ks, mu, km = case
+    m = S.make_method("linear", k_start=ks, mu=mu, k_min=km)
+    k, off = S.stem_budget_m(nb, m)
+    ko, offo = oracle.budget_linear(nb, ks, mu, km)
+    assert np.array_equal(k.numpy(), ko)
+    assert np.array_equal(off.numpy().astype(np.int64), offo)
+    assert S.stem_sel_capacity(nb, 0.0, 0.0, 0, method=m) == int(offo[-1])
+
+
+def test_method_budget_defaults_equal_plain_calls():
+    for nb, r, t, km in [(1024, 0.05, 64.0, 8), (256, 0.1, 32.0, 4), (16, 0.25, 4.0, 2)]:
+        m = S.make_method("exp", rho_min=r, tau=t, k_min=km, metric="additive", beta=0.2,
+                          vsum="max")
+        k1, off1 = S.stem_budget_m(nb, m)
+        k2, off2 = S.stem_budget(nb, r, t, km)
+        assert np.array_equal(k1.numpy(), k2.numpy()) and np.array_equal(off1.numpy(), off2.numpy())
+
+
+@pytest.mark.parametrize("bad", [
+    dict(schedule="linear", k_start=0.0, mu=0.7), dict(schedule="linear", k_start=-3.0, mu=0.7),
+    dict(schedule="linear", k_start=float("inf"), mu=0.7),
+    dict(schedule="linear", k_start=8.0, mu=0.0), dict(schedule="linear", k_start=8.0, mu=1.5),
+    dict(schedule="linear", k_start=8.0, mu=float("nan")),
+    dict(schedule="exp", rho_min=0.0, tau=4.0), dict(schedule="exp", rho_min=0.5, tau=0.0),
+    dict(schedule="exp", rho_min=0.5, tau=4.0, k_min=0),
+    dict(schedule="exp", rho_min=0.5, tau=4.0, metric="additive", beta=-0.1),
+    dict(schedule="exp", rho_min=0.5, tau=4.0, metric="additive", beta=float("nan")),
+], ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
+def test_method_validation(bad):
+    m = S.make_method(**{"k_min": 1, **bad})
+    assert S.lib().stem_budget_m(64, ctypes.byref(m), None, None) == S.STEM_ERR_ARG
+    assert S.lib().stem_sel_capacity_m(64, ctypes.byref(m)) == S.STEM_ERR_ARG
+    # enum fields outside their sets
+    for field, val in (("schedule", 2), ("metric", 5), ("vsum", -1)):
+        m2 = S.make_method("exp", rho_min=0.5, tau=4.0, k_min=1)
+        setattr(m2, field, val)
+        assert S.lib().stem_budget_m(64, ctypes.byref(m2), None, None) == S.STEM_ERR_ARG
+    m3 = S.make_method("exp", rho_min=0.5, tau=4.0, k_min=1, metric="additive", beta=0.2)
+    m3.clamp = 2
+    assert S.lib().stem_budget_m(64, ctypes.byref(m3), None, None) == S.STEM_ERR_ARG
+    assert S.lib().stem_budget_m(64, None, None, None) == S.STEM_ERR_ARG
+
+
 def test_workspace_size_layout():
     B, Hq, Hkv, Sq, D, block = 1, 32, 8, 131072, 128, 128
     nb = Sq // block
@@ -80,6 +131,7 @@ def test_argument_validation_rejects_before_any_device_work():
         "workspace_small": S.STEM_ERR_WORKSPACE,
         "workspace_misaligned": S.STEM_ERR_WORKSPACE,
         "select_no_workspace": S.STEM_ERR_WORKSPACE,
+        "select_m_no_workspace": S.STEM_ERR_WORKSPACE,
         "attn_small_workspace": S.STEM_ERR_WORKSPACE,
         "nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "select_nb_too_large": S.STEM_ERR_UNSUPPORTED,
