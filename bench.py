@@ -58,6 +58,11 @@ def parse():
     p.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--method", choices=["default", "pages"], default="default",
+                   help="default: exponential budget, product metric, mean V norms; pages: the "
+                        "pages' linear budget (mu 0.7) with the additive metric (beta 0.2, "
+                        "clamped) and max-pooled V norms, k_start set for the default's mean "
+                        "budget")
     return p.parse_args()
 
 
@@ -158,18 +163,39 @@ class ClockSampler:
 # ------------------------------------------------------------------ CPU oracle (reference arm)
 
 
-def oracle_sample_step(w, q, k, v, rows):
+def method_params(w, name):
+    """Method parameters of a bench run (None: the library's default). "pages": the pages' own
+    forms with their ablation optimum (mu 0.7, beta 0.2); k_start gives the linear budget the
+    same mean as the workload's default budget, 2 * mean / (1 + mu), to one decimal."""
+    if name == "default":
+        return None
+    from block_sparse_causal_pooling_b200 import stem as S
+
+    kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
+    mu = 0.7
+    k_start = round(2.0 * float(kk.double().mean()) / (1.0 + mu), 1)
+    return dict(schedule="linear", k_start=k_start, mu=mu, k_min=w.k_min, metric="additive",
+                beta=0.2, clamp=True, vsum="max")
+
+
+def oracle_sample_step(w, q, k, v, rows, mp=None):
     """The oracle as it stands on one kv-head group: pooling, metric, selection for every query
     block of the group's heads, then exact attention for the listed rows. Returns (effective
-    FLOP of the listed rows, seconds for attention + selection prorated to those rows)."""
+    FLOP of the listed rows, seconds for attention + selection prorated to those rows).
+    mp: method parameters (method_params) or None for the default."""
     import oracle
 
     G = w.Hq // w.Hkv
     qs, ks, vs = q[:, :G].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous()
     t0 = time.perf_counter()
-    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
-    qb, kb, vn = oracle.pool(qs, ks, vs, w.block)
-    m = oracle.metric(qb, kb, vn)
+    if mp is None:
+        kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+        qb, kb, vn = oracle.pool(qs, ks, vs, w.block)
+        m = oracle.metric(qb, kb, vn)
+    else:
+        kk, off = oracle.budget_linear(w.nb, mp["k_start"], mp["mu"], mp["k_min"])
+        qb, kb, vn = oracle.pool(qs, ks, vs, w.block, mp["vsum"])
+        m = oracle.metric_additive(qb, kb, vn, mp["beta"], mp["clamp"])
     si, sc = oracle.select(m, kk, off)
     t1 = time.perf_counter()
     oracle.attention(qs, ks, vs, w.block, si, sc, off, rows)
@@ -190,6 +216,7 @@ def run_reference(args, world, rank):
     import oracle
 
     w = wl.WORKLOADS[args.workload]
+    mp = method_params(w, args.method)
     q, k, v = cpu_inputs(w)
     G = w.Hq // w.Hkv
     import random
@@ -199,7 +226,7 @@ def run_reference(args, world, rank):
     samples = []
     for step in range(args.warmup + args.steps):
         rows = [(0, rng.randrange(G), rng.randrange(w.nb)) for _ in range(n_rows)]
-        flop, sec, _ = oracle_sample_step(w, q, k, v, rows)
+        flop, sec, _ = oracle_sample_step(w, q, k, v, rows, mp)
         if step >= args.warmup:
             samples.append((flop, sec))
     flop = sum(f for f, _ in samples)
@@ -213,7 +240,7 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sec / len(samples), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w),
+        "config": config_of(w, mp),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -280,10 +307,15 @@ class RawEvents:
         self.made = []
 
 
-def config_of(w):
-    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
-            "block": w.block, "rho_min": w.rho_min, "tau": w.tau, "k_min": w.k_min,
-            "input_dtype": w.dtype, "l2": "inputs (Q+K+V) larger than L2; no flush"}
+def config_of(w, mp=None):
+    c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
+         "block": w.block, "rho_min": w.rho_min, "tau": w.tau, "k_min": w.k_min,
+         "input_dtype": w.dtype, "l2": "inputs (Q+K+V) larger than L2; no flush"}
+    if mp is not None:
+        c.pop("rho_min")
+        c.pop("tau")
+        c["method"] = dict(mp)
+    return c
 
 
 def run_ours(args, world, rank, local):
@@ -292,10 +324,15 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = wl.WORKLOADS[args.workload]
+    mp = method_params(w, args.method)
+    meth = None if mp is None else S.make_method(**mp)
     q, k, v = wl.make_inputs(rank_workload(w, rank), dev)
-    out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min)
+    out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min, meth)
     ws = S.alloc_workspace(q, k, w.block)
-    kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
+    if meth is None:
+        kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
+    else:
+        kk, _ = S.stem_budget_m(w.nb, meth)
     pairs = w.B * w.Hq * int(kk.sum())
     flop = wl.effective_flops(pairs, w.block, w.D)
     stream = torch.cuda.current_stream(dev)
@@ -304,9 +341,9 @@ def run_ours(args, world, rank, local):
     raw = RawEvents()
     ev = [[raw.create() for _ in range(4)] for _ in range(K)]
     args_warm = S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
-                            ws)
+                            ws, method=meth)
     call_args = [S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
-                             ws, events=ev[s]) for s in range(K)]
+                             ws, events=ev[s], method=meth) for s in range(K)]
     lib = S.lib()
     hstream = S.ctypes.c_void_p(stream.cuda_stream)
 
@@ -349,12 +386,14 @@ def run_ours(args, world, rank, local):
         hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
         hsi = torch.empty(sel_idx.shape, dtype=torch.int32).pin_memory()
         hsc = torch.empty(sel_cnt.shape, dtype=torch.int32).pin_memory()
-        S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc)
+        S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc,
+                            method=meth)
         if world > 1:
             torch.distributed.barrier()
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
-            S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc)
+            S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc,
+                                method=meth)
         e2e_s = max_over_ranks((time.perf_counter() - t0) / args.e2e_steps, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
         d2h = sum(t.numel() * t.element_size() for t in (hout, hsi, hsc))
@@ -381,11 +420,11 @@ def run_ours(args, world, rank, local):
         "data": f"synthetic, seeded ({w.name}: N(0,1) Q/K/V, RoPE theta {w.rope_theta}, K row 0 "
                 f"x{w.sink_scale}, {w.n_v_outliers()} V rows per kv-head x{w.v_outlier_scale}, "
                 f"heavy-tail fraction {w.heavy_tail_frac})",
-        "config": dict(config_of(w), kept_pairs=pairs, effective_tflop=flop / 1e12,
+        "config": dict(config_of(w, mp), kept_pairs=pairs, effective_tflop=flop / 1e12,
                        causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                     "traffic": attn_traffic(w.name),
+                     "traffic": attn_traffic(w.name) if mp is None else None,
                      "peak_source": f"{pk_kind} {'sustained' if long_region else 'burst'} "
                                     "bf16 dense"},
         "kernels": {
@@ -401,11 +440,11 @@ def run_ours(args, world, rank, local):
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, mp)
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w):
+def cpu_baseline(w, mp=None):
     """The oracle, as it stands, on a bounded sample: one kv-head group's selection plus exact
     attention of 64 query blocks per q-head (blocks 0, 1, nb-1 and 61 random, seed 7)."""
     import oracle
@@ -414,7 +453,7 @@ def cpu_baseline(w):
     G = w.Hq // w.Hkv
     wg = w.replace(Hq=G, Hkv=1)
     rows = wl.sample_rows(wg, n_random=61, seed=7)
-    flop, sec, parts = oracle_sample_step(w, q, k, v, rows)
+    flop, sec, parts = oracle_sample_step(w, q, k, v, rows, mp)
     return {"value": flop / sec / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
             "kind": "oracle",
             "sample": (f"one kv-head group ({G} q-heads): pooling, metric and selection of all "
