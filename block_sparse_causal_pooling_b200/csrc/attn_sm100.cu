@@ -26,9 +26,11 @@
 //               both warps agree on going on, so an abort cannot strand one), exp2 with the
 //               1/sqrt(D) scale folded in, per-thread partial row sums in fp32 (f32x2
 //               arithmetic); P packed to bf16 and stored over the first half of S_T
-//               (tcgen05.st); O rescaled in TMEM only when the running max grows by more than
-//               2^8 (exact: the final 1/l uses the same reference max). At an item's end:
-//               O * (1/l) -> bf16 -> global (streaming stores).
+//               (tcgen05.st). Only an item's first step takes the exact row max; later steps
+//               use it as the reference and fall back to the exact max, an O rescale in TMEM
+//               and a recompute only when a partial row sum reaches 2^16 (exact: the final
+//               1/l uses the same reference as P). At an item's end: O * (1/l) -> bf16 ->
+//               global (streaming stores).
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).
 //
 // Synchronisation is by mbarriers, plus the warp-pair barrier above. Every mbarrier wait is
@@ -633,12 +635,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tile >= 0) mbar_arrive(&bars->kv_empty[tile % kSlots]);
     };
     // one step of tile tl on key block blk; returns false on abort
+    // Row max of this thread's half of S (log2 units, scale folded in) agreed with the partner
+    // half through shared memory; both warps of the pair call it at the same point.
+    auto pair_max = [&](const uint32_t* sr, bool& ok) -> float {
+      float mx[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
+#pragma unroll
+      for (int c = 4; c < kH; c += 2)
+        mx[(c >> 1) & 3] =
+            max3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      bars->xch[xp][half][row] = mt;
+      ok = pair_and(bar_id, true);
+      mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // both halves alike
+      xp ^= 1;
+      return mt;
+    };
+    // P = exp2(S * sl2 - m_run) packed to bf16; returns this thread's partial row sum.
+    auto exp_pack = [&](const uint32_t* sr, float m_run, uint32_t* p) -> float {
+      const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
+      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
+#pragma unroll
+      for (int c = 0; c < kH / 2; ++c) {
+        const f2 x = fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
+        const f2 e{ex2(x.x), ex2(x.y)};
+        sum[c & 1] = add2(sum[c & 1], e);
+        p[c] = pack_bf16(e.x, e.y);
+      }
+      return (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
+    };
+    // One step of tile tl on key block blk; returns false on abort.
+    //
+    // The exponentials use the row's running reference max m_run. The first step of an item
+    // sets it to the exact row max; later steps form P against it without looking for their
+    // own max, and only if some row's partial sum reaches 2^16 (a score that grew by ~10 in
+    // log2 units, or an overflow) does the pair take the exact max, rescale O and recompute.
+    // The result is exact either way: the final 1/l uses the same reference as P.
+    //
+    // Barriers of the warp pair per step, the same sequence on both warps: [first step: max
+    // exchange] check; if the check fails: agree on going on, then the max exchange. A warp
+    // that gives up joins every barrier its partner will meet with "stop".
     auto step = [&](int tl, int blk, int qi, bool first, int64_t& nsteps, float& m_run,
                     float& lsum, int64_t rel_k, int64_t rel_v, bool rel_q) -> bool {
       const int64_t r = nsteps++;
       bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(r & 1), bars, status);
       if (!__all_sync(0xffffffffu, w)) {
-        pair_and(bar_id, false);
+        pair_and(bar_id, false);  // [first: the max exchange | the check]
+        if (!first) pair_and(bar_id, false);  // the agreement after a failed check
         return false;
       }
       if (releaser) {
@@ -657,31 +701,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kH; ++c)
           if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
-#pragma unroll
-      for (int c = 4; c < kH; c += 2)
-        mx[(c >> 1) & 3] =
-            max3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-      float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      bars->xch[xp][half][row] = mt;
-      if (!pair_and(bar_id, true)) return false;
-      mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // row max, both halves alike
-      xp ^= 1;
+      bool ok = true;
       if (first) {
-        m_run = mt;
+        m_run = pair_max(sr, ok);
+        if (!ok) return false;
         lsum = 0.f;
-      } else if (__any_sync(0xffffffffu, mt > m_run + 8.0f)) {
-        // a row's max grew by more than 2^8: the warp rescales its part of O_T (each row by
-        // its own factor, 1 where the max did not grow). The previous P V of this tile is
+      }
+      uint32_t p[kH / 2];
+      float part = exp_pack(sr, m_run, p);
+      const bool small = part < 65536.0f;  // false for inf and NaN too
+      if (!pair_and(bar_id, __all_sync(0xffffffffu, small))) {
+        if (!pair_and(bar_id, true)) return false;
+        // a row's scores grew past the reference (never on a first step, whose reference is
+        // the exact max): the warp rescales its part of O_T (each row by its own factor, 1
+        // where the max did not grow) and recomputes P. The previous P V of this tile is
         // complete: this S was issued after it and s_full tracks every earlier product.
+        const float mt = pair_max(sr, ok);
+        if (!ok) return false;
         const float m_new = fmaxf(m_run, mt);
         const float alpha = ex2(m_run - m_new);
         m_run = m_new;
         lsum *= alpha;
         const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < kDH / 32; ++c) {
           uint32_t o[32];
           TC_LD32(o_addr + 32 * c, o);
@@ -691,20 +733,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           TC_ST32(o_addr + 32 * c, o);
         }
         tc_wait_st();
+        part = exp_pack(sr, m_run, p);
       }
-      const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
-      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
-      uint32_t p[kH / 2];
-#pragma unroll
-      for (int c = 0; c < kH / 2; ++c) {
-        const f2 x = fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
-        const f2 e{ex2(x.x), ex2(x.y)};
-        sum[c & 1] = add2(sum[c & 1], e);
-        p[c] = pack_bf16(e.x, e.y);
-      }
-      lsum += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
+      lsum += part;
       // P over S_T columns [0, 64): this half's keys go to columns half*32 .. +32 (both halves
-      // finished reading S before the pair barrier above)
+      // finished reading S before the pair's check barrier above)
       TC_ST32(s_addr + half * (kH / 2), p);
       tc_wait_st();
       tc_fence_before();
