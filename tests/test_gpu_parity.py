@@ -115,6 +115,37 @@ def test_end_to_end(name):
     parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, name)
 
 
+@pytest.mark.parametrize("rho_min", [0.2, 1.0])
+def test_scores_growing_after_the_first_block(rho_min):
+    """Two key blocks halfway through the sequence are scaled x6 and there is no sink, so the
+    rows that keep them see scores far above those of their first block: the attention kernel's
+    reference max must be raised (O rescaled, P recomputed) for those rows."""
+    w = wl.LLAMA_32K.replace(name="growth", Hq=4, Hkv=2, S=4096, sink_scale=1.0,
+                             rho_min=rho_min, tau=8.0)
+    q, k, v = wl.make_inputs(w, "cpu")
+    k = k.clone()
+    k[:, :, 16 * w.block:18 * w.block] *= 6
+    ref = oracle.prefill(q, k, v, w.block, w.rho_min, w.tau, w.k_min)
+    dev = [t.to(DEV) for t in (q, k, v)]
+    status = torch.full((1,), 7, dtype=torch.int32, device=DEV)
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(*dev, w.block, w.rho_min, w.tau, w.k_min,
+                                              status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    res = parity.compare_selection(sel_idx, sel_cnt, ref["sel_idx"], ref["sel_cnt"], ref["m"],
+                                   ref["k"], ref["off"])
+    assert not res["violations"], res["violations"][:5]
+    # many rows after the boosted blocks keep one of them (all of them at rho_min = 1)
+    kept = [bool({16, 17} & set(oracle.row_list(ref["sel_idx"], ref["off"], ref["k"], 0, h, i)))
+            for h in range(w.Hq) for i in range(18, w.nb)]
+    assert sum(kept) >= (len(kept) if rho_min == 1.0 else len(kept) // 4), sum(kept)
+    swapped = set(res["rows_bad"])
+    rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
+    keep = [t for t, r in enumerate(rows) if r not in swapped]
+    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
+    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, "growth")
+
+
 def test_dense_budget_matches_torch_sdpa():
     """rho_min = 1 keeps every causal block: the path is dense causal attention."""
     w = wl.LLAMA_32K.replace(Hq=8, Hkv=2, S=8192, rho_min=1.0)
