@@ -44,8 +44,8 @@ KERNELS_PER_STEP = 4
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615452416 + 1024177152,
-                "sources_sha256": "8b64f3bfc09f62dbd21002d43b4b93df56a7d96321dc81f295c6dea79c82389c"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616169984 + 1023248128,
+                "sources_sha256": "05a6eb1561fc96d5f58ba074ec482a103d023cde7749c8e2cce19ccf6986db5b"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -9,8 +9,8 @@ max(1, |M|): |M_a - M_b| <= REL_TIE * max(1, |M_a|, |M_b|).
 
 Attention output: max-abs error <= 2e-2 and mean-abs error <= 1e-3 against the oracle's
 double-precision result for bfloat16 inputs (float32 accumulation); tighter for float32 inputs.
-Where |reference| >= 8 the bfloat16 bound is one bfloat16 ulp of the reference instead (the
-output format cannot resolve 2e-2 there).
+For bfloat16 the per-element max-abs bound grows as 2^-7 |reference| above |reference| = 2.56
+(the bfloat16 rounding of P and of the output; see assert_out_close).
 """
 
 from __future__ import annotations
@@ -95,22 +95,18 @@ def out_error(gpu: np.ndarray, ref: np.ndarray):
                 max_ref=float(np.abs(ref).max()) if ref.size else 0.0)
 
 
-def bf16_ulp(x: np.ndarray) -> np.ndarray:
-    """Spacing of bfloat16 numbers at |x| (8 significant bits)."""
-    ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
-    return np.exp2(np.floor(np.log2(ax)) - 7)
-
-
 def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
-    """Max-abs and mean-abs error against the oracle. For bfloat16 outputs the per-element
-    bound is max(max_abs, one bfloat16 ulp of the reference): at |out| >= 8 a correctly rounded
-    bfloat16 output is already up to half an ulp (>= 0.031) away, more than the 2e-2 bound."""
+    """Max-abs and mean-abs error against the oracle. For bfloat16 the per-element bound is
+    max(max_abs, 2^-7 |reference|): P enters P V rounded to bfloat16 (relative error <= 2^-9)
+    and the output is rounded to bfloat16 (<= 2^-8 relative), so where one key dominates a
+    large output the error of any such kernel approaches 2^-7 |out|. Up to |out| = 2.56 the
+    bound is max_abs itself."""
     e = out_error(gpu, ref)
     t = tol_for(dtype)
     bound = t["max_abs"]
     if dtype == torch.bfloat16 and ref.size:
-        bound = np.maximum(t["max_abs"], bf16_ulp(ref))
-        e["n_ref_above_8"] = int((np.abs(ref) >= 8).sum())
+        bound = np.maximum(t["max_abs"], np.abs(ref) * 2.0 ** -7)
+        e["n_bound_above_max_abs"] = int((np.abs(ref) * 2.0 ** -7 > t["max_abs"]).sum())
     worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
     assert worst <= 0 and e["mean_abs"] <= t["mean_abs"], (what, e, t)
     return e
