@@ -12,7 +12,8 @@ Parity status: every function here is pinned by the CPU test suite (budget:
 arbitrary-precision recomputation, closed forms; linear budget: cases worked by
 hand, closed forms, exact rational recomputation; pooling, metric, selection,
 attention: brute force from token-level definitions, the additive-metric
-equivalence and closed forms, dense attention via a library routine). See the
+equivalence and closed forms, dense attention via a library routine; a partial
+last block: slicing and token-mask brute force, prefix invariance). See the
 tests for the pins.
 """
 
@@ -122,7 +123,7 @@ def pool(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, vsum: st
     q, k, v = _host(q), _host(k), _host(v)
     B, Hq, S, D = q.shape
     Hkv = k.shape[1]
-    nb = S // block
+    nb = -(-S // block)  # a partial last block counts
     qbar = np.zeros((B, Hq, nb, D))
     kbar = np.zeros((B, Hkv, nb, D))
     vnorm = np.zeros((B, Hkv, nb))
@@ -193,7 +194,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
     q, k, v = _host(q), _host(k), _host(v)
     B, Hq, S, D = q.shape
     Hkv = k.shape[1]
-    nb = S // block
+    nb = -(-S // block)
     if rows is None:
         ids = np.arange(B * Hq * nb, dtype=np.int64)
     else:
@@ -221,7 +222,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
     schedule "exp" uses rho_min, tau; "linear" uses k_start, mu. metric_form "product" is
     softmax(s) * n, "additive" is s + beta * max(0, log n^2) (clamp=False drops the max)."""
     B, Hq, S, D = q.shape
-    nb = S // block
+    nb = -(-S // block)
     if schedule == "exp":
         kk, off = budget(nb, rho_min, tau, k_min)
     elif schedule == "linear":

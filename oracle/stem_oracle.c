@@ -36,7 +36,9 @@
  *            the kept blocks, token-causal inside the diagonal block.
  *
  * Layouts: Q [B,Hq,S,D], K and V [B,Hkv,S,D], contiguous. Query head h reads
- * key/value head h / (Hq/Hkv). dtype 0 = bfloat16 (raw 16-bit patterns),
+ * key/value head h / (Hq/Hkv). S need not be a multiple of block: there are
+ * nb = ceil(S/block) blocks and the last one holds the S - (nb-1)*block
+ * remaining tokens (pooled over those rows only). dtype 0 = bfloat16 (raw 16-bit patterns),
  * dtype 1 = float32. Every value is widened to double before any arithmetic.
  */
 #include <math.h>
@@ -137,30 +139,32 @@ int64_t stem_oracle_budget_linear(int nb, double k_start, double mu, int k_min,
 void stem_oracle_pool(const void* q, const void* k, const void* v, int dtype, int B,
                       int Hq, int Hkv, int S, int D, int block, int vmax, double* qbar,
                       double* kbar, double* vnorm) {
-  const int nb = S / block;
+  const int nb = (S + block - 1) / block;
   const int64_t nq = (int64_t)B * Hq * nb;
   const int64_t nk = (int64_t)B * Hkv * nb;
 #pragma omp parallel for schedule(static)
   for (int64_t u = 0; u < nq; ++u) {
     const int64_t bh = u / nb, i = u % nb;
     const int64_t row0 = bh * S + i * block;
+    const int n = S - i * block < block ? (int)(S - i * block) : block; /* rows of block i */
     for (int d = 0; d < D; ++d) {
       double acc = 0.0;
-      for (int r = 0; r < block; ++r) acc += elem(q, dtype, (row0 + r) * D + d);
-      qbar[u * D + d] = acc / block;
+      for (int r = 0; r < n; ++r) acc += elem(q, dtype, (row0 + r) * D + d);
+      qbar[u * D + d] = acc / n;
     }
   }
 #pragma omp parallel for schedule(static)
   for (int64_t u = 0; u < nk; ++u) {
     const int64_t bh = u / nb, i = u % nb;
     const int64_t row0 = bh * S + i * block;
+    const int n = S - i * block < block ? (int)(S - i * block) : block;
     for (int d = 0; d < D; ++d) {
       double acc = 0.0;
-      for (int r = 0; r < block; ++r) acc += elem(k, dtype, (row0 + r) * D + d);
-      kbar[u * D + d] = acc / block;
+      for (int r = 0; r < n; ++r) acc += elem(k, dtype, (row0 + r) * D + d);
+      kbar[u * D + d] = acc / n;
     }
     double nacc = 0.0, nmax = 0.0;
-    for (int r = 0; r < block; ++r) {
+    for (int r = 0; r < n; ++r) {
       double sq = 0.0;
       for (int d = 0; d < D; ++d) {
         double x = elem(v, dtype, (row0 + r) * D + d);
@@ -170,7 +174,7 @@ void stem_oracle_pool(const void* q, const void* k, const void* v, int dtype, in
       nacc += norm;
       if (norm > nmax) nmax = norm;
     }
-    vnorm[u] = vmax ? nmax : nacc / block;
+    vnorm[u] = vmax ? nmax : nacc / n;
   }
 }
 
@@ -321,15 +325,16 @@ void stem_oracle_select(const double* m, const int32_t* k, const int64_t* off, i
  * keys are every token of every kept block j < i, plus tokens i*block .. r of
  * the diagonal block; logits Q[r].K[c] / sqrt(D); output sum_c softmax_c * V[c].
  *
- * Computes the listed query blocks only: rows[t] = (b*Hq + h)*nb + i.
- * out_rows [nrows, block, D] (double).
+ * Computes the listed query blocks only: rows[t] = (b*Hq + h)*nb + i,
+ * nb = ceil(S/block). out_rows [nrows, block, D] (double); rows of a partial
+ * last block past token S-1 are left 0.
  */
 void stem_oracle_attention(const void* q, const void* k, const void* v, int dtype, int B,
                            int Hq, int Hkv, int S, int D, int block,
                            const int32_t* sel_idx, const int32_t* sel_cnt,
                            const int64_t* off, int64_t cap, const int64_t* rows,
                            int64_t nrows, double* out_rows) {
-  const int nb = S / block;
+  const int nb = (S + block - 1) / block;
   const int G = Hq / Hkv;
   const double scale = 1.0 / sqrt((double)D);
   (void)B;
@@ -348,14 +353,18 @@ void stem_oracle_attention(const void* q, const void* k, const void* v, int dtyp
       const int64_t kvbase = (b * Hkv + h / G) * (int64_t)S; /* row index of token 0 */
       const int32_t* list = sel_idx + bh * cap + off[i];
       const int cnt = sel_cnt[u];
-      for (int r = 0; r < block; ++r) {
+      double* ob = out_rows + t * block * (int64_t)D;
+      for (int64_t e = 0; e < (int64_t)block * D; ++e) ob[e] = 0.0;
+      for (int r = 0; r < block && (int64_t)i * block + r < S; ++r) {
         const int64_t qtok = (int64_t)i * block + r;
         for (int d = 0; d < D; ++d) qrow[d] = elem(q, dtype, (bh * S + qtok) * D + d);
         int nkeys = 0;
         double mx = -INFINITY;
         for (int e = 0; e < cnt; ++e) {
           const int j = list[e];
-          const int last = (j == i) ? r : block - 1; /* token-causal on the diagonal */
+          /* token-causal on the diagonal; a partial last block has S - j*block tokens */
+          int last = (j == i) ? r : block - 1;
+          if ((int64_t)j * block + last > S - 1) last = (int)(S - 1 - (int64_t)j * block);
           for (int c = 0; c <= last; ++c) {
             const int64_t krow = kvbase + (int64_t)j * block + c;
             double dot = 0.0;

@@ -18,13 +18,16 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 
 def pool(q, k, v, block):
+    """Block means by slicing; a partial last block (S % block != 0) is the mean of its rows."""
     Q, K, V = f64(q), f64(k), f64(v)
     B, Hq, S, D = Q.shape
     Hkv = K.shape[1]
-    nb = S // block
-    qbar = Q.reshape(B, Hq, nb, block, D).mean(axis=3)
-    kbar = K.reshape(B, Hkv, nb, block, D).mean(axis=3)
-    vnorm = np.linalg.norm(V, axis=-1).reshape(B, Hkv, nb, block).mean(axis=3)
+    nb = -(-S // block)
+    blocks = [slice(i * block, min(S, (i + 1) * block)) for i in range(nb)]
+    qbar = np.stack([Q[:, :, sl].mean(axis=2) for sl in blocks], axis=2)
+    kbar = np.stack([K[:, :, sl].mean(axis=2) for sl in blocks], axis=2)
+    norms = np.linalg.norm(V, axis=-1)
+    vnorm = np.stack([norms[:, :, sl].mean(axis=2) for sl in blocks], axis=2)
     return qbar, kbar, vnorm
 
 
@@ -65,7 +68,7 @@ def attention_masked(q, k, v, block, kept):
     Q, K, V = f64(q), f64(k), f64(v)
     B, Hq, S, D = Q.shape
     G = Hq // K.shape[1]
-    nb = S // block
+    nb = -(-S // block)
     tok_block = np.arange(S) // block
     out = np.zeros_like(Q)
     for b in range(B):

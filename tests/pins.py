@@ -30,6 +30,10 @@ What pins what:
              scaled_dot_product_attention in float64; token 0 returns V[0];
              a constant-key block gives the mean of the visible V rows; dense
              token-mask brute force.
+  ragged S   S % block != 0: pooling and attention against the slicing / token-mask
+             brute force; a partial block of constant rows pools to that row; the
+             full blocks do not depend on the tokens past them (a prefix of the
+             sequence gives the same pooled values, selection and outputs).
 """
 
 from __future__ import annotations
@@ -495,6 +499,44 @@ def pin_attention_brute():
         np.testing.assert_allclose(res["out"].reshape(ref.shape), ref, rtol=1e-10, atol=1e-12)
 
 
+def pin_ragged():
+    for dtype in (torch.float32, torch.bfloat16):
+        S, block = 16 * 7 + 5, 16
+        q, k, v = _tiny_inputs(61, Hq=4, Hkv=2, S=S, D=16, block=block, dtype=dtype)
+        got = oracle.pool(q, k, v, block)
+        ref = brute.pool(q, k, v, block)
+        for a, b in zip(got, ref):
+            assert a.shape == b.shape and a.shape[2] == 8
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+        res = oracle.prefill(q, k, v, block, 0.3, 3.0, 2)
+        nb = 8
+        kept = _kept_from_csr(res["sel_idx"], res["sel_cnt"], res["off"], 1, 4, nb)
+        out = brute.attention_masked(q, k, v, block, kept)  # [1, 4, S, D]
+        got = res["out"].reshape(1, 4, nb, block, 16)
+        for h in range(4):
+            for i in range(nb):
+                n = min(block, S - i * block)
+                np.testing.assert_allclose(got[0, h, i, :n], out[0, h, i * block:i * block + n],
+                                           rtol=1e-10, atol=1e-12)
+                assert not got[0, h, i, n:].any(), "rows past S stay 0"
+        # prefix: the first 7 full blocks alone give the same everything for those blocks
+        pre = oracle.prefill(q[:, :, :112], k[:, :, :112], v[:, :, :112], block, 0.3, 3.0, 2)
+        for a, b in (("qbar", 2), ("kbar", 2), ("vnorm", 2)):
+            np.testing.assert_array_equal(res[a][:, :, :7], pre[a])
+        off7 = pre["off"]
+        np.testing.assert_array_equal(res["sel_idx"][:, :, :off7[7]], pre["sel_idx"])
+        np.testing.assert_array_equal(res["out"].reshape(1, 4, nb, block, 16)[:, :, :7],
+                                      pre["out"].reshape(1, 4, 7, block, 16))
+    # a partial block of 5 identical rows x pools to x, its V norm to |x|
+    x = torch.randn(1, 1, 1, 8, generator=torch.Generator().manual_seed(9))
+    z = torch.zeros(1, 1, 16, 8)
+    qq = torch.cat([z, x.repeat(1, 1, 5, 1)], dim=2)
+    qb, kb, vn = oracle.pool(qq, qq, qq, 16)
+    np.testing.assert_allclose(qb[0, 0, 1], x[0, 0, 0].double().numpy(), rtol=1e-12)
+    np.testing.assert_allclose(vn[0, 0, 1], float(torch.linalg.vector_norm(x.double())),
+                               rtol=1e-12)
+
+
 PINS = [
     pin_budget_decimal,
     pin_budget_closed_forms,
@@ -511,6 +553,7 @@ PINS = [
     pin_attention_dense_sdpa,
     pin_attention_closed_forms,
     pin_attention_brute,
+    pin_ragged,
 ]
 
 

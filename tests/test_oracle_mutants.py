@@ -30,7 +30,7 @@ MUTANTS = [
      "ceil(k_lin);\n    double kk = want > (double)k_min ? want : (double)k_min;\n"),
     ("linear-no-floor", "double want = ceil(k_lin);\n    double kk = want > (double)k_min ? want : (double)k_min;",
      "double want = ceil(k_lin);\n    double kk = want;"),
-    ("pool-divisor", "qbar[u * D + d] = acc / block;", "qbar[u * D + d] = acc / (block - 1);"),
+    ("pool-divisor", "qbar[u * D + d] = acc / n;", "qbar[u * D + d] = acc / (n - 1);"),
     ("pool-no-sqrt", "const double norm = sqrt(sq);", "const double norm = sq;"),
     ("pool-norm-of-mean", "sq += x * x;", "sq += x;"),
     ("metric-no-scale", "mrow[j] = dot * scale; /* s_ij", "mrow[j] = dot; /* s_ij"),
@@ -49,16 +49,23 @@ MUTANTS = [
     ("select-tie-order", "return (a->j > b->j) - (a->j < b->j);", "return (a->j < b->j) - (a->j > b->j);"),
     ("select-shift", "c[j - 1].m = mrow[j];", "c[j - 1].m = mrow[j - 1];"),
     ("select-no-sink", "chosen[n++] = 0;\n", "chosen[n++] = 1;\n"),
-    ("attn-no-causal", "const int last = (j == i) ? r : block - 1;", "const int last = block - 1;"),
+    ("attn-no-causal", "int last = (j == i) ? r : block - 1;", "int last = block - 1;"),
     ("attn-no-scale", "logit[nkeys] = dot * scale;", "logit[nkeys] = dot;"),
     ("attn-no-normalise", "const double w = logit[c] / z;", "const double w = logit[c];"),
     ("linear-denominator", "(double)i / (double)(nb - 1)", "(double)i / (double)nb"),
     ("linear-direction", "k_start * (1.0 - (1.0 - mu) * t)", "k_start * (mu + (1.0 - mu) * t)"),
     ("linear-floor", "double want = ceil(k_lin);", "double want = floor(k_lin);"),
-    ("pool-max-is-mean", "vnorm[u] = vmax ? nmax : nacc / block;", "vnorm[u] = nacc / block;"),
+    ("pool-max-is-mean", "vnorm[u] = vmax ? nmax : nacc / n;", "vnorm[u] = nacc / n;"),
     ("additive-no-clamp", "if (clamp && energy < 0.0) energy = 0.0;", ""),
     ("additive-no-square", "double energy = log(n * n);", "double energy = log(n);"),
     ("additive-no-scale", "mrow[j] = dot * scale + (beta", "mrow[j] = dot + (beta"),
+    ("ragged-nb-floor", "  const int nb = (S + block - 1) / block;\n  const int64_t nq",
+     "  const int nb = S / block;\n  const int64_t nq"),
+    ("ragged-divisor", "qbar[u * D + d] = acc / n;", "qbar[u * D + d] = acc / block;"),
+    ("ragged-vnorm-divisor", "vnorm[u] = vmax ? nmax : nacc / n;",
+     "vnorm[u] = vmax ? nmax : nacc / block;"),
+    ("ragged-last-rows", "for (int r = 0; r < block && (int64_t)i * block + r < S; ++r) {",
+     "for (int r = 0; r < block && (int64_t)i * block + r < S - 1; ++r) {"),
 ]
 
 
