@@ -172,14 +172,16 @@ Layout layout(int B, int Hq, int Hkv, int nb, int D) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+int nblocks(int S, int block) { return (S + block - 1) / block; }
+
 int check_shape(int B, int Hq, int Hkv, int S, int D, int block, int dtype) {
   if (B < 0 || S < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return STEM_ERR_ARG;
   if (D != 64 && D != 128) return STEM_ERR_ARG;
   if (block != 64 && block != 128) return STEM_ERR_ARG;
   if (dtype != STEM_BF16 && dtype != STEM_F32) return STEM_ERR_ARG;
-  if (S % block != 0) return STEM_ERR_ARG;
-  // element counts must fit comfortably in int64 and grid sizes in int32
-  const int64_t nb = S / block;
+  // element counts must fit comfortably in int64 and grid sizes in int32; a partial last block
+  // (S % block != 0) is a block of its own
+  const int64_t nb = nblocks(S, block);
   if (static_cast<int64_t>(B) * Hq * nb > 0x7fffffffLL / 4) return STEM_ERR_UNSUPPORTED;
   if (nb > STEM_MAX_NB) return STEM_ERR_UNSUPPORTED;
   return STEM_OK;
@@ -238,7 +240,7 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   if (a == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(a->B, a->Hq, a->Hkv, a->S, a->D, a->block, a->dtype);
   if (rc != STEM_OK) return rc;
-  const int nb = a->S / a->block;
+  const int nb = nblocks(a->S, a->block);
   const stem_method_t m = args_method(a);
   rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
@@ -378,7 +380,7 @@ int64_t stem_sel_capacity(int nb, float rho_min, float tau, int k_min) {
 size_t stem_workspace_size(int B, int Hq, int Hkv, int S, int D, int block) {
   if (check_shape(B, Hq, Hkv, S, D, block, STEM_BF16) != STEM_OK) return 0;
   if (is_empty(B, S)) return 0;
-  return layout(B, Hq, Hkv, S / block, D).total;
+  return layout(B, Hq, Hkv, nblocks(S, block), D).total;
 }
 
 const char* stem_strerror(int code) {
@@ -421,7 +423,7 @@ int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int
   int rc = check_shape(B, Hq, Hkv, S, D, block, STEM_BF16);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, S)) return run_prefill(&a, nullptr);
-  rc = check_params(S / block, default_method(rho_min, tau, k_min));
+  rc = check_params(nblocks(S, block), default_method(rho_min, tau, k_min));
   if (rc != STEM_OK) return rc;
   a.workspace_bytes = stem_workspace_size(B, Hq, Hkv, S, D, block);
   rc = get_scratch(a.workspace_bytes, &a.workspace, 0);
@@ -433,7 +435,7 @@ int stem_prefill_host(const stem_args_t* h) {
   if (h == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(h->B, h->Hq, h->Hkv, h->S, h->D, h->block, h->dtype);
   if (rc != STEM_OK) return rc;
-  const int nb = h->S / h->block;
+  const int nb = nblocks(h->S, h->block);
   const stem_method_t m = args_method(h);
   rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
@@ -556,7 +558,7 @@ int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, i
   if (m == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
   if (rc != STEM_OK) return rc;
-  const int nb = S / block;
+  const int nb = nblocks(S, block);
   rc = check_params(nb, *m);
   if (rc != STEM_OK) return rc;
   if (is_empty(B, S)) return STEM_OK;

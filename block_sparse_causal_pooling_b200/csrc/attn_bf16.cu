@@ -10,7 +10,8 @@
 // (XOR-swizzled 16-byte chunks, conflict-free ldmatrix); S = Q K^T and O += P V run on
 // mma.sync.m16n8k16 (bf16 in, f32 accumulate) with an online softmax in float32 (exp2 with the
 // 1/sqrt(D) scale folded in). Work items are ordered kv-head-group-major so the CTAs in flight
-// share one kv head's K/V in L2, heaviest query blocks first.
+// share one kv head's K/V in L2, heaviest query blocks first. In a partial last block (S not a
+// multiple of BLOCK) rows past S are zero-filled on load and never stored.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -27,6 +28,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+// 16 bytes, or 16 zero bytes (nothing read) when !valid; src must still point into the tensor.
+__device__ __forceinline__ void cp_async16z(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0));
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
@@ -112,8 +118,10 @@ __global__ void __launch_bounds__(BLOCK * 2) attn_bf16_mma_kernel(
     const uint32_t vb = smem_u32(vs + stage * kKT * D * 2);
     for (int idx = t; idx < kKT * CH; idx += NT) {
       const int r = idx / CH, c = idx % CH;
-      cp_async16(kb + swz<D>(r, c), ksrc + (row0 + r) * D + c * 8);
-      cp_async16(vb + swz<D>(r, c), vsrc + (row0 + r) * D + c * 8);
+      const bool ok = row0 + r < S;
+      const int64_t rr = ok ? row0 + r : S - 1;
+      cp_async16z(kb + swz<D>(r, c), ksrc + rr * D + c * 8, ok);
+      cp_async16z(vb + swz<D>(r, c), vsrc + rr * D + c * 8, ok);
     }
   };
 
@@ -122,7 +130,8 @@ __global__ void __launch_bounds__(BLOCK * 2) attn_bf16_mma_kernel(
     const uint32_t qb = smem_u32(qs);
     for (int idx = t; idx < BLOCK * CH; idx += NT) {
       const int r = idx / CH, c = idx % CH;
-      cp_async16(qb + swz<D>(r, c), qsrc + static_cast<int64_t>(r) * D + c * 8);
+      const bool ok = static_cast<int64_t>(i) * BLOCK + r < S;
+      cp_async16z(qb + swz<D>(r, c), qsrc + static_cast<int64_t>(ok ? r : 0) * D + c * 8, ok);
     }
   }
   load_tile(0, 0);
@@ -243,6 +252,7 @@ __global__ void __launch_bounds__(BLOCK * 2) attn_bf16_mma_kernel(
     l += __shfl_xor_sync(0xffffffffu, l, 2);
     const float inv = 1.0f / l;
     const int64_t tok = static_cast<int64_t>(i) * BLOCK + wrow + gq + hr * 8;
+    if (tok >= S) continue;  // partial last block
     __nv_bfloat16* dst = out + (bh * S + tok) * D;
 #pragma unroll
     for (int n = 0; n < NTD; ++n) {
@@ -256,7 +266,7 @@ template <int D, int BLOCK>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
                          int S, PlanDev plan, int64_t cap, const int32_t* sel_idx, void* out,
                          cudaStream_t st) {
-  const int nb = S / BLOCK;
+  const int nb = (S + BLOCK - 1) / BLOCK;
   const int64_t items = static_cast<int64_t>(B) * Hq * nb;
   if (items == 0) return cudaSuccess;
   if (items > 0x7fffffff) return cudaErrorInvalidConfiguration;

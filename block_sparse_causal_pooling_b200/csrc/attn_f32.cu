@@ -41,7 +41,9 @@ __global__ void __launch_bounds__(BLOCK* kTPR) attn_f32_kernel(
   const int t = threadIdx.x;
   const int r = t / kTPR;   // query row within the block
   const int part = t % kTPR;
-  const int64_t qrow = bh * S + static_cast<int64_t>(i) * BLOCK + r;
+  const int64_t qtok = static_cast<int64_t>(i) * BLOCK + r;
+  const bool qvalid = qtok < S;  // rows past S of a partial last block: computed on 0, not stored
+  const int64_t qrow = bh * S + (qvalid ? qtok : S - 1);
   const float* kvk = k + (bg * S) * D;
   const float* kvv = v + (bg * S) * D;
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(BLOCK* kTPR) attn_f32_kernel(
   float qv[DS], o[DS];
 #pragma unroll
   for (int d = 0; d < DS; ++d) {
-    qv[d] = q[qrow * D + part * DS + d] * scale;
+    qv[d] = qvalid ? q[qrow * D + part * DS + d] * scale : 0.f;
     o[d] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
@@ -61,9 +63,12 @@ __global__ void __launch_bounds__(BLOCK* kTPR) attn_f32_kernel(
     __syncthreads();
     const float4* srcK = reinterpret_cast<const float4*>(kvk + static_cast<int64_t>(j) * BLOCK * D);
     const float4* srcV = reinterpret_cast<const float4*>(kvv + static_cast<int64_t>(j) * BLOCK * D);
+    const int nrows = static_cast<int>(min(static_cast<int64_t>(BLOCK),
+                                           S - static_cast<int64_t>(j) * BLOCK));
     for (int idx = t; idx < BLOCK * D / 4; idx += BLOCK * kTPR) {
-      reinterpret_cast<float4*>(ks)[idx] = srcK[idx];
-      reinterpret_cast<float4*>(vs)[idx] = srcV[idx];
+      const bool ok = idx / (D / 4) < nrows;  // rows past S: zeros (causally masked anyway)
+      reinterpret_cast<float4*>(ks)[idx] = ok ? srcK[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(vs)[idx] = ok ? srcV[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     const int last = (j == i) ? r : BLOCK - 1;  // token-causal on the diagonal block
@@ -101,6 +106,7 @@ __global__ void __launch_bounds__(BLOCK* kTPR) attn_f32_kernel(
     }
   }
   const float inv = 1.0f / l;
+  if (!qvalid) return;
 #pragma unroll
   for (int d = 0; d < DS; ++d) out[qrow * D + part * DS + d] = o[d] * inv;
 }
@@ -109,7 +115,7 @@ template <int D, int BLOCK>
 cudaError_t launch_typed(const float* q, const float* k, const float* v, int B, int Hq, int Hkv,
                          int S, PlanDev plan, int64_t cap, const int32_t* sel_idx, float* out,
                          cudaStream_t st) {
-  const int nb = S / BLOCK;
+  const int nb = (S + BLOCK - 1) / BLOCK;
   const int64_t items = static_cast<int64_t>(B) * Hq * nb;
   if (items == 0) return cudaSuccess;
   if (items > 0x7fffffff) return cudaErrorInvalidConfiguration;

@@ -157,12 +157,13 @@ __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
   }
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+// Box (x: 64 columns, y: 128 tokens, z: one head) of a [heads, S, D] view; rows past S read 0.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
                                             uint64_t* bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar)), "l"(policy)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(su32(bar)), "l"(policy)
       : "memory");
 }
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -457,10 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(&bars->kv_empty[s], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
           return false;
         mbar_expect_tx(&bars->kv_full[s], C::kTile);
-        const int row =
-            static_cast<int>((static_cast<int64_t>(st.it.b) * Hkv + st.it.g) * S) + blk * kN;
+        const int head = st.it.b * Hkv + st.it.g;
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_2d(kv_tiles + s * C::kTile + x * (kN * 128), map, x * 64, row,
+          tma_load_3d(kv_tiles + s * C::kTile + x * (kN * 128), map, x * 64, blk * kN, head,
                       &bars->kv_full[s], pol_kv);
         slot_round[s] = r;
         ++f;
@@ -472,11 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         mbar_expect_tx(&bars->q_full[tile], C::kTile);
         const int h = tile == 0 ? st.it.hA : st.it.hB;
-        const int qrow = static_cast<int>((static_cast<int64_t>(st.it.b) * Hq + h) * S +
-                                          static_cast<int64_t>(st.it.i) * kM);
         for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_2d(q_tiles + tile * C::kTile + x * (kM * 128), &tm_q, x * 64, qrow,
-                      &bars->q_full[tile], pol_q);
+          tma_load_3d(q_tiles + tile * C::kTile + x * (kM * 128), &tm_q, x * 64, st.it.i * kM,
+                      st.it.b * Hq + h, &bars->q_full[tile], pol_q);
         ++q_loads[tile];
         return true;
       };
@@ -755,6 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = tl == 0 ? it.hA : it.hB;
       __nv_bfloat16* dst = out + ((static_cast<int64_t>(it.b) * Hq + h) * S +
                                   static_cast<int64_t>(it.i) * kM + row) * D + half * kDH;
+      const bool valid = static_cast<int64_t>(it.i) * kM + row < S;  // partial last block
       const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
 #pragma unroll
       for (int c = 0; c < kDH / 32; ++c) {
@@ -767,8 +766,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e)
           wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+        if (valid) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) __stcs(d4 + e, pk[e]);  // evict-first: keep K/V in L2
+          for (int e = 0; e < 4; ++e) __stcs(d4 + e, pk[e]);  // evict-first: keep K/V in L2
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars->o_empty[tl]);
@@ -833,15 +834,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D view [rows, D] of a bf16 tensor, boxes of 64 columns x 128 rows, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
+// 3-D view [heads, S, D] of a bf16 tensor, boxes of 64 columns x 128 tokens x 1 head, 128B
+// swizzle. Token rows past S are outside the view: a box over a partial last block reads them
+// as 0 instead of the next head's first rows.
+bool make_map(CUtensorMap* m, const void* base, uint64_t heads, int S, int D) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), heads};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -850,14 +853,14 @@ template <int D>
 cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
                          int S, PlanDev plan, int64_t cap, const int32_t* sel_idx,
                          uint32_t* sched, void* out, int32_t* status, cudaStream_t st) {
-  const int nb = S / kM;
+  const int nb = (S + kM - 1) / kM;
   const int G = Hq / Hkv;
   const int64_t items = static_cast<int64_t>(B) * Hkv * nb * ((G + 1) / 2);  // head pairs
   if (items == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, static_cast<uint64_t>(B) * Hq * S, D) ||
-      !make_map(&tk, k, static_cast<uint64_t>(B) * Hkv * S, D) ||
-      !make_map(&tv, v, static_cast<uint64_t>(B) * Hkv * S, D))
+  if (!make_map(&tq, q, static_cast<uint64_t>(B) * Hq, S, D) ||
+      !make_map(&tk, k, static_cast<uint64_t>(B) * Hkv, S, D) ||
+      !make_map(&tv, v, static_cast<uint64_t>(B) * Hkv, S, D))
     return cudaErrorInvalidValue;
   // one CTA per SM: each CTA takes all 512 TMEM columns
   const size_t smem = std::max<size_t>(1024 + (2 + kSlots) * Cfg<D>::kTile + sizeof(Bars),

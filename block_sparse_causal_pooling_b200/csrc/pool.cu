@@ -6,6 +6,8 @@
 //   kbar[b,g,i,:] = mean of K rows of block i,
 //   vnorm[b,g,i]  = mean over the block's rows of the row's Euclidean norm, or (vmax) the
 //                   largest row norm ("maximised magnitudes of V", gist.science/nl step 1).
+// A partial last block (S % block != 0) is pooled over its S - i*block rows: rows past S are
+// neither read nor counted.
 //
 // Design (HBM-bound: every input byte is read once, outputs are ~1/64 of the input):
 //   - one CTA of 256 threads per (tensor, b, head, block) unit; a unit is one contiguous
@@ -98,10 +100,14 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict_
   const int64_t i = unit % nb;
   const uint4* base =
       reinterpret_cast<const uint4*>(src + (bh * S + i * BLOCK) * static_cast<int64_t>(D));
+  const int n = static_cast<int>(min(static_cast<int64_t>(BLOCK), S - i * BLOCK));  // rows
 
   uint4 raw[ITERS];
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) raw[it] = __ldcs(base + (rg + it * RPI) * CPR + c);
+  for (int it = 0; it < ITERS; ++it) {
+    const int row = rg + it * RPI;
+    raw[it] = row < n ? __ldcs(base + row * CPR + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
 
   if (kind < 2) {
     float acc[E];
@@ -128,7 +134,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict_
       __syncthreads();
     }
     float* dst = (kind == 0 ? qbar : kbar) + unit * D;
-    for (int d = t; d < D; d += kPoolThreads) dst[d] = part[0][d] * (1.0f / BLOCK);
+    for (int d = t; d < D; d += kPoolThreads) dst[d] = part[0][d] / static_cast<float>(n);
   } else {
     float norms[ITERS];
 #pragma unroll
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const T* __restrict_
       if (t < s) part[t][0] = vmax ? fmaxf(part[t][0], part[t + s][0]) : part[t][0] + part[t + s][0];
       __syncthreads();
     }
-    if (t == 0) vnorm[unit] = vmax ? part[0][0] : part[0][0] * (1.0f / BLOCK);
+    if (t == 0) vnorm[unit] = vmax ? part[0][0] : part[0][0] / static_cast<float>(n);
   }
 }
 
@@ -165,7 +171,7 @@ template <typename T, int D, int BLOCK>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
                          int S, bool vmax, float* qbar, float* kbar, float* vnorm,
                          cudaStream_t st) {
-  const int nb = S / BLOCK;
+  const int nb = (S + BLOCK - 1) / BLOCK;
   const int64_t nq = static_cast<int64_t>(B) * Hq * nb;
   const int64_t nk = static_cast<int64_t>(B) * Hkv * nb;
   const int64_t units = nq + 2 * nk;

@@ -197,7 +197,7 @@ def alloc_outputs(q: torch.Tensor, k: torch.Tensor, block: int, rho_min: float, 
                   k_min: int, method=None):
     """(out, sel_idx, sel_cnt) allocated on q's device."""
     B, Hq, Hkv, S, D = _shape(q, k)
-    nb = S // block
+    nb = -(-S // block)  # a partial last block counts
     cap = stem_sel_capacity(nb, rho_min, tau, k_min, method)
     out = torch.empty_like(q)
     sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=q.device)
@@ -271,7 +271,7 @@ def stem_prefill_host(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt
 
 def stem_pool(q, k, v, block, qbar=None, kbar=None, vnorm=None, stream=None, method=None):
     B, Hq, Hkv, S, D = _shape(q, k)
-    nb = S // block
+    nb = -(-S // block)  # a partial last block counts
     dev = q.device
     if qbar is None:
         qbar = torch.empty((B, Hq, nb, D), dtype=torch.float32, device=dev)

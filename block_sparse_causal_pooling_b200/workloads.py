@@ -54,7 +54,7 @@ class Workload:
 
     @property
     def nb(self) -> int:
-        return self.S // self.block
+        return -(-self.S // self.block)  # a partial last block counts
 
     @property
     def torch_dtype(self) -> torch.dtype:

@@ -11,7 +11,7 @@
  * attention over Q, K, V in which each query block attends only to a kept set of
  * key blocks. The pages leave the budget schedule and the pooling open; this
  * library fixes them as parameters:
- *   nb = S / block, query block i in [0, nb);
+ *   nb = ceil(S / block), query block i in [0, nb);
  *   rho(i) = rho_min + (1 - rho_min) * exp(-i / tau);
  *   k(i)   = min(i+1, max(k_min, ceil(rho(i) * (i+1)))), raised to 2 for i >= 1, k(0) = 1;
  *   pooled qbar_i, kbar_j = mean of the block's rows; n_j = mean of the block's V-row L2 norms;
@@ -33,8 +33,11 @@
  *   - CSR layout of the kept blocks: row (b, h, i) occupies
  *       sel_idx[(b*Hq + h)*cap + off(i) .. + k(i)), ascending block indices,
  *     with off(i) = k(0) + ... + k(i-1) and cap = off(nb) (stem_sel_capacity); sel_cnt[b,h,i] = k(i).
- *   - Supported shapes: D in {64, 128}; block in {64, 128}; S % block == 0; Hq % Hkv == 0;
- *     nb <= STEM_MAX_NB. B == 0 or S == 0 is an empty problem: success, nothing launched.
+ *   - Supported shapes: D in {64, 128}; block in {64, 128}; Hq % Hkv == 0; any S >= 0, with
+ *     nb = ceil(S / block) <= STEM_MAX_NB. When S is not a multiple of block the last block
+ *     holds the S - (nb-1)*block remaining tokens: it is pooled over those rows only, and
+ *     out rows past S are never written. B == 0 or S == 0 is an empty problem: success,
+ *     nothing launched.
  *   - Device calls are asynchronous on the given stream: a 0 return means the work was enqueued.
  *     Faults surface at the caller's next synchronisation. The library never prints or aborts.
  *   - Arguments are validated before anything is enqueued; on a negative return nothing was

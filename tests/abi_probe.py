@@ -43,7 +43,7 @@ res = {
     "hkv_zero": ex(Hkv=0),
     "d_96": ex(D=96),
     "block_32": ex(block=32),
-    "ragged_S": ex(S=1000),
+    "negative_S": ex(S=-128),
     "negative_B": ex(B=-1),
     "dtype_7": ex(dtype=7),
     "rho_zero": ex(rho_min=0.0),
@@ -65,7 +65,7 @@ res = {
     "empty_S": ex(S=0, q=None, k=None, v=None, out=None, sel_idx=None, sel_cnt=None),
     "ex_null_args": L.stem_prefill_ex(None, None),
     "host_null_args": L.stem_prefill_host(None),
-    "host_ragged": L.stem_prefill_host(ctypes.byref(base(S=1000))),
+    "host_bad_block": L.stem_prefill_host(ctypes.byref(base(block=96))),
     "simple_bad_block": L.stem_prefill(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 96, 0.25, 4.0, 2,
                                        FAKE, FAKE, FAKE),
     "simple_bad_rho": L.stem_prefill(FAKE, FAKE, FAKE, 1, 4, 2, 1024, 128, 128, -0.1, 4.0, 2,
@@ -123,7 +123,7 @@ res.update({
     "attn_m_bad_beta": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128,
                                             M(BAD_BETA), FAKE, FAKE, FAKE, FAKE, 1 << 20, None,
                                             None),
-    "attn_m_ragged": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1000, 128, 128, M(GOOD),
+    "attn_m_bad_block": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1000, 128, 96, M(GOOD),
                                           FAKE, FAKE, FAKE, FAKE, 1 << 20, None, None),
 })
 print(json.dumps(res))

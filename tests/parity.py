@@ -80,9 +80,11 @@ def compare_selection(gpu_idx, gpu_cnt, ref_idx, ref_cnt, m_ref, k, off, rel=REL
 
 
 def out_rows(out: torch.Tensor, rows, block: int) -> np.ndarray:
-    """GPU output gathered to [len(rows), block, D] float64 for the listed (b, h, i)."""
+    """GPU output gathered to [len(rows), block, D] float64 for the listed (b, h, i). Rows of
+    a partial last block past the sequence end are 0, as in the oracle's output."""
     o = out.detach()
-    parts = [o[b, h, i * block:(i + 1) * block] for (b, h, i) in rows]
+    pad = lambda x: torch.nn.functional.pad(x, (0, 0, 0, block - x.shape[0]))  # noqa: E731
+    parts = [pad(o[b, h, i * block:(i + 1) * block]) for (b, h, i) in rows]
     if not parts:
         return np.zeros((0, block, out.shape[-1]))
     return torch.stack(parts).double().cpu().numpy()

@@ -108,7 +108,10 @@ def test_workspace_size_layout():
     # head-pair step schedule, bounded for any budget: one uint32 per causal block pair
     sched = 4 * B * Hkv * ((Hq // Hkv + 1) // 2) * nb * (nb + 1) // 2
     assert pooled + sched < n < pooled + sched + 64 * 1024
-    assert S.stem_workspace_size(B, Hq, Hkv, 1000, D, block) == 0  # ragged: invalid
+    # a partial last block is a block of its own: 1000 tokens need the layout of 8 blocks
+    assert S.stem_workspace_size(B, Hq, Hkv, 1000, D, block) == \
+        S.stem_workspace_size(B, Hq, Hkv, 1024, D, block) > 0
+    assert S.stem_workspace_size(B, Hq, Hkv, 1000, 96, block) == 0  # unsupported D
     assert S.stem_workspace_size(0, Hq, Hkv, Sq, D, block) == 0  # empty
 
 

@@ -21,7 +21,9 @@ from tests import parity
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 DEV = "cuda:0"
-FULL = [wl.LLAMA_32K, wl.LLAMA_128K, wl.QWEN_64K] + list(wl.SWEEP_128K[1:]) + list(wl.SWEEP_B4_16K)
+FULL = ([wl.LLAMA_32K, wl.LLAMA_128K, wl.QWEN_64K] + list(wl.SWEEP_128K[1:]) +
+        list(wl.SWEEP_B4_16K) +
+        [wl.LLAMA_128K.replace(name="llama3-8b-128k-ragged", S=131072 - 37)])
 ORACLE_GFLOP_BUDGET = 40.0
 
 

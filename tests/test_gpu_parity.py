@@ -35,6 +35,16 @@ CASES = {
                                   k_min=1),
     "dense": wl.LLAMA_32K.replace(name="dense", Hq=4, Hkv=2, S=2048, rho_min=1.0),
     "nb37": wl.LLAMA_32K.replace(name="nb37", Hq=2, Hkv=2, S=37 * 128, tau=5.0),
+    # sequences that end inside a block (the last block holds the remaining tokens)
+    "ragged-blk128": wl.LLAMA_32K.replace(name="ragged-blk128", Hq=4, Hkv=2, S=37 * 128 + 77,
+                                          tau=5.0),
+    "ragged-one-token": wl.LLAMA_32K.replace(name="ragged-one-token", Hq=2, Hkv=1,
+                                             S=20 * 128 + 1, tau=5.0),
+    "ragged-short": wl.LLAMA_32K.replace(name="ragged-short", Hq=2, Hkv=1, S=100),
+    "ragged-blk64": wl.LLAMA_32K.replace(name="ragged-blk64", Hq=4, Hkv=2, S=40 * 64 + 13,
+                                         block=64, tau=8.0),
+    "ragged-f32": wl.TINY.replace(name="ragged-f32", Hq=4, Hkv=2, S=16 * 128 + 100, D=128,
+                                  block=128),
 }
 
 
