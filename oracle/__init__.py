@@ -162,6 +162,21 @@ def metric_additive(qbar: np.ndarray, kbar: np.ndarray, vnorm: np.ndarray, beta:
     return m
 
 
+def metric_group(m: np.ndarray, G: int) -> np.ndarray:
+    """GQA-group metric: the per-head metric summed over the G query heads that share a
+    kv-head (heads g*G .. g*G+G-1), [B, Hq/G, T]. The pages are silent on GQA; this is the
+    group-shared selection's score (one kept list per kv-head group)."""
+    B, Hq, T = m.shape
+    return m.reshape(B, Hq // G, G, T).sum(axis=2)
+
+
+def select_group(mg: np.ndarray, k: np.ndarray, off: np.ndarray, G: int):
+    """Selection from a group metric [B, Hkv, T], replicated to the G query heads of each
+    group: sel_idx [B, Hq, cap], sel_cnt [B, Hq, nb]."""
+    gi, gc = select(mg, k, off)
+    return np.repeat(gi, G, axis=1), np.repeat(gc, G, axis=1)
+
+
 def metric_row(m: np.ndarray, b: int, h: int, i: int) -> np.ndarray:
     """Row i (j = 0..i) of a packed metric."""
     s = i * (i + 1) // 2
@@ -216,11 +231,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
             tau: float, k_min: int, rows: Optional[Sequence] = None, with_metric: bool = True,
             schedule: str = "exp", k_start: float = 0.0, mu: float = 1.0,
             metric_form: str = "product", beta: float = 0.0, clamp: bool = True,
-            vsum: str = "mean"):
+            vsum: str = "mean", share: str = "head"):
     """All stages. Returns a dict with k, off, qbar, kbar, vnorm, m, sel_idx, sel_cnt and
     out ([len(rows), block, D] for the listed query blocks; all blocks when rows is None).
     schedule "exp" uses rho_min, tau; "linear" uses k_start, mu. metric_form "product" is
-    softmax(s) * n, "additive" is s + beta * max(0, log n^2) (clamp=False drops the max)."""
+    softmax(s) * n, "additive" is s + beta * max(0, log n^2) (clamp=False drops the max).
+    share "group" selects once per kv-head group by the metric summed over its query heads
+    (metric_group); m is then the group metric replicated to each head."""
     B, Hq, S, D = q.shape
     nb = -(-S // block)
     if schedule == "exp":
@@ -236,7 +253,14 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
         m = metric_additive(qbar, kbar, vnorm, beta, clamp)
     else:
         raise ValueError(metric_form)
-    sel_idx, sel_cnt = select(m, kk, off)
+    if share == "group":
+        G = q.shape[1] // k.shape[1]
+        m = np.repeat(metric_group(m, G), G, axis=1)  # every head of a group: the group metric
+        sel_idx, sel_cnt = select_group(m[:, ::G], kk, off, G)
+    elif share == "head":
+        sel_idx, sel_cnt = select(m, kk, off)
+    else:
+        raise ValueError(share)
     out = attention(q, k, v, block, sel_idx, sel_cnt, off, rows)
     res = dict(k=kk, off=off, qbar=qbar, kbar=kbar, vnorm=vnorm, sel_idx=sel_idx,
                sel_cnt=sel_cnt, out=out)

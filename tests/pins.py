@@ -30,6 +30,10 @@ What pins what:
              scaled_dot_product_attention in float64; token 0 returns V[0];
              a constant-key block gives the mean of the visible V rows; dense
              token-mask brute force.
+  group      GQA-group-shared selection: G = 1 is the per-head selection; query heads
+             that are all equal give the per-head selection of any of them; the full
+             sort of the numpy brute-force metric summed over the group's heads; the
+             additive form sums to sum_h s + G*beta*e.
   ragged S   S % block != 0: pooling and attention against the slicing / token-mask
              brute force; a partial block of constant rows pools to that row; the
              full blocks do not depend on the tokens past them (a prefix of the
@@ -499,6 +503,40 @@ def pin_attention_brute():
         np.testing.assert_allclose(res["out"].reshape(ref.shape), ref, rtol=1e-10, atol=1e-12)
 
 
+def pin_group():
+    q, k, v = _tiny_inputs(71, Hq=4, Hkv=2, S=256, D=16, block=16)
+    G = 2
+    # G = 1: one head per group, the group metric is the head's metric
+    res1 = oracle.prefill(q[:, :2], k, v, 16, 0.2, 3.0, 2)
+    resg = oracle.prefill(q[:, :2], k, v, 16, 0.2, 3.0, 2, share="group")
+    np.testing.assert_array_equal(res1["sel_idx"], resg["sel_idx"])
+    # identical query heads in each group: the group keeps what each head keeps
+    qq = q[:, ::G].repeat_interleave(G, dim=1)
+    ref = oracle.prefill(qq, k, v, 16, 0.2, 3.0, 2)
+    got = oracle.prefill(qq, k, v, 16, 0.2, 3.0, 2, share="group")
+    np.testing.assert_array_equal(got["sel_idx"], ref["sel_idx"])
+    # brute force: numpy metric summed over the group's heads, full sort, replicated
+    res = oracle.prefill(q, k, v, 16, 0.2, 3.0, 2, share="group")
+    md = brute.metric_dense(*brute.pool(q, k, v, 16))  # [B, Hq, nb, nb]
+    mg = md.reshape(1, 2, G, 16, 16).sum(axis=2)
+    rows = brute.select_rows(mg, res["k"])
+    kept = _kept_from_csr(res["sel_idx"], res["sel_cnt"], res["off"], 1, 4, 16)
+    for (b, g, i), lst in rows.items():
+        for h in range(G):
+            assert kept[(b, g * G + h, i)] == lst, (g, h, i)
+    # additive: the group score is sum_h s + G * beta * max(0, log n^2)
+    qb, kb, vn = oracle.pool(q, k, v, 16)
+    ma = oracle.metric_additive(qb, kb, vn, 0.2, True)
+    mga = oracle.metric_group(ma, G)
+    beta = float(np.float32(0.2))
+    for g in range(2):
+        for i in (3, 9, 15):
+            s_sum = sum(qb[0, g * G + h, i] @ kb[0, g, : i + 1].T for h in range(G)) / 4.0
+            e = np.maximum(0.0, np.log(vn[0, g, : i + 1] ** 2))
+            np.testing.assert_allclose(oracle.metric_row(mga, 0, g, i), s_sum + G * beta * e,
+                                       rtol=1e-12, atol=1e-12)
+
+
 def pin_ragged():
     for dtype in (torch.float32, torch.bfloat16):
         S, block = 16 * 7 + 5, 16
@@ -554,6 +592,7 @@ PINS = [
     pin_attention_closed_forms,
     pin_attention_brute,
     pin_ragged,
+    pin_group,
 ]
 
 
