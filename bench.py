@@ -58,11 +58,11 @@ def parse():
     p.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--method", choices=["default", "pages"], default="default",
+    p.add_argument("--method", choices=["default", "pages", "group"], default="default",
                    help="default: exponential budget, product metric, mean V norms; pages: the "
                         "pages' linear budget (mu 0.7) with the additive metric (beta 0.2, "
                         "clamped) and max-pooled V norms, k_start set for the default's mean "
-                        "budget")
+                        "budget; group: the default with one selection per kv-head group")
     return p.parse_args()
 
 
@@ -169,6 +169,8 @@ def method_params(w, name):
     same mean as the workload's default budget, 2 * mean / (1 + mu), to one decimal."""
     if name == "default":
         return None
+    if name == "group":
+        return dict(schedule="exp", rho_min=w.rho_min, tau=w.tau, k_min=w.k_min, share="group")
     from block_sparse_causal_pooling_b200 import stem as S
 
     kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
@@ -188,15 +190,19 @@ def oracle_sample_step(w, q, k, v, rows, mp=None):
     G = w.Hq // w.Hkv
     qs, ks, vs = q[:, :G].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous()
     t0 = time.perf_counter()
-    if mp is None:
+    if mp is None or mp.get("schedule") == "exp":
         kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
-        qb, kb, vn = oracle.pool(qs, ks, vs, w.block)
-        m = oracle.metric(qb, kb, vn)
     else:
         kk, off = oracle.budget_linear(w.nb, mp["k_start"], mp["mu"], mp["k_min"])
-        qb, kb, vn = oracle.pool(qs, ks, vs, w.block, mp["vsum"])
+    qb, kb, vn = oracle.pool(qs, ks, vs, w.block, "mean" if mp is None else mp.get("vsum", "mean"))
+    if mp is not None and mp.get("metric") == "additive":
         m = oracle.metric_additive(qb, kb, vn, mp["beta"], mp["clamp"])
-    si, sc = oracle.select(m, kk, off)
+    else:
+        m = oracle.metric(qb, kb, vn)
+    if mp is not None and mp.get("share") == "group":
+        si, sc = oracle.select_group(oracle.metric_group(m, G), kk, off, G)
+    else:
+        si, sc = oracle.select(m, kk, off)
     t1 = time.perf_counter()
     oracle.attention(qs, ks, vs, w.block, si, sc, off, rows)
     t2 = time.perf_counter()

@@ -39,6 +39,7 @@ stem_method_t default_method(float rho_min, float tau, int k_min) {
   m.metric = STEM_METRIC_PRODUCT;
   m.clamp = 1;
   m.vsum = STEM_VSUM_MEAN;
+  m.share = STEM_SHARE_HEAD;
   return m;
 }
 
@@ -61,6 +62,7 @@ bool method_ok(int nb, const stem_method_t& m) {
   } else if (m.metric != STEM_METRIC_PRODUCT) {
     return false;
   }
+  if (m.share != STEM_SHARE_HEAD && m.share != STEM_SHARE_GROUP) return false;
   return m.vsum == STEM_VSUM_MEAN || m.vsum == STEM_VSUM_MAX;
 }
 
@@ -200,6 +202,7 @@ int check_params(int nb, const stem_method_t& m) {
   // off[] is int32: the capacity must fit
   const int64_t cap = capacity(nb, m);
   if (cap > 0x7fffffffLL) return STEM_ERR_UNSUPPORTED;
+  if (m.share == STEM_SHARE_GROUP && nb > kGroupMaxNb) return STEM_ERR_UNSUPPORTED;
   return STEM_OK;
 }
 
@@ -208,6 +211,7 @@ SelMetric sel_metric(const stem_method_t& m) {
   s.additive = m.metric == STEM_METRIC_ADDITIVE;
   s.beta = m.beta;
   s.clamp = m.clamp != 0;
+  s.group = m.share == STEM_SHARE_GROUP;
   return s;
 }
 

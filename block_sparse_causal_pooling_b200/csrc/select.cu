@@ -44,6 +44,141 @@ __device__ __forceinline__ uint64_t order_bits(double x) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
+// Kept set of row i: {0, i} plus the k(i)-2 largest keys over j in [1, i-1] (equal keys: lower
+// j first), written ascending to dst + t*dstride for t < ndst (the same list at every
+// destination). One warp; key_bits(j) is the order-preserving image of column j's key; hist is
+// the warp's 256-bin histogram.
+template <typename KeyBits>
+__device__ __forceinline__ void select_row(int i, int kk, KeyBits key_bits, int* hist, int lane,
+                                           int32_t* dst, int64_t dstride, int ndst) {
+  const unsigned lt_mask = (1u << lane) - 1u;
+  if (i == 0) {
+    if (lane == 0)
+      for (int t = 0; t < ndst; ++t) dst[t * dstride] = 0;
+    return;
+  }
+  const int need = kk - 2;  // picks among j in [1, i-1]
+  if (need >= i - 1) {      // every causal block
+    for (int j = lane; j <= i; j += 32)
+      for (int t = 0; t < ndst; ++t) dst[t * dstride + j] = j;
+    return;
+  }
+  if (need <= 0) {
+    if (lane == 0)
+      for (int t = 0; t < ndst; ++t) {
+        dst[t * dstride] = 0;
+        dst[t * dstride + 1] = i;
+      }
+    return;
+  }
+  // the highest bit where this row's candidate keys differ
+  uint64_t umin = ~0ull, umax = 0ull;
+  for (int j = 1 + lane; j < i; j += 32) {
+    const uint64_t u = key_bits(j);
+    umin = u < umin ? u : umin;
+    umax = u > umax ? u : umax;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const uint64_t a = __shfl_xor_sync(0xffffffffu, umin, o);
+    const uint64_t c = __shfl_xor_sync(0xffffffffu, umax, o);
+    umin = a < umin ? a : umin;
+    umax = c > umax ? c : umax;
+  }
+  uint64_t prefix, pmask;
+  int rem = need;
+  bool exact = false;
+  if (umin == umax) {  // all candidates tie: lowest indices
+    prefix = umin;
+    pmask = ~0ull;
+  } else {
+    const int top = 63 - __clzll(static_cast<long long>(umin ^ umax));  // highest differing bit
+    pmask = top >= 63 ? 0ull : (~0ull << (top + 1));
+    prefix = umin & pmask;
+    int shift = top - 7 < 0 ? 0 : top - 7;
+    while (true) {
+      for (int bin = lane; bin < 256; bin += 32) hist[bin] = 0;
+      __syncwarp();
+      for (int j = 1 + lane; j < i; j += 32) {
+        const uint64_t u = key_bits(j);
+        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xff], 1);
+      }
+      __syncwarp();
+      // lane l owns bins 255-8l .. 248-8l (descending)
+      int cnt[8];
+      int local = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt[e] = hist[255 - 8 * lane - e];
+        local += cnt[e];
+      }
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int excl = incl - local;
+      const bool owner = excl < rem && rem <= incl;
+      int digit = 0, above = 0, dcount = 0;
+      if (owner) {
+        int run = excl;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (run + cnt[e] >= rem) {
+            digit = 255 - 8 * lane - e;
+            above = run;
+            dcount = cnt[e];
+            break;
+          }
+          run += cnt[e];
+        }
+      }
+      const int src = __ffs(__ballot_sync(0xffffffffu, owner)) - 1;
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      dcount = __shfl_sync(0xffffffffu, dcount, src);
+      __syncwarp();
+      rem -= above;
+      prefix = (prefix & ~(0xffull << shift)) | (static_cast<uint64_t>(digit) << shift);
+      pmask |= 0xffull << shift;
+      if (dcount == rem) {
+        exact = true;
+        break;
+      }
+      if (shift == 0) break;
+      shift = shift - 8 < 0 ? 0 : shift - 8;
+    }
+  }
+  // ascending emission; threshold ties (full key equal) lowest-j first
+  int written = 0, ties = 0;
+  for (int j0 = 0; j0 <= i; j0 += 32) {
+    const int j = j0 + lane;
+    bool sel = false, tie = false;
+    if (j <= i) {
+      if (j == 0 || j == i) {
+        sel = true;
+      } else {
+        const uint64_t um = key_bits(j) & pmask;
+        if (um > prefix) {
+          sel = true;
+        } else if (um == prefix) {
+          if (exact) sel = true;
+          else tie = true;
+        }
+      }
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    if (tie && ties + __popc(tb & lt_mask) < rem) sel = true;
+    ties += __popc(tb);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    const int pos = written + __popc(sb & lt_mask);
+    if (sel && pos < kk)  // never past this row's slot
+      for (int t = 0; t < ndst; ++t) dst[t * dstride + pos] = j;
+    written += __popc(sb);
+  }
+}
+
 struct SelSmem {
   float* s;       // [R][ldS] scaled logits
   float* qs;      // [R][D]
@@ -147,7 +282,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
 
   // ---- phase 2: one warp per row
   int* hist = sm.hist + warp * 256;
-  const unsigned lt_mask = (1u << lane) - 1u;
   for (int r = warp; r < rows; r += kWarps) {
     const int i = i0 + r;
     const float* srow = sm.s + r * ldS;
@@ -174,131 +308,186 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
       for (int j = lane; j <= i; j += 32) mrow[j] = expf(srow[j] - mx) / z * nsrc[j];
     }
 
-    if (i == 0) {
-      if (lane == 0) dst[0] = 0;
-      continue;
-    }
-    const int need = kk - 2;  // picks among j in [1, i-1]
-    if (need >= i - 1) {      // every causal block
-      for (int j = lane; j <= i; j += 32) dst[j] = j;
-      continue;
-    }
-    if (need <= 0) {
-      if (lane == 0) {
-        dst[0] = 0;
-        dst[1] = i;
-      }
-      continue;
-    }
     auto key_bits = [&](int j) -> uint64_t {
       return order_bits(static_cast<double>(srow[j]) + sm.lnn[j]);
     };
-    // the highest bit where this row's candidate keys differ
-    uint64_t umin = ~0ull, umax = 0ull;
-    for (int j = 1 + lane; j < i; j += 32) {
-      const uint64_t u = key_bits(j);
-      umin = u < umin ? u : umin;
-      umax = u > umax ? u : umax;
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const uint64_t a = __shfl_xor_sync(0xffffffffu, umin, o);
-      const uint64_t c = __shfl_xor_sync(0xffffffffu, umax, o);
-      umin = a < umin ? a : umin;
-      umax = c > umax ? c : umax;
-    }
-    uint64_t prefix, pmask;
-    int rem = need;
-    bool exact = false;
-    if (umin == umax) {  // all candidates tie: lowest indices
-      prefix = umin;
-      pmask = ~0ull;
+    select_row(i, kk, key_bits, hist, lane, dst, 0, 1);
+  }
+}
+
+// ---- GQA-group-shared selection: one kept list per (b, kv-head group, query block), chosen by
+// the metric summed over the group's G query heads and written to each of them.
+//   product:  sum_h m_hij = n_j * sum_h p_hij, ranked by ln n_j + logsumexp_h(s_hij - lse_hi),
+//             lse_hi = logsumexp over j <= i of s_hij; the head terms are combined in double by
+//             log-add-exp, so columns whose probabilities underflow float still rank;
+//   additive: sum_h M_hij = sum_h s_hij + G * beta * e_j.
+// One CTA (8 warps) per (b, g, 8 consecutive query blocks); the heads are visited in turn: the
+// scores of one head's 8 rows are computed into shared memory, folded into a double key row per
+// query block, and the next head reuses the space.
+constexpr int kGR = 8;  // query blocks per CTA (one per warp)
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) select_group_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar,
+    const float* __restrict__ vnorm, int B, int Hq, int Hkv, int nb, int ldS, PlanDev plan,
+    int64_t cap, SelMetric metric, int32_t* __restrict__ sel_idx, int32_t* __restrict__ sel_cnt,
+    float* __restrict__ m_out) {
+  constexpr int KLD = D + 4;
+  static_assert(kGR == kWarps, "one query block per warp");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* acc = reinterpret_cast<double*>(smem_raw);  // [kGR][ldS] key under construction
+  double* lnn = acc + kGR * ldS;                       // [ldS] per-column term
+  float* srow_all = reinterpret_cast<float*>(lnn + ldS);  // [kGR][ldS] one head's scores
+  float* qs = srow_all + kGR * ldS;                       // [kGR][D]
+  float* ks = qs + kGR * D;                               // [kTileJ][KLD]
+  int* hist_all = reinterpret_cast<int*>(ks + kTileJ * KLD);  // [kWarps][256]
+
+  const int G = Hq / Hkv;
+  const int BG = B * Hkv;
+  const int ntiles = (nb + kGR - 1) / kGR;
+  const int tile = ntiles - 1 - static_cast<int>(blockIdx.x / BG);  // heaviest tiles first
+  const int bgi = static_cast<int>(blockIdx.x % BG);
+  const int b = bgi / Hkv, g = bgi % Hkv;
+  const int i0 = tile * kGR;
+  const int rows = min(kGR, nb - i0);
+  const int jend = i0 + rows;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int64_t bg = static_cast<int64_t>(b) * Hkv + g;
+  const float* ksrc = kbar + bg * nb * D;
+  const float* nsrc = vnorm + bg * nb;
+  const float scale = rsqrtf(static_cast<float>(D));
+
+  for (int j = t; j < jend; j += kSelThreads) {
+    double c;
+    if (!metric.additive) {
+      c = log(static_cast<double>(nsrc[j]));
+    } else if (metric.beta == 0.f) {
+      c = 0.0;
     } else {
-      const int top = 63 - __clzll(static_cast<long long>(umin ^ umax));  // highest differing bit
-      pmask = top >= 63 ? 0ull : (~0ull << (top + 1));
-      prefix = umin & pmask;
-      int shift = top - 7 < 0 ? 0 : top - 7;
-      while (true) {
-        for (int bin = lane; bin < 256; bin += 32) hist[bin] = 0;
-        __syncwarp();
-        for (int j = 1 + lane; j < i; j += 32) {
-          const uint64_t u = key_bits(j);
-          if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xff], 1);
-        }
-        __syncwarp();
-        // lane l owns bins 255-8l .. 248-8l (descending)
-        int cnt[8];
-        int local = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          cnt[e] = hist[255 - 8 * lane - e];
-          local += cnt[e];
-        }
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int excl = incl - local;
-        const bool owner = excl < rem && rem <= incl;
-        int digit = 0, above = 0, dcount = 0;
-        if (owner) {
-          int run = excl;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (run + cnt[e] >= rem) {
-              digit = 255 - 8 * lane - e;
-              above = run;
-              dcount = cnt[e];
-              break;
-            }
-            run += cnt[e];
-          }
-        }
-        const int src = __ffs(__ballot_sync(0xffffffffu, owner)) - 1;
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above = __shfl_sync(0xffffffffu, above, src);
-        dcount = __shfl_sync(0xffffffffu, dcount, src);
-        __syncwarp();
-        rem -= above;
-        prefix = (prefix & ~(0xffull << shift)) | (static_cast<uint64_t>(digit) << shift);
-        pmask |= 0xffull << shift;
-        if (dcount == rem) {
-          exact = true;
-          break;
-        }
-        if (shift == 0) break;
-        shift = shift - 8 < 0 ? 0 : shift - 8;
-      }
+      double e = 2.0 * log(static_cast<double>(nsrc[j]));
+      if (metric.clamp && e < 0.0) e = 0.0;
+      c = static_cast<double>(metric.beta) * e;
     }
-    // ascending emission; threshold ties (full key equal) lowest-j first
-    int written = 0, ties = 0;
-    for (int j0 = 0; j0 <= i; j0 += 32) {
-      const int j = j0 + lane;
-      bool sel = false, tie = false;
-      if (j <= i) {
-        if (j == 0 || j == i) {
-          sel = true;
-        } else {
-          const uint64_t um = key_bits(j) & pmask;
-          if (um > prefix) {
-            sel = true;
-          } else if (um == prefix) {
-            if (exact) sel = true;
-            else tie = true;
+    lnn[j] = c;
+  }
+
+  const int r = warp;  // this warp's query block in phases 1b and 2
+  const int i = i0 + r;
+  double* arow = acc + r * ldS;
+  float* srow = srow_all + r * ldS;
+  for (int h = 0; h < G; ++h) {
+    const int64_t bh = static_cast<int64_t>(b) * Hq + g * G + h;
+    const float* qsrc = qbar + (bh * nb + i0) * D;
+    __syncthreads();  // the previous head's scores and qs are consumed
+    for (int idx = t; idx < kGR * D / 4; idx += kSelThreads) {
+      const int rr = idx / (D / 4), c4 = idx % (D / 4);
+      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (rr < rows) val = reinterpret_cast<const float4*>(qsrc + rr * D)[c4];
+      reinterpret_cast<float4*>(qs + rr * D)[c4] = val;
+    }
+    // ---- phase 1: s[r][j] of head h for j < jend (warp w computes row w)
+    for (int j0 = 0; j0 < jend; j0 += kTileJ) {
+      __syncthreads();  // previous tile consumed (qs visible on the first pass)
+      for (int idx = t; idx < kTileJ * D / 4; idx += kSelThreads) {
+        const int rr = idx / (D / 4), c4 = idx % (D / 4);
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 + rr < jend) val = reinterpret_cast<const float4*>(ksrc + (j0 + rr) * D)[c4];
+        *reinterpret_cast<float4*>(ks + rr * KLD + c4 * 4) = val;
+      }
+      __syncthreads();
+      float a0 = 0.f, a1 = 0.f;
+      const float* k0 = ks + lane * KLD;
+      const float* k1 = ks + (lane + 32) * KLD;
+      const float* qv = qs + r * D;
+#pragma unroll 4
+      for (int d = 0; d < D; d += 4) {
+        const float4 x0 = *reinterpret_cast<const float4*>(k0 + d);
+        const float4 x1 = *reinterpret_cast<const float4*>(k1 + d);
+        const float4 q4 = *reinterpret_cast<const float4*>(qv + d);
+        a0 = fmaf(q4.x, x0.x, a0);
+        a0 = fmaf(q4.y, x0.y, a0);
+        a0 = fmaf(q4.z, x0.z, a0);
+        a0 = fmaf(q4.w, x0.w, a0);
+        a1 = fmaf(q4.x, x1.x, a1);
+        a1 = fmaf(q4.y, x1.y, a1);
+        a1 = fmaf(q4.z, x1.z, a1);
+        a1 = fmaf(q4.w, x1.w, a1);
+      }
+      if (j0 + lane < jend) srow[j0 + lane] = a0 * scale;
+      if (j0 + lane + 32 < jend) srow[j0 + lane + 32] = a1 * scale;
+    }
+    __syncwarp();
+    // ---- phase 1b: fold head h into the row's key (this warp's row only)
+    if (r < rows) {
+      if (!metric.additive) {
+        float mx = -INFINITY;
+        for (int j = lane; j <= i; j += 32) mx = fmaxf(mx, srow[j]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        double z = 0.0;
+        for (int j = lane; j <= i; j += 32) z += exp(static_cast<double>(srow[j] - mx));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        const double lse = static_cast<double>(mx) + log(z);
+        for (int j = lane; j <= i; j += 32) {
+          const double x = static_cast<double>(srow[j]) - lse;  // log p_hij
+          if (h == 0) {
+            arow[j] = x;
+          } else {  // log-add-exp
+            const double a = arow[j];
+            const double hi = fmax(a, x), lo = fmin(a, x);
+            arow[j] = hi + log1p(exp(lo - hi));
           }
         }
+      } else {
+        for (int j = lane; j <= i; j += 32)
+          arow[j] = (h == 0 ? 0.0 : arow[j]) + static_cast<double>(srow[j]);
       }
-      const unsigned tb = __ballot_sync(0xffffffffu, tie);
-      if (tie && ties + __popc(tb & lt_mask) < rem) sel = true;
-      ties += __popc(tb);
-      const unsigned sb = __ballot_sync(0xffffffffu, sel);
-      const int pos = written + __popc(sb & lt_mask);
-      if (sel && pos < kk) dst[pos] = j;  // never past this row's slot
-      written += __popc(sb);
     }
   }
+  __syncwarp();
+  if (r >= rows) return;  // no __syncthreads below
+  // ---- phase 2: the key, the diagnostic metric, the selection (this warp's row)
+  const double gterm = metric.additive ? static_cast<double>(G) : 1.0;
+  for (int j = lane; j <= i; j += 32) arow[j] += gterm * lnn[j];
+  __syncwarp();
+  const int kk = plan.k[i];
+  const int64_t bh0 = static_cast<int64_t>(b) * Hq + g * G;
+  for (int h = lane; h < G; h += 32) sel_cnt[(bh0 + h) * nb + i] = kk;
+  if (m_out != nullptr) {
+    // sum over the group's heads of the metric: n_j * sum_h p_hij (product) or the summed
+    // additive score; the same row for every head of the group
+    const int64_t tri = static_cast<int64_t>(nb) * (nb + 1) / 2;
+    for (int j = lane; j <= i; j += 32) {
+      const float mv = static_cast<float>(metric.additive ? arow[j] : exp(arow[j]));
+      for (int h = 0; h < G; ++h)
+        m_out[(bh0 + h) * tri + static_cast<int64_t>(i) * (i + 1) / 2 + j] = mv;
+    }
+  }
+  auto key_bits = [&](int j) -> uint64_t { return order_bits(arow[j]); };
+  select_row(i, kk, key_bits, hist_all + warp * 256, lane, sel_idx + bh0 * cap + plan.off[i], cap,
+             G);
+}
+
+template <int D>
+cudaError_t launch_group(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                         int Hkv, int nb, PlanDev plan, int64_t cap, SelMetric metric,
+                         int32_t* sel_idx, int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  const int ldS = (nb + 3) & ~3;
+  const size_t smem = sizeof(double) * (static_cast<size_t>(kGR) * ldS + ldS) +
+                      sizeof(float) * (static_cast<size_t>(kGR) * ldS + kGR * D +
+                                       kTileJ * (D + 4)) +
+                      sizeof(int) * kWarps * 256;
+  auto kern = select_group_kernel<D>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t grid = static_cast<int64_t>(B) * Hkv * ((nb + kGR - 1) / kGR);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kSelThreads, smem, st>>>(qbar, kbar, vnorm, B, Hq, Hkv, nb,
+                                                             ldS, plan, cap, metric, sel_idx,
+                                                             sel_cnt, m_out);
+  return cudaGetLastError();
 }
 
 template <int D, int R>
@@ -342,6 +531,15 @@ cudaError_t launch_select(const float* qbar, const float* kbar, const float* vno
                           SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
                           cudaStream_t st) {
   if (B * Hq == 0 || nb == 0) return cudaSuccess;
+  if (metric.group && Hq != Hkv) {
+    if (D == 128)
+      return launch_group<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                               sel_cnt, m_out, st);
+    if (D == 64)
+      return launch_group<64>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                              sel_cnt, m_out, st);
+    return cudaErrorInvalidValue;
+  }
   if (D == 128)
     return launch_d<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt,
                          m_out, st);

@@ -25,7 +25,11 @@ struct SelMetric {
   bool additive = false;
   float beta = 0.f;
   bool clamp = true;
+  bool group = false;  // one selection per kv-head group (metric summed over its query heads)
 };
+
+// Largest nb the group-shared selection supports (its per-CTA key rows live in shared memory).
+constexpr int kGroupMaxNb = 1024;
 
 // Metric + top-k selection (select.cu).
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,

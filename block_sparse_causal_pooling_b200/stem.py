@@ -33,6 +33,8 @@ STEM_METRIC_PRODUCT = 0
 STEM_METRIC_ADDITIVE = 1
 STEM_VSUM_MEAN = 0
 STEM_VSUM_MAX = 1
+STEM_SHARE_HEAD = 0
+STEM_SHARE_GROUP = 1
 
 
 class StemError(RuntimeError):
@@ -46,21 +48,24 @@ class stem_method_t(ctypes.Structure):
         ("schedule", ctypes.c_int32), ("rho_min", ctypes.c_float), ("tau", ctypes.c_float),
         ("k_start", ctypes.c_float), ("mu", ctypes.c_float), ("k_min", ctypes.c_int32),
         ("metric", ctypes.c_int32), ("beta", ctypes.c_float), ("clamp", ctypes.c_int32),
-        ("vsum", ctypes.c_int32),
+        ("vsum", ctypes.c_int32), ("share", ctypes.c_int32),
     ]
 
 
 def make_method(schedule: str = "exp", rho_min: float = 1.0, tau: float = 1.0,
                 k_start: float = 1.0, mu: float = 1.0, k_min: int = 1, metric: str = "product",
-                beta: float = 0.0, clamp: bool = True, vsum: str = "mean") -> stem_method_t:
+                beta: float = 0.0, clamp: bool = True, vsum: str = "mean",
+                share: str = "head") -> stem_method_t:
     """Method parameters (stem_method_t): schedule "exp" (rho_min, tau) or "linear" (k_start,
-    mu); metric "product" or "additive" (beta, clamp); vsum "mean" or "max"."""
+    mu); metric "product" or "additive" (beta, clamp); vsum "mean" or "max"; share "head" or
+    "group" (one selection per kv-head group)."""
     m = stem_method_t()
     m.schedule = {"exp": STEM_SCHED_EXP, "linear": STEM_SCHED_LINEAR}[schedule]
     m.rho_min, m.tau, m.k_start, m.mu, m.k_min = rho_min, tau, k_start, mu, k_min
     m.metric = {"product": STEM_METRIC_PRODUCT, "additive": STEM_METRIC_ADDITIVE}[metric]
     m.beta, m.clamp = beta, int(bool(clamp))
     m.vsum = {"mean": STEM_VSUM_MEAN, "max": STEM_VSUM_MAX}[vsum]
+    m.share = {"head": STEM_SHARE_HEAD, "group": STEM_SHARE_GROUP}[share]
     return m
 
 

@@ -72,6 +72,8 @@ extern "C" {
 #define STEM_METRIC_ADDITIVE 1 /* M_ij = s_ij + beta * max(0, log n_j^2) */
 #define STEM_VSUM_MEAN 0       /* n_j = mean of the block's V-row L2 norms (the default) */
 #define STEM_VSUM_MAX 1        /* n_j = largest V-row L2 norm of the block */
+#define STEM_SHARE_HEAD 0      /* one selection per query head (the default) */
+#define STEM_SHARE_GROUP 1     /* one selection per kv-head group, shared by its query heads */
 
 /*
  * Method parameters: budget schedule, block metric and V summary.
@@ -86,6 +88,11 @@ extern "C" {
  *                         1; beta >= 0 and finite (beta == 0: e_j is not evaluated, so
  *                         n_j = 0 is allowed); clamp in {0, 1}.
  *   vsum: STEM_VSUM_MEAN or STEM_VSUM_MAX (pooling of ||V row|| into n_j).
+ *   share: STEM_SHARE_HEAD, or STEM_SHARE_GROUP: the G = Hq/Hkv query heads of a kv-head group
+ *          keep one list, chosen by the metric summed over them (product: n_j * sum_h p_hij,
+ *          ranked in log space; additive: sum_h s_hij + G * beta * e_j) and written to each
+ *          head's CSR row. The pages are silent on GQA; this is an alternative reading. With
+ *          share = GROUP and G > 1, nb beyond 1024 returns STEM_ERR_UNSUPPORTED.
  * Fields the chosen schedule and metric do not use are ignored.
  */
 typedef struct stem_method {
@@ -99,6 +106,7 @@ typedef struct stem_method {
   float beta;
   int32_t clamp;
   int32_t vsum;
+  int32_t share;
 } stem_method_t;
 
 /* Largest number of blocks per sequence (the selection kernel keeps one score row per

@@ -103,11 +103,16 @@ BAD_BETA = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2, metric="additive
 BAD_VSUM = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2)
 BAD_VSUM.vsum = 7
 GOOD = S.make_method("linear", k_start=8.0, mu=0.7, k_min=2, metric="additive", beta=0.2)
+BAD_SHARE = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2)
+BAD_SHARE.share = 3
+GROUP = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2, share="group")
 M = lambda m: ctypes.byref(m)  # noqa: E731
 res.update({
     "method_bad_mu": ex(method=ctypes.pointer(BAD_MU)),
     "method_bad_beta": ex(method=ctypes.pointer(BAD_BETA)),
     "method_bad_vsum": ex(method=ctypes.pointer(BAD_VSUM)),
+    "method_bad_share": ex(method=ctypes.pointer(BAD_SHARE)),
+    "group_nb_too_large": ex(S=1025 * 128, method=ctypes.pointer(GROUP)),
     "method_overrides_bad_rho": ex(rho_min=-1.0, method=ctypes.pointer(BAD_MU)),
     "host_method_bad": L.stem_prefill_host(ctypes.byref(base(method=ctypes.pointer(BAD_BETA)))),
     "pool_m_bad_vsum": L.stem_pool_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, M(BAD_VSUM),

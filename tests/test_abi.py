@@ -139,6 +139,7 @@ def test_argument_validation_rejects_before_any_device_work():
         "nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "select_nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "static_nb_too_large": S.STEM_ERR_UNSUPPORTED,
+        "group_nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "empty_B": S.STEM_OK,
         "empty_S": S.STEM_OK,
     })

@@ -30,6 +30,10 @@ METHODS = {
     "routing-only": dict(schedule="exp", rho_min=0.2, tau=4.0, k_min=3, metric="additive",
                          beta=0.0),
     "product-vmax": dict(schedule="exp", rho_min=0.2, tau=4.0, k_min=3, vsum="max"),
+    # GQA-group-shared selection (one list per kv-head group)
+    "group-product": dict(schedule="exp", rho_min=0.2, tau=4.0, k_min=3, share="group"),
+    "group-pages": dict(schedule="linear", k_start=12.0, mu=0.7, k_min=4, metric="additive",
+                        beta=0.2, clamp=True, vsum="max", share="group"),
 }
 
 WORKLOADS = {
@@ -41,7 +45,8 @@ WORKLOADS = {
                                        block=128),
 }
 
-CASES = [(m, "llama-4k") for m in METHODS] + [("pages", w) for w in WORKLOADS if w != "llama-4k"]
+CASES = ([(m, "llama-4k") for m in METHODS] +
+         [(m, w) for m in ("pages", "group-product") for w in WORKLOADS if w != "llama-4k"])
 
 
 def _method(name):
@@ -53,7 +58,8 @@ def _oracle_kwargs(name):
     return dict(rho_min=d.get("rho_min", 1.0), tau=d.get("tau", 1.0), k_min=d["k_min"],
                 schedule=d.get("schedule", "exp"), k_start=d.get("k_start", 0.0),
                 mu=d.get("mu", 1.0), metric_form=d.get("metric", "product"),
-                beta=d.get("beta", 0.0), clamp=d.get("clamp", True), vsum=d.get("vsum", "mean"))
+                beta=d.get("beta", 0.0), clamp=d.get("clamp", True), vsum=d.get("vsum", "mean"),
+                share=d.get("share", "head"))
 
 
 def _oracle_budget(name, nb):
@@ -64,10 +70,22 @@ def _oracle_budget(name, nb):
 
 
 def _oracle_metric(name, qbar, kbar, vnorm):
+    """Per-head metric [B, Hq, T]; for group sharing the group metric replicated per head."""
     d = _oracle_kwargs(name)
     if d["metric_form"] == "additive":
-        return oracle.metric_additive(qbar, kbar, vnorm, d["beta"], d["clamp"])
-    return oracle.metric(qbar, kbar, vnorm)
+        m = oracle.metric_additive(qbar, kbar, vnorm, d["beta"], d["clamp"])
+    else:
+        m = oracle.metric(qbar, kbar, vnorm)
+    if d["share"] == "group":
+        G = qbar.shape[1] // kbar.shape[1]
+        m = np.repeat(oracle.metric_group(m, G), G, axis=1)
+    return m
+
+
+def _oracle_select(name, m, kk, off, G):
+    if _oracle_kwargs(name)["share"] == "group":
+        return oracle.select_group(m[:, ::G], kk, off, G)
+    return oracle.select(m, kk, off)
 
 
 def inputs(w):
@@ -98,7 +116,7 @@ def test_select_from_oracle_pooling(mname, wname):
     q32, k32, n32 = (torch.from_numpy(x).float() for x in (rq, rk, rn))
     m = _oracle_metric(mname, q32.double().numpy(), k32.double().numpy(), n32.double().numpy())
     kk, off = _oracle_budget(mname, w.nb)
-    ref_idx, ref_cnt = oracle.select(m, kk, off)
+    ref_idx, ref_cnt = _oracle_select(mname, m, kk, off, w.Hq // w.Hkv)
     sel_idx, sel_cnt, m_gpu = S.stem_select(q32.to(DEV), k32.to(DEV), n32.to(DEV), 0.0, 0.0, 0,
                                             with_metric=True, method=_method(mname))
     torch.cuda.synchronize()
@@ -112,6 +130,11 @@ def test_select_from_oracle_pooling(mname, wname):
         np.testing.assert_allclose(mg, m, rtol=0, atol=2e-5 * max(1.0, float(np.abs(m).max())))
     else:
         np.testing.assert_allclose(mg, m, rtol=2e-5, atol=1e-30)
+    if _oracle_kwargs(mname)["share"] == "group":  # every head of a group keeps the same list
+        G = w.Hq // w.Hkv
+        si = sel_idx.cpu().numpy()[:, :, :int(off[-1])]
+        for h in range(w.Hq):
+            assert np.array_equal(si[:, h], si[:, (h // G) * G])
 
 
 @pytest.mark.parametrize("mname,wname", CASES)
