@@ -240,6 +240,9 @@ stem_method_t args_method(const stem_args_t* a) {
   return a->method ? *a->method : default_method(a->rho_min, a->tau, a->k_min);
 }
 
+int enqueue_kernels(const stem_args_t* a, const stem_method_t& m, int nb, int64_t cap,
+                    PlanDev pd, cudaStream_t st);
+
 int run_prefill(const stem_args_t* a, cudaStream_t st) {
   if (a == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(a->B, a->Hq, a->Hkv, a->S, a->D, a->block, a->dtype);
@@ -267,6 +270,16 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   PlanDev pd;
   rc = upload_plan(plan, ws, L, st, &pd);
   if (rc != STEM_OK) return rc;
+  return enqueue_kernels(a, m, nb, plan->cap, pd, st);
+}
+
+// The three stages of a validated call whose plan is already on the device (pd) and whose status
+// word, if any, is already cleared: kernels (and the optional timing events) only, no copies.
+int enqueue_kernels(const stem_args_t* a, const stem_method_t& m, int nb, int64_t cap,
+                    PlanDev pd, cudaStream_t st) {
+  int rc = STEM_OK;
+  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D);
+  auto* ws = static_cast<unsigned char*>(a->workspace);
   float* qbar = reinterpret_cast<float*>(ws + L.qbar);
   float* kbar = reinterpret_cast<float*>(ws + L.kbar);
   float* vnorm = reinterpret_cast<float*>(ws + L.vnorm);
@@ -279,20 +292,20 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
                             a->block, m.vsum == STEM_VSUM_MAX, qbar, kbar, vnorm, st));
   if (rc != STEM_OK) return rc;
   if ((rc = mark(1)) != STEM_OK) return rc;
-  rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, plan->cap,
+  rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, cap,
                               sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st));
   if (rc != STEM_OK) return rc;
   if ((rc = mark(2)) != STEM_OK) return rc;
   if (a->dtype == STEM_BF16) {
     rc = cuda_err(launch_attn_bf16(a->q, a->k, a->v, a->B, a->Hq, a->Hkv, a->S, a->D, a->block,
-                                   pd, plan->cap, a->sel_idx, a->sel_cnt,
+                                   pd, cap, a->sel_idx, a->sel_cnt,
                                    reinterpret_cast<uint32_t*>(ws + L.sched), a->out, a->status,
                                    st));
   } else {
     rc = cuda_err(launch_attn_f32(static_cast<const float*>(a->q),
                                   static_cast<const float*>(a->k),
                                   static_cast<const float*>(a->v), a->B, a->Hq, a->Hkv, a->S,
-                                  a->D, a->block, pd, plan->cap, a->sel_idx, a->sel_cnt,
+                                  a->D, a->block, pd, cap, a->sel_idx, a->sel_cnt,
                                   static_cast<float*>(a->out), st));
   }
   if (rc != STEM_OK) return rc;
@@ -435,6 +448,11 @@ int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int
   return run_prefill(&a, nullptr);
 }
 
+// Host buffers: the problem splits into B*Hkv independent chunks (batch b, kv-head group g: the
+// group's G query heads, its K and V head, their outputs and CSR rows, each contiguous). Chunk
+// c's inputs go up on one stream, its kernels run on a second once they have arrived, and its
+// results come down on a third once its kernels are done, so the copies of one chunk overlap
+// the kernels of the others and the two PCIe directions overlap each other.
 int stem_prefill_host(const stem_args_t* h) {
   if (h == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(h->B, h->Hq, h->Hkv, h->S, h->D, h->block, h->dtype);
@@ -445,55 +463,104 @@ int stem_prefill_host(const stem_args_t* h) {
   if (rc != STEM_OK) return rc;
   if (is_empty(h->B, h->S)) return STEM_OK;
   if (!h->q || !h->k || !h->v || !h->out || !h->sel_idx || !h->sel_cnt) return STEM_ERR_ARG;
+  const int G = h->Hq / h->Hkv;
+  const int nc = h->B * h->Hkv;  // chunks
   const size_t es = elem_size(h->dtype);
-  const size_t qb = es * static_cast<size_t>(h->B) * h->Hq * h->S * h->D;
-  const size_t kvb = es * static_cast<size_t>(h->B) * h->Hkv * h->S * h->D;
   const int64_t cap = capacity(nb, m);
-  const size_t sib = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * cap;
-  const size_t scb = sizeof(int32_t) * static_cast<size_t>(h->B) * h->Hq * nb;
-  const Layout L = layout(h->B, h->Hq, h->Hkv, nb, h->D);
-  // device arena: workspace | q | k | v | out | sel_idx | sel_cnt
-  const size_t o_q = L.total, o_k = o_q + align_up(qb), o_v = o_k + align_up(kvb),
-               o_out = o_v + align_up(kvb), o_si = o_out + align_up(qb),
-               o_sc = o_si + align_up(sib), total = o_sc + align_up(scb);
+  const size_t qcb = es * static_cast<size_t>(G) * h->S * h->D;  // per chunk
+  const size_t kvcb = es * static_cast<size_t>(h->S) * h->D;
+  const size_t sicb = sizeof(int32_t) * static_cast<size_t>(G) * cap;
+  const size_t sccb = sizeof(int32_t) * static_cast<size_t>(G) * nb;
+  const Layout Lc = layout(1, G, 1, nb, h->D);  // one chunk's workspace
+  const Plan* plan = get_plan(nb, m);
+  if (plan == nullptr) return STEM_ERR_CUDA;
+  // device arena: chunk status words | the plan | chunk workspaces | q | k | v | out | sel_idx |
+  // sel_cnt. The plan and the cleared status words go up first on the input stream: a copy
+  // issued on the compute stream would wait in the copy engine behind every chunk's inputs.
+  const size_t o_plan = align_up(sizeof(int32_t) * nc);
+  const size_t o_ws = o_plan + plan_bytes(nb);
+  const size_t wsb = align_up(Lc.total);
+  const size_t o_q = o_ws + wsb * nc, o_k = o_q + align_up(qcb * nc),
+               o_v = o_k + align_up(kvcb * nc), o_out = o_v + align_up(kvcb * nc),
+               o_si = o_out + align_up(qcb * nc), o_sc = o_si + align_up(sicb * nc),
+               total = o_sc + align_up(sccb * nc);
   static std::mutex host_mu;  // host-buffer calls share one arena: one at a time
   std::lock_guard<std::mutex> lock(host_mu);
   void* arena = nullptr;
   rc = get_scratch(total, &arena, 1);
   if (rc != STEM_OK) return rc;
   auto* base = static_cast<unsigned char*>(arena);
-  cudaStream_t st = nullptr;
-  cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
-  if (e != cudaSuccess) return cuda_err(e);
-  stem_args_t d = *h;
-  d.q = base + o_q;
-  d.k = base + o_k;
-  d.v = base + o_v;
-  d.out = base + o_out;
-  d.sel_idx = reinterpret_cast<int32_t*>(base + o_si);
-  d.sel_cnt = reinterpret_cast<int32_t*>(base + o_sc);
-  d.workspace = base;
-  d.workspace_bytes = L.total;
-  d.status = reinterpret_cast<int32_t*>(base + L.status);
-  d.events = nullptr;
-  int32_t status = 0;
+  cudaStream_t sin = nullptr, srun = nullptr, sout = nullptr;
+  std::vector<cudaEvent_t> ev(2 * static_cast<size_t>(nc), nullptr);
+  cudaError_t e = cudaSuccess;
+  auto cleanup = [&]() {
+    for (cudaStream_t s : {sin, srun, sout})
+      if (s) cudaStreamSynchronize(s);
+    for (cudaEvent_t x : ev)
+      if (x) cudaEventDestroy(x);
+    for (cudaStream_t s : {sin, srun, sout})
+      if (s) cudaStreamDestroy(s);
+  };
   do {
-    if ((e = cudaMemcpyAsync(const_cast<void*>(d.q), h->q, qb, cudaMemcpyHostToDevice, st))) break;
-    if ((e = cudaMemcpyAsync(const_cast<void*>(d.k), h->k, kvb, cudaMemcpyHostToDevice, st))) break;
-    if ((e = cudaMemcpyAsync(const_cast<void*>(d.v), h->v, kvb, cudaMemcpyHostToDevice, st))) break;
-    rc = run_prefill(&d, st);
-    if (rc != STEM_OK) break;
-    if ((e = cudaMemcpyAsync(h->out, d.out, qb, cudaMemcpyDeviceToHost, st))) break;
-    if ((e = cudaMemcpyAsync(h->sel_idx, d.sel_idx, sib, cudaMemcpyDeviceToHost, st))) break;
-    if ((e = cudaMemcpyAsync(h->sel_cnt, d.sel_cnt, scb, cudaMemcpyDeviceToHost, st))) break;
-    if ((e = cudaMemcpyAsync(&status, d.status, sizeof status, cudaMemcpyDeviceToHost, st))) break;
-    e = cudaStreamSynchronize(st);
+    if ((e = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking))) break;
+    if ((e = cudaStreamCreateWithFlags(&srun, cudaStreamNonBlocking))) break;
+    if ((e = cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking))) break;
+    for (auto& x : ev)
+      if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming))) break;
+    if (e) break;
+    if ((e = cudaMemsetAsync(base, 0, sizeof(int32_t) * nc, sin))) break;
+    if ((e = cudaMemcpyAsync(base + o_plan, plan->host, plan->bytes, cudaMemcpyHostToDevice, sin)))
+      break;
+    PlanDev pd;
+    pd.k = reinterpret_cast<const int32_t*>(base + o_plan);
+    pd.off = pd.k + nb;
+    pd.order = pd.k + 2 * nb + 1;
+    for (int c = 0; c < nc && rc == STEM_OK && e == cudaSuccess; ++c) {
+      const auto* hq = static_cast<const unsigned char*>(h->q) + qcb * c;
+      const auto* hk = static_cast<const unsigned char*>(h->k) + kvcb * c;
+      const auto* hv = static_cast<const unsigned char*>(h->v) + kvcb * c;
+      stem_args_t d = *h;
+      d.B = 1;
+      d.Hq = G;
+      d.Hkv = 1;
+      d.q = base + o_q + qcb * c;
+      d.k = base + o_k + kvcb * c;
+      d.v = base + o_v + kvcb * c;
+      d.out = base + o_out + qcb * c;
+      d.sel_idx = reinterpret_cast<int32_t*>(base + o_si + sicb * c);
+      d.sel_cnt = reinterpret_cast<int32_t*>(base + o_sc + sccb * c);
+      d.workspace = base + o_ws + wsb * c;
+      d.workspace_bytes = Lc.total;
+      d.status = reinterpret_cast<int32_t*>(base) + c;
+      d.events = nullptr;
+      if ((e = cudaMemcpyAsync(const_cast<void*>(d.q), hq, qcb, cudaMemcpyHostToDevice, sin))) break;
+      if ((e = cudaMemcpyAsync(const_cast<void*>(d.k), hk, kvcb, cudaMemcpyHostToDevice, sin))) break;
+      if ((e = cudaMemcpyAsync(const_cast<void*>(d.v), hv, kvcb, cudaMemcpyHostToDevice, sin))) break;
+      if ((e = cudaEventRecord(ev[2 * c], sin))) break;
+      if ((e = cudaStreamWaitEvent(srun, ev[2 * c], 0))) break;
+      if ((rc = enqueue_kernels(&d, m, nb, plan->cap, pd, srun)) != STEM_OK) break;
+      if ((e = cudaEventRecord(ev[2 * c + 1], srun))) break;
+      if ((e = cudaStreamWaitEvent(sout, ev[2 * c + 1], 0))) break;
+      if ((e = cudaMemcpyAsync(static_cast<unsigned char*>(h->out) + qcb * c, d.out, qcb,
+                               cudaMemcpyDeviceToHost, sout)))
+        break;
+      if ((e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(h->sel_idx) + sicb * c,
+                               d.sel_idx, sicb, cudaMemcpyDeviceToHost, sout)))
+        break;
+      if ((e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(h->sel_cnt) + sccb * c,
+                               d.sel_cnt, sccb, cudaMemcpyDeviceToHost, sout)))
+        break;
+    }
   } while (false);
-  cudaStreamSynchronize(st);
-  cudaStreamDestroy(st);
+  cleanup();
   if (rc != STEM_OK) return rc;
   if (e != cudaSuccess) return cuda_err(e);
-  return status < 0 ? status : STEM_OK;
+  std::vector<int32_t> status(nc, 0);
+  e = cudaMemcpy(status.data(), base, sizeof(int32_t) * nc, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(e);
+  for (int32_t x : status)
+    if (x < 0) return x;
+  return STEM_OK;
 }
 
 int stem_pool_m(const void* q, const void* k, const void* v, int dtype, int B, int Hq, int Hkv,
