@@ -44,8 +44,8 @@ KERNELS_PER_STEP = 4
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616352768 + 1023481088,
-                "sources_sha256": "88d840a84ec15a20507ba01f9c2d0782060b8b67d0d8c7a2163b1870f371d0c9"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615536128 + 1023997440,
+                "sources_sha256": "01d0c89698de2d0b5e9e849b14c3e348330e4c12402f65143710731da57d4678"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

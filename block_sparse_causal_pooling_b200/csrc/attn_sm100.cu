@@ -43,12 +43,17 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "stem.h"
 #include "stem_internal.h"
 
 namespace stem {
+
+// Test switch (stem_test_withhold_q): when set, the producer of every CTA skips its first Q
+// tile, so the MMA thread's bounded wait for it expires and the whole CTA takes the abort path.
+std::atomic<int> g_withhold_q{0};
 
 cudaError_t launch_attn_bf16_mma(const void* q, const void* k, const void* v, int B, int Hq,
                                  int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
@@ -398,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, int Hq, int Hkv, int S, int nb,
                       int64_t items, PlanDev plan, int64_t cap,
                       const uint32_t* __restrict__ sched, __nv_bfloat16* __restrict__ out,
-                      int32_t* status) {
+                      int32_t* status, int withhold_q) {
   using C = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -467,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       auto load_q = [&](const Step& st, int tile) -> bool {
+        if (withhold_q && tile == 0 && q_loads[0] == 0) return true;  // test switch: never sent
         const int64_t r = q_loads[tile];
         if (!wait_bar(&bars->q_empty[tile], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
           return false;
@@ -875,7 +881,7 @@ cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, Hq, Hkv, S, nb, items,
                                                            plan, cap, sched,
                                                            static_cast<__nv_bfloat16*>(out),
-                                                           status);
+                                                           status, g_withhold_q.load());
   return cudaGetLastError();
 }
 
@@ -893,3 +899,5 @@ cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B,
 }
 
 }  // namespace stem
+
+extern "C" int stem_test_withhold_q(int on) { return stem::g_withhold_q.exchange(on ? 1 : 0); }

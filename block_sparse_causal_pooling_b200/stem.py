@@ -109,6 +109,7 @@ def _load() -> ctypes.CDLL:
         "stem_pool_m": (I, [P, P, P, I, I, I, I, I, I, I, M, P, P, P, P]),
         "stem_select_m": (I, [P, P, P, I, I, I, I, I, M, P, P, P, P, Z, P]),
         "stem_sparse_attn_m": (I, [P, P, P, I, I, I, I, I, I, I, M, P, P, P, P, Z, P, P]),
+        "stem_test_withhold_q": (I, [I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -123,7 +124,8 @@ _lib = _load()
 EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget",
             "stem_sel_capacity", "stem_workspace_size", "stem_strerror", "stem_pool",
             "stem_select", "stem_sparse_attn", "stem_budget_m", "stem_sel_capacity_m",
-            "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_select_static")
+            "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_select_static",
+            "stem_test_withhold_q")
 
 
 def lib() -> ctypes.CDLL:

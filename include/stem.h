@@ -271,6 +271,17 @@ int stem_select_static(const float* qbar, const float* kbar, const float* vnorm,
                        int Hkv, int nb, int D, float rho_min, float tau, int k_min,
                        int32_t* sel_idx, int32_t* sel_cnt, void* stream);
 
+/*
+ * stem_test_withhold_q: TEST ONLY. With on != 0, later launches of the bfloat16 block-128
+ * attention kernel (stem_prefill*, stem_sparse_attn*) skip each CTA's first Q tile, so the
+ * kernel's bounded wait for it expires (after about 2 s): the kernel then records
+ * STEM_ERR_TIMEOUT in the status word, every role leaves its loop, issued copies and products
+ * are drained, TMEM is freed and the kernel returns, leaving the CUDA context usable. It exists
+ * to exercise that path; the outputs of such a call are undefined. Process-wide; returns the
+ * previous setting (0 or 1). The paper has no counterpart.
+ */
+int stem_test_withhold_q(int on);
+
 #ifdef __cplusplus
 }
 #endif

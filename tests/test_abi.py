@@ -100,6 +100,17 @@ def test_method_validation(bad):
     assert S.lib().stem_budget_m(64, None, None, None) == S.STEM_ERR_ARG
 
 
+def test_withhold_switch_is_host_state_only():
+    """The test switch for the timeout path is a host-side flag: it toggles, reports the previous
+    value and is left off."""
+    L = S.lib()
+    assert L.stem_test_withhold_q(0) in (0, 1)
+    assert L.stem_test_withhold_q(1) == 0
+    assert L.stem_test_withhold_q(7) == 1
+    assert L.stem_test_withhold_q(0) == 1
+    assert L.stem_test_withhold_q(0) == 0
+
+
 def test_workspace_size_layout():
     B, Hq, Hkv, Sq, D, block = 1, 32, 8, 131072, 128, 128
     nb = Sq // block

@@ -1,0 +1,51 @@
+"""The attention kernel's bounded waits, on a B200: a wait that runs out (a Q tile the producer
+never sends, via the library's test switch) ends the kernel with STEM_ERR_TIMEOUT in the status
+word instead of hanging it, and the CUDA context stays usable: the next call is exact again.
+"""
+
+import time
+
+import pytest
+import torch
+
+import oracle
+from block_sparse_causal_pooling_b200 import stem as S
+from block_sparse_causal_pooling_b200 import workloads as wl
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def test_expired_wait_reports_timeout_and_the_context_survives():
+    w = wl.LLAMA_32K.replace(name="timeout-4k", Hq=8, Hkv=2, S=4096)
+    q, k, v = wl.make_inputs(w, "cpu")
+    dq, dk, dv = (t.to(DEV) for t in (q, k, v))
+    status = torch.full((1,), 7, dtype=torch.int32, device=DEV)
+    lib = S.lib()
+    assert lib.stem_test_withhold_q(1) == 0
+    try:
+        t0 = time.perf_counter()
+        S.stem_prefill_ex(dq, dk, dv, w.block, w.rho_min, w.tau, w.k_min, status=status)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        lib.stem_test_withhold_q(0)
+    assert int(status.item()) == S.STEM_ERR_TIMEOUT
+    assert elapsed < 30.0, elapsed  # one bounded wait (2 s) plus the bounded drains
+    # the context is usable and the next call is exact
+    status.fill_(7)
+    out, sel_idx, sel_cnt = S.stem_prefill_ex(dq, dk, dv, w.block, w.rho_min, w.tau, w.k_min,
+                                              status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle.prefill(q, k, v, w.block, w.rho_min, w.tau, w.k_min)
+    res = parity.compare_selection(sel_idx, sel_cnt, ref["sel_idx"], ref["sel_cnt"], ref["m"],
+                                   ref["k"], ref["off"])
+    assert not res["violations"], res["violations"][:5]
+    swapped = set(res["rows_bad"])
+    rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
+    keep = [t for t, r in enumerate(rows) if r not in swapped]
+    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
+    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, "after timeout")
