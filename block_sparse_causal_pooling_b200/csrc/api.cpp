@@ -670,4 +670,108 @@ int stem_sparse_attn(const void* q, const void* k, const void* v, int dtype, int
                             workspace, workspace_bytes, status, stream);
 }
 
+// ------------------------------------------------------------------ variable-length batches
+
+static int check_cu(int nseq, const int32_t* cu) {
+  if (nseq < 0 || cu == nullptr || cu[0] != 0) return STEM_ERR_ARG;
+  for (int s = 0; s < nseq; ++s)
+    if (cu[s + 1] < cu[s]) return STEM_ERR_ARG;
+  return STEM_OK;
+}
+
+int64_t stem_varlen_sel_capacity(int nseq, const int32_t* cu, int block, const stem_method_t* m) {
+  if (m == nullptr || (block != 64 && block != 128)) return STEM_ERR_ARG;
+  if (check_cu(nseq, cu) != STEM_OK) return STEM_ERR_ARG;
+  int64_t total = 0;
+  for (int s = 0; s < nseq; ++s) {
+    const int nb = nblocks(cu[s + 1] - cu[s], block);
+    if (!method_ok(nb, *m)) return STEM_ERR_ARG;
+    total += capacity(nb, *m);
+  }
+  return total;
+}
+
+size_t stem_varlen_workspace_size(int nseq, const int32_t* cu, int Hq, int Hkv, int D,
+                                  int block) {
+  if (check_cu(nseq, cu) != STEM_OK) return 0;
+  size_t most = 0;
+  for (int s = 0; s < nseq; ++s) {
+    const int S = cu[s + 1] - cu[s];
+    if (S == 0) continue;
+    const size_t n = stem_workspace_size(1, Hq, Hkv, S, D, block);
+    if (n == 0) return 0;
+    most = std::max(most, n);
+  }
+  return most;
+}
+
+int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream) {
+  if (a == nullptr || a->method == nullptr) return STEM_ERR_ARG;
+  int rc = check_cu(a->nseq, a->cu_seqlens);
+  if (rc != STEM_OK) return rc;
+  const stem_method_t& m = *a->method;
+  const int32_t* cu = a->cu_seqlens;
+  // validate every sequence before anything is enqueued
+  size_t need = 0;
+  for (int s = 0; s < a->nseq; ++s) {
+    const int S = cu[s + 1] - cu[s];
+    rc = check_shape(1, a->Hq, a->Hkv, S, a->D, a->block, a->dtype);
+    if (rc != STEM_OK) return rc;
+    rc = check_params(nblocks(S, a->block), m);
+    if (rc != STEM_OK) return rc;
+    if (S > 0) need = std::max(need, layout(1, a->Hq, a->Hkv, nblocks(S, a->block), a->D).total);
+  }
+  if (need == 0) return STEM_OK;  // no tokens
+  if (!a->q || !a->k || !a->v || !a->out || !a->sel_idx || !a->sel_cnt) return STEM_ERR_ARG;
+  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->out, 16) ||
+      !aligned(a->sel_idx, 4) || !aligned(a->sel_cnt, 4) || !aligned(a->status, 4))
+    return STEM_ERR_ARG;
+  if (a->workspace == nullptr || !aligned(a->workspace, kAlign) || a->workspace_bytes < need)
+    return STEM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a->status) {
+    rc = cuda_err(cudaMemsetAsync(a->status, 0, sizeof(int32_t), st));
+    if (rc != STEM_OK) return rc;
+  }
+  const size_t es = elem_size(a->dtype);
+  int64_t capo = 0, nbo = 0;  // CSR and count offsets of the sequences before s
+  for (int s = 0; s < a->nseq; ++s) {
+    const int S = cu[s + 1] - cu[s];
+    if (S == 0) continue;
+    const int nb = nblocks(S, a->block);
+    const Plan* plan = get_plan(nb, m);
+    if (plan == nullptr) return STEM_ERR_CUDA;
+    const int64_t tok = cu[s];
+    stem_args_t d;
+    std::memset(&d, 0, sizeof d);
+    d.q = static_cast<const unsigned char*>(a->q) + es * a->Hq * a->D * tok;
+    d.k = static_cast<const unsigned char*>(a->k) + es * a->Hkv * a->D * tok;
+    d.v = static_cast<const unsigned char*>(a->v) + es * a->Hkv * a->D * tok;
+    d.out = static_cast<unsigned char*>(a->out) + es * a->Hq * a->D * tok;
+    d.sel_idx = a->sel_idx + static_cast<int64_t>(a->Hq) * capo;
+    d.sel_cnt = a->sel_cnt + static_cast<int64_t>(a->Hq) * nbo;
+    d.B = 1;
+    d.Hq = a->Hq;
+    d.Hkv = a->Hkv;
+    d.S = S;
+    d.D = a->D;
+    d.block = a->block;
+    d.dtype = a->dtype;
+    d.workspace = a->workspace;
+    d.workspace_bytes = a->workspace_bytes;
+    d.status = a->status;
+    d.method = a->method;
+    // the plan goes into the shared workspace in stream order, after the previous sequence's
+    // kernels have read theirs
+    PlanDev pd;
+    rc = upload_plan(plan, a->workspace, layout(1, a->Hq, a->Hkv, nb, a->D), st, &pd);
+    if (rc != STEM_OK) return rc;
+    rc = enqueue_kernels(&d, m, nb, plan->cap, pd, st);
+    if (rc != STEM_OK) return rc;
+    capo += plan->cap;
+    nbo += nb;
+  }
+  return STEM_OK;
+}
+
 }  // extern "C"

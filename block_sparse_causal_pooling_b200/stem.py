@@ -84,6 +84,19 @@ class stem_args_t(ctypes.Structure):
     ]
 
 
+class stem_varlen_args_t(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("nseq", ctypes.c_int32), ("cu_seqlens", ctypes.POINTER(ctypes.c_int32)),
+        ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+        ("block", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("method", ctypes.POINTER(stem_method_t)),
+        ("out", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("status", ctypes.c_void_p),
+    ]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -110,6 +123,9 @@ def _load() -> ctypes.CDLL:
         "stem_select_m": (I, [P, P, P, I, I, I, I, I, M, P, P, P, P, Z, P]),
         "stem_sparse_attn_m": (I, [P, P, P, I, I, I, I, I, I, I, M, P, P, P, P, Z, P, P]),
         "stem_test_withhold_q": (I, [I]),
+        "stem_prefill_varlen": (I, [ctypes.POINTER(stem_varlen_args_t), P]),
+        "stem_varlen_workspace_size": (Z, [I, ctypes.POINTER(ctypes.c_int32), I, I, I, I]),
+        "stem_varlen_sel_capacity": (ctypes.c_int64, [I, ctypes.POINTER(ctypes.c_int32), I, M]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -124,7 +140,8 @@ _lib = _load()
 EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget",
             "stem_sel_capacity", "stem_workspace_size", "stem_strerror", "stem_pool",
             "stem_select", "stem_sparse_attn", "stem_budget_m", "stem_sel_capacity_m",
-            "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_select_static",
+            "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_prefill_varlen",
+            "stem_varlen_workspace_size", "stem_varlen_sel_capacity", "stem_select_static",
             "stem_test_withhold_q")
 
 
@@ -361,3 +378,53 @@ def stem_select_static(qbar, kbar, vnorm, rho_min, tau, k_min, sel_idx=None, sel
                                    Hkv, nb, D, rho_min, tau, k_min, sel_idx.data_ptr(),
                                    sel_cnt.data_ptr(), _stream(stream)), "stem_select_static")
     return sel_idx, sel_cnt
+
+
+# ------------------------------------------------------------------ variable-length batches
+
+
+def _cu_array(cu_seqlens):
+    cu = [int(x) for x in cu_seqlens]
+    return (ctypes.c_int32 * len(cu))(*cu), len(cu) - 1
+
+
+def pack_varlen(seqs):
+    """Pack per-sequence [H, S_s, D] tensors back to back (the varlen layout)."""
+    return torch.cat([t.reshape(-1) for t in seqs]), [0] + list(
+        __import__("itertools").accumulate(t.shape[-2] for t in seqs))
+
+
+def stem_varlen_sel_capacity(cu_seqlens, block, method) -> int:
+    arr, n = _cu_array(cu_seqlens)
+    cap = int(_lib.stem_varlen_sel_capacity(n, arr, block, ctypes.byref(method)))
+    if cap < 0:
+        raise StemError(cap, "stem_varlen_sel_capacity")
+    return cap
+
+
+def stem_prefill_varlen(q, k, v, cu_seqlens, Hq, Hkv, D, block, method, out=None, sel_idx=None,
+                        sel_cnt=None, workspace=None, status=None, stream=None):
+    """Variable-length batch on device tensors in the packed layout (pack_varlen): returns
+    (out, sel_idx [Hq * total cap], sel_cnt [Hq * total nb]) as flat tensors."""
+    arr, n = _cu_array(cu_seqlens)
+    dev = q.device
+    cap = stem_varlen_sel_capacity(cu_seqlens, block, method)
+    nbt = sum(-(-(int(cu_seqlens[s + 1]) - int(cu_seqlens[s])) // block) for s in range(n))
+    if out is None:
+        out = torch.empty_like(q)
+        sel_idx = torch.empty(max(Hq * cap, 1), dtype=torch.int32, device=dev)
+        sel_cnt = torch.empty(max(Hq * nbt, 1), dtype=torch.int32, device=dev)
+    if workspace is None:
+        nbytes = int(_lib.stem_varlen_workspace_size(n, arr, Hq, Hkv, D, block))
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    a = stem_varlen_args_t()
+    a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    a.nseq, a.cu_seqlens = n, arr
+    a.Hq, a.Hkv, a.D, a.block, a.dtype = Hq, Hkv, D, block, _dtype_code(q)
+    a.method = ctypes.pointer(method)
+    a.out, a.sel_idx, a.sel_cnt = out.data_ptr(), sel_idx.data_ptr(), sel_cnt.data_ptr()
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    if status is not None:
+        a.status = status.data_ptr()
+    _check(_lib.stem_prefill_varlen(ctypes.byref(a), _stream(stream)), "stem_prefill_varlen")
+    return out, sel_idx, sel_cnt

@@ -253,6 +253,42 @@ int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, i
                        const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
                        void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Variable-length batches. nseq sequences of lengths S_s = cu_seqlens[s+1] - cu_seqlens[s]
+ * (cu_seqlens: host int32[nseq+1], cu_seqlens[0] = 0, non-decreasing), packed back to back, each
+ * as a contiguous [H, S_s, D] slab: sequence s's Q (and out) starts at element Hq*D*cu[s], its K
+ * and V at element Hkv*D*cu[s]. Every sequence is its own problem (its own nb_s = ceil(S_s/block),
+ * budget, selection and attention); an empty sequence contributes nothing. The CSR of sequence s
+ * is [Hq, cap_s] at sel_idx + Hq * (cap_0 + ... + cap_{s-1}), its counts [Hq, nb_s] at
+ * sel_cnt + Hq * (nb_0 + ... + nb_{s-1}), cap_s = stem_sel_capacity_m(nb_s, method).
+ * --------------------------------------------------------------------------------------- */
+typedef struct stem_varlen_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  int32_t nseq;
+  const int32_t* cu_seqlens; /* host */
+  int32_t Hq, Hkv, D, block;
+  int32_t dtype;
+  const stem_method_t* method; /* required */
+  void* out;
+  int32_t* sel_idx;
+  int32_t* sel_cnt;
+  void* workspace;             /* stem_varlen_workspace_size bytes, 256-byte aligned */
+  size_t workspace_bytes;
+  int32_t* status;             /* optional, as in stem_args_t: one word for the whole call */
+} stem_varlen_args_t;
+
+/* Runs the sequences one after another on the stream (the workspace is reused between them). */
+int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream);
+/* Workspace bytes for these sequences (the largest sequence's), 0 on invalid input. Host only. */
+size_t stem_varlen_workspace_size(int nseq, const int32_t* cu_seqlens, int Hq, int Hkv, int D,
+                                  int block);
+/* Total CSR entries per query head: sum over the sequences of cap_s; negative STEM_ERR_* on
+ * invalid input. Host only. */
+int64_t stem_varlen_sel_capacity(int nseq, const int32_t* cu_seqlens, int block,
+                                 const stem_method_t* m);
+
 /*
  * stem_select_static: stem_select for callers that cannot allocate device memory. The paper
  * has no counterpart; this is an interface addition.

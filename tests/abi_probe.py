@@ -107,7 +107,29 @@ BAD_SHARE = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2)
 BAD_SHARE.share = 3
 GROUP = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2, share="group")
 M = lambda m: ctypes.byref(m)  # noqa: E731
+def varlen(cu, method=GOOD, **kw):
+    a = S.stem_varlen_args_t()
+    a.q = a.k = a.v = FAKE
+    a.out, a.sel_idx, a.sel_cnt = FAKE + 0x100, FAKE + 0x200, FAKE + 0x300
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+    a.nseq, a.cu_seqlens = len(cu) - 1, arr
+    a.Hq, a.Hkv, a.D, a.block, a.dtype = 4, 2, 128, 128, 0
+    a.method = ctypes.pointer(method) if method is not None else None
+    a.workspace, a.workspace_bytes = FAKE + 0x1000, 1 << 30
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return L.stem_prefill_varlen(ctypes.byref(a), None)
+
+
 res.update({
+    "varlen_decreasing_cu": varlen([0, 300, 200]),
+    "varlen_cu0_nonzero": varlen([5, 300]),
+    "varlen_no_method": varlen([0, 300], method=None),
+    "varlen_bad_hq": varlen([0, 300], Hq=3),
+    "varlen_q_null": varlen([0, 300], q=None),
+    "varlen_small_workspace": varlen([0, 300], workspace_bytes=64),
+    "varlen_all_empty": varlen([0, 0, 0], q=None, k=None, v=None, out=None, sel_idx=None,
+                               sel_cnt=None),
     "method_bad_mu": ex(method=ctypes.pointer(BAD_MU)),
     "method_bad_beta": ex(method=ctypes.pointer(BAD_BETA)),
     "method_bad_vsum": ex(method=ctypes.pointer(BAD_VSUM)),

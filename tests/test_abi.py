@@ -100,6 +100,23 @@ def test_method_validation(bad):
     assert S.lib().stem_budget_m(64, None, None, None) == S.STEM_ERR_ARG
 
 
+def test_varlen_capacity_and_workspace():
+    m = S.make_method("exp", rho_min=0.2, tau=8.0, k_min=3)
+    cu = [0, 4096, 4173, 4173, 6746]
+    total = sum(S.stem_sel_capacity(-(-(cu[s + 1] - cu[s]) // 128), 0, 0, 0, method=m)
+                for s in range(4))
+    assert S.stem_varlen_sel_capacity(cu, 128, m) == total
+    arr = (ctypes.c_int32 * 5)(*cu)
+    ws = S.lib().stem_varlen_workspace_size(4, arr, 8, 2, 128, 128)
+    assert ws == max(S.stem_workspace_size(1, 8, 2, cu[s + 1] - cu[s], 128, 128)
+                     for s in range(4))
+    for bad in ([1, 5], [0, 5, 3]):
+        arr = (ctypes.c_int32 * len(bad))(*bad)
+        assert S.lib().stem_varlen_sel_capacity(len(bad) - 1, arr, 128, ctypes.byref(m)) == \
+            S.STEM_ERR_ARG
+        assert S.lib().stem_varlen_workspace_size(len(bad) - 1, arr, 8, 2, 128, 128) == 0
+
+
 def test_withhold_switch_is_host_state_only():
     """The test switch for the timeout path is a host-side flag: it toggles, reports the previous
     value and is left off."""
@@ -146,6 +163,8 @@ def test_argument_validation_rejects_before_any_device_work():
         "workspace_misaligned": S.STEM_ERR_WORKSPACE,
         "select_no_workspace": S.STEM_ERR_WORKSPACE,
         "select_m_no_workspace": S.STEM_ERR_WORKSPACE,
+        "varlen_small_workspace": S.STEM_ERR_WORKSPACE,
+        "varlen_all_empty": S.STEM_OK,
         "attn_small_workspace": S.STEM_ERR_WORKSPACE,
         "nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "select_nb_too_large": S.STEM_ERR_UNSUPPORTED,
