@@ -59,6 +59,9 @@ def _load():
         lib.stem_oracle_select.restype = None
         lib.stem_oracle_select.argtypes = [_c_f64p, _c_i32p, _c_i64p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int64, _c_i32p, _c_i32p]
+        lib.stem_oracle_antidiag.restype = None
+        lib.stem_oracle_antidiag.argtypes = ([ctypes.c_void_p] * 2 + [ctypes.c_int] * 8 +
+                                             [_c_i64p, ctypes.c_int64, _c_f64p])
         lib.stem_oracle_attention.restype = None
         lib.stem_oracle_attention.argtypes = ([ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
                                               [_c_i32p, _c_i32p, _c_i64p, ctypes.c_int64,
@@ -162,6 +165,62 @@ def metric_additive(qbar: np.ndarray, kbar: np.ndarray, vnorm: np.ndarray, beta:
     return m
 
 
+def antidiag(q: torch.Tensor, k: torch.Tensor, block: int, stride: int,
+             rows: Optional[Sequence] = None) -> np.ndarray:
+    """Block probabilities estimated by anti-diagonal sampling (see stem_oracle_antidiag).
+
+    rows=None: every query block, packed by row like metric(): [B, Hq, nb*(nb+1)/2].
+    rows = [(b, h, i), ...]: [len(rows), nb], row i's p_ij in columns j <= i."""
+    q, k = _host(q), _host(k)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    if stride < 1 or block % stride or S % stride:
+        raise ValueError("stride must divide the block and the sequence length")
+    nb = -(-S // block)
+    if rows is None:
+        ids = np.arange(B * Hq * nb, dtype=np.int64)
+    else:
+        ids = np.array([(b * Hq + h) * nb + i for (b, h, i) in rows], dtype=np.int64)
+    out = np.zeros((len(ids), nb))
+    if len(ids):
+        _load().stem_oracle_antidiag(q.data_ptr(), k.data_ptr(), _dtype_code(q), B, Hq, Hkv, S,
+                                     D, block, stride, _ptr(ids, _c_i64p), len(ids),
+                                     _ptr(out, _c_f64p))
+    if rows is not None:
+        return out
+    packed = np.zeros((B, Hq, nb * (nb + 1) // 2))
+    full = out.reshape(B, Hq, nb, nb)
+    for i in range(nb):
+        packed[:, :, i * (i + 1) // 2:i * (i + 1) // 2 + i + 1] = full[:, :, i, :i + 1]
+    return packed
+
+
+def metric_from_p(p: np.ndarray, vnorm: np.ndarray, beta: float = 0.0, clamp: bool = True,
+                  form: str = "product") -> np.ndarray:
+    """Output-aware metric from block probabilities p [B, Hq, T] (packed rows) and the V
+    magnitudes vnorm [B, Hkv, nb]: "product" m_ij = p_ij * n_j; "additive"
+    M_ij = ln p_ij + beta * max(0, log n_j^2) (clamp=False drops the max; beta == 0 gives
+    ln p). ln p_ij plays the part of the pooled score s_ij: within a row they differ by the
+    row's log-normaliser only. Query head h reads kv-head h / (Hq/Hkv)."""
+    B, Hq, T = p.shape
+    Hkv, nb = vnorm.shape[1], vnorm.shape[2]
+    G = Hq // Hkv
+    jj = np.concatenate([np.arange(i + 1) for i in range(nb)]) if nb else np.zeros(0, int)
+    n = np.repeat(vnorm, G, axis=1)[:, :, jj]  # n_j per packed entry
+    if form == "product":
+        return p * n
+    if form != "additive":
+        raise ValueError(form)
+    with np.errstate(divide="ignore"):
+        lp = np.log(p)
+        if f32(beta) == 0.0:
+            return lp
+        e = 2.0 * np.log(n)
+    if clamp:
+        e = np.maximum(e, 0.0)
+    return lp + f32(beta) * e
+
+
 def metric_group(m: np.ndarray, G: int) -> np.ndarray:
     """GQA-group metric: the per-head metric summed over the G query heads that share a
     kv-head (heads g*G .. g*G+G-1), [B, Hq/G, T]. The pages are silent on GQA; this is the
@@ -231,13 +290,15 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
             tau: float, k_min: int, rows: Optional[Sequence] = None, with_metric: bool = True,
             schedule: str = "exp", k_start: float = 0.0, mu: float = 1.0,
             metric_form: str = "product", beta: float = 0.0, clamp: bool = True,
-            vsum: str = "mean", share: str = "head"):
+            vsum: str = "mean", share: str = "head", score: str = "pooled", stride: int = 16):
     """All stages. Returns a dict with k, off, qbar, kbar, vnorm, m, sel_idx, sel_cnt and
     out ([len(rows), block, D] for the listed query blocks; all blocks when rows is None).
     schedule "exp" uses rho_min, tau; "linear" uses k_start, mu. metric_form "product" is
     softmax(s) * n, "additive" is s + beta * max(0, log n^2) (clamp=False drops the max).
     share "group" selects once per kv-head group by the metric summed over its query heads
-    (metric_group); m is then the group metric replicated to each head."""
+    (metric_group); m is then the group metric replicated to each head. score "antidiag"
+    takes the block probabilities from anti-diagonal sampling with the given stride
+    (antidiag(), returned as "p") instead of the pooled softmax."""
     B, Hq, S, D = q.shape
     nb = -(-S // block)
     if schedule == "exp":
@@ -247,7 +308,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
     else:
         raise ValueError(schedule)
     qbar, kbar, vnorm = pool(q, k, v, block, vsum)
-    if metric_form == "product":
+    p = None
+    if score == "antidiag":
+        p = antidiag(q, k, block, stride)
+        m = metric_from_p(p, vnorm, beta, clamp, metric_form)
+    elif score != "pooled":
+        raise ValueError(score)
+    elif metric_form == "product":
         m = metric(qbar, kbar, vnorm)
     elif metric_form == "additive":
         m = metric_additive(qbar, kbar, vnorm, beta, clamp)
@@ -266,6 +333,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, rho_m
                sel_cnt=sel_cnt, out=out)
     if with_metric:
         res["m"] = m
+    if p is not None:
+        res["p"] = p
     return res
 
 

@@ -393,3 +393,71 @@ void stem_oracle_attention(const void* q, const void* k, const void* v, int dtyp
     free(keyrow);
   }
 }
+
+/*
+ * Block scores by anti-diagonal sampling ([fr] 2.C step 1: the per-block
+ * metrics are computed with anti-diagonal sampling for efficiency). The pages
+ * give no formula; the reading used here:
+ *   - tokens are grouped into runs of `stride` (sigma) consecutive tokens; a
+ *     group of query tokens u and a group of key tokens w span a sigma x sigma
+ *     sub-tile of the token logit matrix Q K^T / sqrt(D);
+ *   - that sub-tile is sampled along its anti-diagonal (query token
+ *     u*sigma + t with key token w*sigma + sigma-1-t, t = 0..sigma-1), and the
+ *     mean of the sigma samples stands for it:
+ *       a_uw = (1/sigma) sum_t Q[u*sigma+t] . K[w*sigma+sigma-1-t] / sqrt(D);
+ *   - each query group takes a softmax over the key groups it may see
+ *     causally (w <= u);
+ *   - the block probability p_ij is the mass that the query groups of block i
+ *     put on the key groups of block j, averaged over the query groups of
+ *     block i (block / sigma of them; fewer in a partial last block):
+ *       p_ij = (1/n_i) sum_{u in i} sum_{w in j} softmax_w(a_u.),  j = 0..i.
+ *     Each row of p sums to 1 over j <= i, like the pooled probability.
+ * Requires S % stride == 0 and block % stride == 0 (the caller checks).
+ * Computes the listed query blocks only: ids[t] = (b*Hq + h)*nb + i;
+ * p_out [nids, nb] (double), entries j > i left 0.
+ */
+void stem_oracle_antidiag(const void* q, const void* k, int dtype, int B, int Hq, int Hkv,
+                          int S, int D, int block, int stride, const int64_t* ids,
+                          int64_t nids, double* p_out) {
+  const int nb = (S + block - 1) / block;
+  const int G = Hq / Hkv;
+  const int R = block / stride;   /* query (or key) groups per block */
+  const int nred = S / stride;    /* groups per head */
+  const double scale = 1.0 / ((double)stride * sqrt((double)D));
+  (void)B;
+#pragma omp parallel
+  {
+    double* a = (double*)malloc(sizeof(double) * (size_t)(nred > 0 ? nred : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nids; ++t) {
+      const int64_t id = ids[t];
+      const int64_t bh = id / nb;
+      const int i = (int)(id % nb);
+      const int64_t b = bh / Hq, h = bh % Hq;
+      const int64_t qbase = bh * (int64_t)S;                    /* token 0 of this head */
+      const int64_t kbase = (b * Hkv + h / G) * (int64_t)S;
+      double* prow = p_out + t * (int64_t)nb;
+      for (int j = 0; j < nb; ++j) prow[j] = 0.0;
+      const int u0 = i * R;
+      const int n_i = nred - u0 < R ? nred - u0 : R;             /* query groups of block i */
+      for (int u = u0; u < u0 + n_i; ++u) {
+        double mx = -INFINITY;
+        for (int w = 0; w <= u; ++w) {
+          double acc = 0.0;
+          for (int s = 0; s < stride; ++s) {
+            const int64_t qtok = qbase + (int64_t)u * stride + s;
+            const int64_t ktok = kbase + (int64_t)w * stride + (stride - 1 - s);
+            for (int d = 0; d < D; ++d)
+              acc += elem(q, dtype, qtok * D + d) * elem(k, dtype, ktok * D + d);
+          }
+          a[w] = acc * scale;
+          if (a[w] > mx) mx = a[w];
+        }
+        double z = 0.0;
+        for (int w = 0; w <= u; ++w) z += exp(a[w] - mx);
+        for (int w = 0; w <= u; ++w) prow[w / R] += exp(a[w] - mx) / z / n_i;
+      }
+    }
+    free(a);
+  }
+}

@@ -84,3 +84,32 @@ def attention_masked(q, k, v, block, kept):
             w = scipy.special.softmax(logits, axis=-1)
             out[b, h] = w @ V[b, h // G]
     return out
+
+
+def antidiag(q, k, block, stride):
+    """Anti-diagonal block probabilities from the full token logit matrix: the samples are
+    picked out of Q K^T / sqrt(D) (numpy matmul) by index, averaged per sub-tile, softmaxed
+    per query group (scipy) and summed per block. Returns [B, Hq, nb, nb] (0 above i)."""
+    B, Hq, S, D = q.shape
+    G = Hq // k.shape[1]
+    nb = -(-S // block)
+    R = block // stride
+    nred = S // stride
+    t = np.arange(stride)
+    out = np.zeros((B, Hq, nb, nb))
+    for b in range(B):
+        for h in range(Hq):
+            Q = q[b, h].double().numpy()
+            K = k[b, h // G].double().numpy()
+            X = Q @ K.T / np.sqrt(D)
+            u = np.arange(nred)
+            rows = u[:, None, None] * stride + t[None, None, :]                  # [u, 1, t]
+            cols = u[None, :, None] * stride + (stride - 1 - t)[None, None, :]   # [1, w, t]
+            A = X[rows, cols].mean(axis=2)                                       # [u, w]
+            A = np.where(np.tril(np.ones((nred, nred), bool)), A, -np.inf)
+            P = scipy.special.softmax(A, axis=1)
+            for i in range(nb):
+                us = range(i * R, min((i + 1) * R, nred))
+                for j in range(i + 1):
+                    out[b, h, i, j] = np.mean([P[uu, j * R:(j + 1) * R].sum() for uu in us])
+    return out

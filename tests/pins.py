@@ -34,6 +34,13 @@ What pins what:
              that are all equal give the per-head selection of any of them; the full
              sort of the numpy brute-force metric summed over the group's heads; the
              additive form sums to sum_h s + G*beta*e.
+  antidiag   block probabilities by anti-diagonal sampling: two cases worked by hand
+             (tests/golden/antidiag_hand.txt); the samples picked by index out of the full
+             numpy logit matrix (brute force); stride 1 is the block mass of exact causal
+             attention (torch softmax in float64); stride = block with keys constant per
+             block is the pooled softmax; rows sum to 1; a prefix gives the same rows. The
+             metric from p: the product form in the pooled limit equals the pooled metric,
+             the additive form at beta = 1/2 without the clamp is the log of the product.
   ragged S   S % block != 0: pooling and attention against the slicing / token-mask
              brute force; a partial block of constant rows pools to that row; the
              full blocks do not depend on the tokens past them (a prefix of the
@@ -575,6 +582,108 @@ def pin_ragged():
                                rtol=1e-12)
 
 
+# --------------------------------------------------------------------------- anti-diagonal
+
+
+def _hand_antidiag_cases():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                        "antidiag_hand.txt")
+    cases = []
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        head, qs, ks, ps = line.split("|")
+        S, D, block, stride = (int(x) for x in head.split())
+        rows = [[float(x) for x in r.split()] for r in ps.split(";")]
+        cases.append((S, D, block, stride, [float(x) for x in qs.split()],
+                      [float(x) for x in ks.split()], rows))
+    return cases
+
+
+def pin_antidiag_hand():
+    cases = _hand_antidiag_cases()
+    assert len(cases) == 2
+    for S, D, block, stride, qv, kv, rows in cases:
+        for dtype in (torch.float32, torch.bfloat16):  # every value is exact in bf16
+            q = torch.tensor(qv).reshape(1, 1, S, D).to(dtype)
+            k = torch.tensor(kv).reshape(1, 1, S, D).to(dtype)
+            got = oracle.antidiag(q, k, block, stride, rows=[(0, 0, i) for i in range(len(rows))])
+            for i, want in enumerate(rows):
+                np.testing.assert_allclose(got[i, :i + 1], want, rtol=1e-14, atol=1e-15)
+
+
+def pin_antidiag_brute():
+    for dtype, (S, block, stride) in ((torch.float32, (128, 16, 4)),
+                                      (torch.bfloat16, (16 * 5 + 8, 16, 8)),
+                                      (torch.float32, (96, 32, 2))):
+        q, k, _ = _tiny_inputs(81, Hq=4, Hkv=2, S=S, D=8, block=block, dtype=dtype)
+        got = oracle.antidiag(q, k, block, stride)
+        ref = brute.antidiag(q, k, block, stride)
+        nb = ref.shape[2]
+        for i in range(nb):
+            np.testing.assert_allclose(oracle.metric_row(got, 0, 1, i), ref[0, 1, i, :i + 1],
+                                       rtol=1e-11, atol=1e-14)
+            np.testing.assert_allclose(got[0, :, i * (i + 1) // 2:i * (i + 1) // 2 + i + 1],
+                                       ref[0, :, i, :i + 1], rtol=1e-11, atol=1e-14)
+
+
+def pin_antidiag_stride1():
+    # one token per group: a_uw is the token logit and p_ij the block mass of exact causal
+    # attention, averaged over the block's query tokens
+    for dtype, S in ((torch.float32, 128), (torch.bfloat16, 16 * 6 + 5)):
+        q, k, _ = _tiny_inputs(83, Hq=4, Hkv=2, S=S, D=16, block=16, dtype=dtype)
+        got = oracle.antidiag(q, k, 16, 1)
+        kk = k.double().repeat_interleave(2, dim=1)
+        X = q.double() @ kk.transpose(-1, -2) / 4.0
+        X = X.masked_fill(~torch.ones(S, S, dtype=torch.bool).tril(), float("-inf"))
+        P = torch.softmax(X, dim=-1).numpy()  # [1, 4, S, S]
+        nb = -(-S // 16)
+        for h in range(4):
+            for i in range(nb):
+                r0, r1 = i * 16, min(S, i * 16 + 16)
+                want = [P[0, h, r0:r1, j * 16:min(S, j * 16 + 16)].sum(axis=1).mean()
+                        for j in range(i + 1)]
+                np.testing.assert_allclose(oracle.metric_row(got, 0, h, i), want, rtol=1e-11,
+                                           atol=1e-14)
+
+
+def pin_antidiag_pooled_limit_and_metric():
+    # stride = block and keys constant inside each block: a_ij = qbar_i . k_j / sqrt(D), the
+    # pooled score, so p is the pooled softmax and the product metric the pooled metric
+    q, k, v = _tiny_inputs(85, Hq=4, Hkv=2, S=128, D=16, block=16)
+    kc = k.reshape(1, 2, 8, 16, 16)[:, :, :, :1, :].expand(1, 2, 8, 16, 16).reshape(1, 2, 128, 16)
+    kc = kc.contiguous()
+    p = oracle.antidiag(q, kc, 16, 16)
+    qb, kb, vn = oracle.pool(q, kc, v, 16)
+    np.testing.assert_allclose(p, oracle.metric(qb, kb, np.ones_like(vn)), rtol=1e-11,
+                               atol=1e-14)
+    np.testing.assert_allclose(oracle.metric_from_p(p, vn), oracle.metric(qb, kb, vn),
+                               rtol=1e-11, atol=1e-14)
+    # additive at beta = 1/2 without the clamp: ln p + ln n = ln(p n)
+    p = oracle.antidiag(q, k, 16, 4)
+    _, _, vn = oracle.pool(q, k, v, 16)
+    np.testing.assert_allclose(oracle.metric_from_p(p, vn, 0.5, False, "additive"),
+                               np.log(oracle.metric_from_p(p, vn)), rtol=1e-12, atol=1e-12)
+    # beta = 0: ln p
+    np.testing.assert_allclose(oracle.metric_from_p(p, vn, 0.0, True, "additive"), np.log(p),
+                               rtol=0, atol=0)
+
+
+def pin_antidiag_invariants():
+    S, block, stride = 16 * 7 + 8, 16, 8
+    q, k, _ = _tiny_inputs(87, Hq=4, Hkv=2, S=S, D=16, block=block, dtype=torch.bfloat16)
+    p = oracle.antidiag(q, k, block, stride)
+    nb = 8
+    for h in range(4):
+        for i in range(nb):
+            row = oracle.metric_row(p, 0, h, i)
+            assert np.all(row > 0)
+            assert abs(row.sum() - 1.0) < 1e-12
+    # causality: the first 7 blocks of a prefix give the same rows
+    pre = oracle.antidiag(q[:, :, :112], k[:, :, :112], block, stride)
+    np.testing.assert_array_equal(p[:, :, :pre.shape[2]], pre)
+
+
 PINS = [
     pin_budget_decimal,
     pin_budget_closed_forms,
@@ -593,6 +702,11 @@ PINS = [
     pin_attention_brute,
     pin_ragged,
     pin_group,
+    pin_antidiag_hand,
+    pin_antidiag_brute,
+    pin_antidiag_stride1,
+    pin_antidiag_pooled_limit_and_metric,
+    pin_antidiag_invariants,
 ]
 
 

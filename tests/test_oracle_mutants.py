@@ -66,6 +66,19 @@ MUTANTS = [
      "vnorm[u] = vmax ? nmax : nacc / block;"),
     ("ragged-last-rows", "for (int r = 0; r < block && (int64_t)i * block + r < S; ++r) {",
      "for (int r = 0; r < block && (int64_t)i * block + r < S - 1; ++r) {"),
+    ("antidiag-main-diagonal", "(int64_t)w * stride + (stride - 1 - s);", "(int64_t)w * stride + s;"),
+    ("antidiag-no-stride-scale", "const double scale = 1.0 / ((double)stride * sqrt((double)D));",
+     "const double scale = 1.0 / sqrt((double)D);"),
+    ("antidiag-strict-mask", "for (int w = 0; w <= u; ++w) {\n          double acc = 0.0;",
+     "for (int w = 0; w < u; ++w) {\n          double acc = 0.0;"),
+    ("antidiag-divisor", "prow[w / R] += exp(a[w] - mx) / z / n_i;",
+     "prow[w / R] += exp(a[w] - mx) / z / R;"),
+    ("antidiag-block-map", "prow[w / R] += exp(a[w] - mx) / z / n_i;",
+     "prow[w / stride] += exp(a[w] - mx) / z / n_i;"),
+    ("antidiag-gqa", "const int64_t kbase = (b * Hkv + h / G) * (int64_t)S;",
+     "const int64_t kbase = (b * Hkv + h % Hkv) * (int64_t)S;"),
+    ("antidiag-unnormalised", "prow[w / R] += exp(a[w] - mx) / z / n_i;",
+     "prow[w / R] += exp(a[w] - mx) / n_i;"),
 ]
 
 
