@@ -58,11 +58,15 @@ def parse():
     p.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--method", choices=["default", "pages", "group"], default="default",
+    p.add_argument("--method", choices=["default", "pages", "group", "antidiag"],
+                   default="default",
                    help="default: exponential budget, product metric, mean V norms; pages: the "
                         "pages' linear budget (mu 0.7) with the additive metric (beta 0.2, "
                         "clamped) and max-pooled V norms, k_start set for the default's mean "
-                        "budget; group: the default with one selection per kv-head group")
+                        "budget; group: the default with one selection per kv-head group; "
+                        "antidiag: the default with block probabilities by anti-diagonal "
+                        "sampling (--stride tokens per group)")
+    p.add_argument("--stride", type=int, default=16)
     return p.parse_args()
 
 
@@ -163,7 +167,7 @@ class ClockSampler:
 # ------------------------------------------------------------------ CPU oracle (reference arm)
 
 
-def method_params(w, name):
+def method_params(w, name, stride=16):
     """Method parameters of a bench run (None: the library's default). "pages": the pages' own
     forms with their ablation optimum (mu 0.7, beta 0.2); k_start gives the linear budget the
     same mean as the workload's default budget, 2 * mean / (1 + mu), to one decimal."""
@@ -171,6 +175,9 @@ def method_params(w, name):
         return None
     if name == "group":
         return dict(schedule="exp", rho_min=w.rho_min, tau=w.tau, k_min=w.k_min, share="group")
+    if name == "antidiag":
+        return dict(schedule="exp", rho_min=w.rho_min, tau=w.tau, k_min=w.k_min,
+                    score="antidiag", stride=stride)
     from block_sparse_causal_pooling_b200 import stem as S
 
     kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
@@ -185,10 +192,28 @@ def oracle_sample_step(w, q, k, v, rows, mp=None):
     block of the group's heads, then exact attention for the listed rows. Returns (effective
     FLOP of the listed rows, seconds for attention + selection prorated to those rows).
     mp: method parameters (method_params) or None for the default."""
+    import numpy as np
+
     import oracle
 
     G = w.Hq // w.Hkv
     qs, ks, vs = q[:, :G].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous()
+    if mp is not None and mp.get("score") == "antidiag":
+        # block probabilities of the sampled rows only (the estimator's cost grows with i);
+        # the other rows get uniform placeholders, so their selections are valid but unused
+        t0 = time.perf_counter()
+        kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+        _, _, vn = oracle.pool(qs, ks, vs, w.block)
+        pr = oracle.antidiag(qs, ks, w.block, mp["stride"], rows=rows)
+        p = np.ones((1, G, w.nb * (w.nb + 1) // 2))
+        for (_, h, i), r in zip(rows, pr):
+            p[0, h, i * (i + 1) // 2:i * (i + 1) // 2 + i + 1] = r[:i + 1]
+        si, sc = oracle.select(oracle.metric_from_p(p, vn), kk, off)
+        t1 = time.perf_counter()
+        oracle.attention(qs, ks, vs, w.block, si, sc, off, rows)
+        t2 = time.perf_counter()
+        flop = sum(wl.effective_flops(int(kk[i]), w.block, w.D) for (_, _, i) in rows)
+        return flop, t2 - t0, dict(select_s=t1 - t0, attn_s=t2 - t1)
     t0 = time.perf_counter()
     if mp is None or mp.get("schedule") == "exp":
         kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
@@ -222,7 +247,7 @@ def run_reference(args, world, rank):
     import oracle
 
     w = wl.WORKLOADS[args.workload]
-    mp = method_params(w, args.method)
+    mp = method_params(w, args.method, args.stride)
     q, k, v = cpu_inputs(w)
     G = w.Hq // w.Hkv
     import random
@@ -330,11 +355,11 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = wl.WORKLOADS[args.workload]
-    mp = method_params(w, args.method)
+    mp = method_params(w, args.method, args.stride)
     meth = None if mp is None else S.make_method(**mp)
     q, k, v = wl.make_inputs(rank_workload(w, rank), dev)
     out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min, meth)
-    ws = S.alloc_workspace(q, k, w.block)
+    ws = S.alloc_workspace(q, k, w.block, meth)
     if meth is None:
         kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
     else:
@@ -443,6 +468,16 @@ def run_ours(args, world, rank, local):
         "clocks": clk,
         "gpu_launches": KERNELS_PER_STEP * K,
     }
+    if mp is not None and mp.get("score") == "antidiag":
+        # the estimator: 2 * stride*D FLOP per causal (query group, key group) pair; its time is
+        # the "select" stage, which also holds the selection from p (a lower bound on its rate)
+        nred = w.S // mp["stride"]
+        ad_flop = w.B * w.Hq * 2.0 * mp["stride"] * w.D * nred * (nred + 1) / 2
+        ad_tf = ad_flop / (sel_ms * 1e-3) / 1e12
+        line["kernels"]["select"].update({
+            "what": "antidiag estimator + selection from p", "bound": "tensor",
+            "estimator_tflop": ad_flop / 1e12, "tflops": ad_tf, "frac": ad_tf / peak_tf})
+        line["gpu_launches"] = (KERNELS_PER_STEP + 1) * K
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:

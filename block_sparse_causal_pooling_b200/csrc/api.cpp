@@ -63,7 +63,20 @@ bool method_ok(int nb, const stem_method_t& m) {
     return false;
   }
   if (m.share != STEM_SHARE_HEAD && m.share != STEM_SHARE_GROUP) return false;
+  if (m.score != STEM_SCORE_POOLED && m.score != STEM_SCORE_ANTIDIAG) return false;
   return m.vsum == STEM_VSUM_MEAN || m.vsum == STEM_VSUM_MAX;
+}
+
+bool antidiag(const stem_method_t& m) { return m.score == STEM_SCORE_ANTIDIAG; }
+
+// The anti-diagonal estimator's shape rules: a power-of-two stride dividing the block (at most
+// 32 groups per block) and the sequence; bfloat16 inputs.
+int check_antidiag(int S, int block, int dtype, int stride) {
+  if (stride < 1 || (stride & (stride - 1)) || block % stride || block / stride > 32 ||
+      S % stride)
+    return STEM_ERR_ARG;
+  if (dtype != STEM_BF16) return STEM_ERR_UNSUPPORTED;
+  return STEM_OK;
 }
 
 // Exponential: k(i) = min(i+1, max(k_min, ceil(rho(i) (i+1)))), rho(i) = rho_min + (1-rho_min)
@@ -147,10 +160,12 @@ const Plan* get_plan(int nb, const stem_method_t& m) {
 
 struct Layout {
   size_t status = 0, plan = 0, sched = 0, sched_end = 0, qbar = 0, kbar = 0, vnorm = 0,
-         total = 0;
+         adp = 0, ads = 0, total = 0;
 };
 
-Layout layout(int B, int Hq, int Hkv, int nb, int D) {
+// m (with S and block) adds the anti-diagonal estimator's regions when it asks for them.
+Layout layout(int B, int Hq, int Hkv, int nb, int D, const stem_method_t* m = nullptr, int S = 0,
+              int block = 0) {
   Layout L;
   size_t o = 0;
   L.status = o;
@@ -166,6 +181,12 @@ Layout layout(int B, int Hq, int Hkv, int nb, int D) {
   o += align_up(sizeof(float) * static_cast<size_t>(B) * Hkv * nb * D);
   L.vnorm = o;
   o += align_up(sizeof(float) * static_cast<size_t>(B) * Hkv * nb);
+  if (m != nullptr && antidiag(*m)) {
+    L.adp = o;  // p [B*Hq][nb*(nb+1)/2]
+    o += align_up(sizeof(float) * static_cast<size_t>(B) * Hq * nb * (nb + 1) / 2);
+    L.ads = o;  // estimator scratch
+    o += align_up(sizeof(float) * antidiag_scratch_floats(B, Hq, S, block, m->stride));
+  }
   L.total = o;
   return L;
 }
@@ -251,12 +272,14 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
   const stem_method_t m = args_method(a);
   rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
+  if (antidiag(m) && (rc = check_antidiag(a->S, a->block, a->dtype, m.stride)) != STEM_OK)
+    return rc;
   if (is_empty(a->B, a->S)) return STEM_OK;
   if (!a->q || !a->k || !a->v || !a->out || !a->sel_idx || !a->sel_cnt) return STEM_ERR_ARG;
   if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->out, 16) ||
       !aligned(a->sel_idx, 4) || !aligned(a->sel_cnt, 4) || !aligned(a->status, 4))
     return STEM_ERR_ARG;
-  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D);
+  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D, &m, a->S, a->block);
   if (a->workspace == nullptr || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total)
     return STEM_ERR_WORKSPACE;
   const Plan* plan = get_plan(nb, m);
@@ -278,7 +301,7 @@ int run_prefill(const stem_args_t* a, cudaStream_t st) {
 int enqueue_kernels(const stem_args_t* a, const stem_method_t& m, int nb, int64_t cap,
                     PlanDev pd, cudaStream_t st) {
   int rc = STEM_OK;
-  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D);
+  const Layout L = layout(a->B, a->Hq, a->Hkv, nb, a->D, &m, a->S, a->block);
   auto* ws = static_cast<unsigned char*>(a->workspace);
   float* qbar = reinterpret_cast<float*>(ws + L.qbar);
   float* kbar = reinterpret_cast<float*>(ws + L.kbar);
@@ -292,8 +315,18 @@ int enqueue_kernels(const stem_args_t* a, const stem_method_t& m, int nb, int64_
                             a->block, m.vsum == STEM_VSUM_MAX, qbar, kbar, vnorm, st));
   if (rc != STEM_OK) return rc;
   if ((rc = mark(1)) != STEM_OK) return rc;
-  rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, cap,
-                              sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st));
+  if (antidiag(m)) {
+    float* p = reinterpret_cast<float*>(ws + L.adp);
+    rc = cuda_err(launch_antidiag(a->q, a->k, a->B, a->Hq, a->Hkv, a->S, a->D, a->block,
+                                  m.stride, p, reinterpret_cast<float*>(ws + L.ads), a->status,
+                                  st));
+    if (rc != STEM_OK) return rc;
+    rc = cuda_err(launch_select_p(p, vnorm, a->B, a->Hq, a->Hkv, nb, pd, cap, sel_metric(m),
+                                  a->sel_idx, a->sel_cnt, nullptr, st));
+  } else {
+    rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, cap,
+                                sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st));
+  }
   if (rc != STEM_OK) return rc;
   if ((rc = mark(2)) != STEM_OK) return rc;
   if (a->dtype == STEM_BF16) {
@@ -400,6 +433,17 @@ size_t stem_workspace_size(int B, int Hq, int Hkv, int S, int D, int block) {
   return layout(B, Hq, Hkv, nblocks(S, block), D).total;
 }
 
+size_t stem_workspace_size_m(int B, int Hq, int Hkv, int S, int D, int block,
+                             const stem_method_t* m) {
+  if (m == nullptr) return 0;
+  if (check_shape(B, Hq, Hkv, S, D, block, STEM_BF16) != STEM_OK) return 0;
+  const int nb = nblocks(S, block);
+  if (!method_ok(nb, *m)) return 0;
+  if (antidiag(*m) && check_antidiag(S, block, STEM_BF16, m->stride) != STEM_OK) return 0;
+  if (is_empty(B, S)) return 0;
+  return layout(B, Hq, Hkv, nb, D, m, S, block).total;
+}
+
 const char* stem_strerror(int code) {
   switch (code) {
     case STEM_OK: return "success";
@@ -461,6 +505,8 @@ int stem_prefill_host(const stem_args_t* h) {
   const stem_method_t m = args_method(h);
   rc = check_params(nb, m);
   if (rc != STEM_OK) return rc;
+  if (antidiag(m) && (rc = check_antidiag(h->S, h->block, h->dtype, m.stride)) != STEM_OK)
+    return rc;
   if (is_empty(h->B, h->S)) return STEM_OK;
   if (!h->q || !h->k || !h->v || !h->out || !h->sel_idx || !h->sel_cnt) return STEM_ERR_ARG;
   const int G = h->Hq / h->Hkv;
@@ -471,7 +517,7 @@ int stem_prefill_host(const stem_args_t* h) {
   const size_t kvcb = es * static_cast<size_t>(h->S) * h->D;
   const size_t sicb = sizeof(int32_t) * static_cast<size_t>(G) * cap;
   const size_t sccb = sizeof(int32_t) * static_cast<size_t>(G) * nb;
-  const Layout Lc = layout(1, G, 1, nb, h->D);  // one chunk's workspace
+  const Layout Lc = layout(1, G, 1, nb, h->D, &m, h->S, h->block);  // one chunk's workspace
   const Plan* plan = get_plan(nb, m);
   if (plan == nullptr) return STEM_ERR_CUDA;
   // device arena: chunk status words | the plan | chunk workspaces | q | k | v | out | sel_idx |
@@ -613,6 +659,62 @@ int stem_select_m(const float* qbar, const float* kbar, const float* vnorm, int 
                                 sel_metric(*m), sel_idx, sel_cnt, m_out, st));
 }
 
+int stem_antidiag_m(const void* q, const void* k, int dtype, int B, int Hq, int Hkv, int S, int D,
+                    int block, const stem_method_t* m, float* p, void* workspace,
+                    size_t workspace_bytes, int32_t* status, void* stream) {
+  if (m == nullptr) return STEM_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, S, D, block, dtype);
+  if (rc != STEM_OK) return rc;
+  rc = check_antidiag(S, block, dtype, m->stride);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, S)) return STEM_OK;
+  if (!q || !k || !p) return STEM_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(p, 4) || !aligned(status, 4))
+    return STEM_ERR_ARG;
+  stem_method_t ma = *m;
+  ma.score = STEM_SCORE_ANTIDIAG;
+  const int nb = nblocks(S, block);
+  const Layout L = layout(B, Hq, Hkv, nb, D, &ma, S, block);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.total)
+    return STEM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (status) {
+    rc = cuda_err(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    if (rc != STEM_OK) return rc;
+  }
+  return cuda_err(launch_antidiag(q, k, B, Hq, Hkv, S, D, block, m->stride, p,
+                                  reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
+                                                           L.ads),
+                                  status, st));
+}
+
+int stem_select_p_m(const float* p, const float* vnorm, int B, int Hq, int Hkv, int nb,
+                    const stem_method_t* m, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (nb < 0 || m == nullptr) return STEM_ERR_ARG;
+  if (nb > STEM_MAX_NB) return STEM_ERR_UNSUPPORTED;
+  int rc = check_shape(B, Hq, Hkv, nb * 64, 64, 64, STEM_F32);  // the selection sees blocks only
+  if (rc != STEM_OK) return rc;
+  rc = check_params(nb, *m);
+  if (rc != STEM_OK) return rc;
+  if (is_empty(B, nb)) return STEM_OK;
+  if (!p || !vnorm || !sel_idx || !sel_cnt) return STEM_ERR_ARG;
+  if (!aligned(p, 4) || !aligned(vnorm, 4) || !aligned(sel_idx, 4) || !aligned(sel_cnt, 4) ||
+      !aligned(m_out, 4))
+    return STEM_ERR_ARG;
+  const Layout L = layout(B, Hq, Hkv, nb, 64);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < L.plan + plan_bytes(nb))
+    return STEM_ERR_WORKSPACE;
+  const Plan* plan = get_plan(nb, *m);
+  if (plan == nullptr) return STEM_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  PlanDev pd;
+  rc = upload_plan(plan, workspace, L, st, &pd);
+  if (rc != STEM_OK) return rc;
+  return cuda_err(launch_select_p(p, vnorm, B, Hq, Hkv, nb, pd, plan->cap, sel_metric(*m), sel_idx,
+                                  sel_cnt, m_out, st));
+}
+
 int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
                 int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
                 int32_t* sel_cnt, float* m_out, void* workspace, size_t workspace_bytes,
@@ -691,18 +793,24 @@ int64_t stem_varlen_sel_capacity(int nseq, const int32_t* cu, int block, const s
   return total;
 }
 
-size_t stem_varlen_workspace_size(int nseq, const int32_t* cu, int Hq, int Hkv, int D,
-                                  int block) {
+size_t stem_varlen_workspace_size_m(int nseq, const int32_t* cu, int Hq, int Hkv, int D,
+                                    int block, const stem_method_t* m) {
   if (check_cu(nseq, cu) != STEM_OK) return 0;
   size_t most = 0;
   for (int s = 0; s < nseq; ++s) {
     const int S = cu[s + 1] - cu[s];
     if (S == 0) continue;
-    const size_t n = stem_workspace_size(1, Hq, Hkv, S, D, block);
+    const size_t n = m ? stem_workspace_size_m(1, Hq, Hkv, S, D, block, m)
+                       : stem_workspace_size(1, Hq, Hkv, S, D, block);
     if (n == 0) return 0;
     most = std::max(most, n);
   }
   return most;
+}
+
+size_t stem_varlen_workspace_size(int nseq, const int32_t* cu, int Hq, int Hkv, int D,
+                                  int block) {
+  return stem_varlen_workspace_size_m(nseq, cu, Hq, Hkv, D, block, nullptr);
 }
 
 int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream) {
@@ -719,7 +827,11 @@ int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream) {
     if (rc != STEM_OK) return rc;
     rc = check_params(nblocks(S, a->block), m);
     if (rc != STEM_OK) return rc;
-    if (S > 0) need = std::max(need, layout(1, a->Hq, a->Hkv, nblocks(S, a->block), a->D).total);
+    if (antidiag(m) && (rc = check_antidiag(S, a->block, a->dtype, m.stride)) != STEM_OK)
+      return rc;
+    if (S > 0)
+      need = std::max(need,
+                      layout(1, a->Hq, a->Hkv, nblocks(S, a->block), a->D, &m, S, a->block).total);
   }
   if (need == 0) return STEM_OK;  // no tokens
   if (!a->q || !a->k || !a->v || !a->out || !a->sel_idx || !a->sel_cnt) return STEM_ERR_ARG;
@@ -764,7 +876,8 @@ int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream) {
     // the plan goes into the shared workspace in stream order, after the previous sequence's
     // kernels have read theirs
     PlanDev pd;
-    rc = upload_plan(plan, a->workspace, layout(1, a->Hq, a->Hkv, nb, a->D), st, &pd);
+    rc = upload_plan(plan, a->workspace, layout(1, a->Hq, a->Hkv, nb, a->D, &m, S, a->block), st,
+                     &pd);
     if (rc != STEM_OK) return rc;
     rc = enqueue_kernels(&d, m, nb, plan->cap, pd, st);
     if (rc != STEM_OK) return rc;

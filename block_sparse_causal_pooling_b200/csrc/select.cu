@@ -524,7 +524,131 @@ cudaError_t launch_d(const float* qbar, const float* kbar, const float* vnorm, i
                          m_out, st);
 }
 
+// ---- Selection from block probabilities p_ij (block scores by anti-diagonal sampling). ln p_ij
+// takes the place of s_ij - lse_i: per head the key is ln p_ij + ln n_j (product) or
+// ln p_ij + beta * e_j (additive); shared by a kv-head group it is ln n_j + logsumexp_h ln p_hij
+// (product: the group's summed metric n_j * sum_h p_hij) or sum_h ln p_hij + G * beta * e_j.
+// One CTA (8 warps) per (b, head or group, 8 consecutive query blocks), one row per warp; p rows
+// are read from global memory (L1/L2), the group's combined row is built in shared memory.
+template <bool kGroup>
+__global__ void __launch_bounds__(kSelThreads) select_p_kernel(
+    const float* __restrict__ p, const float* __restrict__ vnorm, int B, int Hq, int Hkv, int nb,
+    int ldS, PlanDev plan, int64_t cap, SelMetric metric, int32_t* __restrict__ sel_idx,
+    int32_t* __restrict__ sel_cnt, float* __restrict__ m_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* lnn = reinterpret_cast<double*>(smem_raw);                 // [ldS]
+  double* acc = lnn + ldS;                                           // kGroup: [kWarps][ldS]
+  int* hist_all = reinterpret_cast<int*>(acc + (kGroup ? kWarps * ldS : 0));  // [kWarps][256]
+  const int G = Hq / Hkv;
+  const int NH = kGroup ? B * Hkv : B * Hq;  // selection heads
+  const int ntiles = (nb + kWarps - 1) / kWarps;
+  const int tile = ntiles - 1 - static_cast<int>(blockIdx.x / NH);  // heaviest rows first
+  const int sh = static_cast<int>(blockIdx.x % NH);
+  const int b = kGroup ? sh / Hkv : sh / Hq;
+  const int g = kGroup ? sh % Hkv : (sh % Hq) / G;  // kv head
+  const int i0 = tile * kWarps;
+  const int rows = min(kWarps, nb - i0);
+  const int jend = i0 + rows;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int64_t bg = static_cast<int64_t>(b) * Hkv + g;
+  const float* nsrc = vnorm + bg * nb;
+  const int64_t tri = static_cast<int64_t>(nb) * (nb + 1) / 2;
+  for (int j = t; j < jend; j += kSelThreads) {
+    double c;
+    if (!metric.additive) {
+      c = log(static_cast<double>(nsrc[j]));
+    } else if (metric.beta == 0.f) {
+      c = 0.0;
+    } else {
+      double e = 2.0 * log(static_cast<double>(nsrc[j]));
+      if (metric.clamp && e < 0.0) e = 0.0;
+      c = static_cast<double>(metric.beta) * e;
+    }
+    lnn[j] = c;
+  }
+  __syncthreads();
+  if (warp >= rows) return;  // no __syncthreads below
+  const int i = i0 + warp;
+  const int kk = plan.k[i];
+  const int64_t rowoff = static_cast<int64_t>(i) * (i + 1) / 2;
+  int* hist = hist_all + warp * 256;
+  if (!kGroup) {
+    const int64_t bh = static_cast<int64_t>(b) * Hq + sh % Hq;
+    const float* prow = p + bh * tri + rowoff;
+    if (lane == 0) sel_cnt[bh * nb + i] = kk;
+    if (m_out != nullptr)
+      for (int j = lane; j <= i; j += 32)
+        m_out[bh * tri + rowoff + j] =
+            metric.additive ? static_cast<float>(log(static_cast<double>(prow[j])) + lnn[j])
+                            : prow[j] * nsrc[j];
+    auto key_bits = [&](int j) -> uint64_t {
+      return order_bits(log(static_cast<double>(__ldg(prow + j))) + lnn[j]);
+    };
+    select_row(i, kk, key_bits, hist, lane, sel_idx + bh * cap + plan.off[i], 0, 1);
+  } else {
+    double* arow = acc + warp * ldS;
+    const int64_t bh0 = static_cast<int64_t>(b) * Hq + g * G;
+    for (int h = 0; h < G; ++h) {
+      const float* prow = p + (bh0 + h) * tri + rowoff;
+      for (int j = lane; j <= i; j += 32) {
+        const double x = log(static_cast<double>(prow[j]));
+        if (metric.additive) {
+          arow[j] = (h == 0 ? 0.0 : arow[j]) + x;
+        } else if (h == 0) {
+          arow[j] = x;
+        } else {  // log-add-exp; a zero probability adds nothing
+          const double a = arow[j];
+          const double hi = fmax(a, x), lo = fmin(a, x);
+          arow[j] = lo == -INFINITY ? hi : hi + log1p(exp(lo - hi));
+        }
+      }
+    }
+    const double gterm = metric.additive ? static_cast<double>(G) : 1.0;
+    for (int j = lane; j <= i; j += 32) arow[j] += gterm * lnn[j];
+    __syncwarp();
+    for (int h = lane; h < G; h += 32) sel_cnt[(bh0 + h) * nb + i] = kk;
+    if (m_out != nullptr)
+      for (int j = lane; j <= i; j += 32) {
+        const float mv = static_cast<float>(metric.additive ? arow[j] : exp(arow[j]));
+        for (int h = 0; h < G; ++h) m_out[(bh0 + h) * tri + rowoff + j] = mv;
+      }
+    auto key_bits = [&](int j) -> uint64_t { return order_bits(arow[j]); };
+    select_row(i, kk, key_bits, hist, lane, sel_idx + bh0 * cap + plan.off[i], cap, G);
+  }
+}
+
+template <bool kGroup>
+cudaError_t launch_p(const float* p, const float* vnorm, int B, int Hq, int Hkv, int nb,
+                     PlanDev plan, int64_t cap, SelMetric metric, int32_t* sel_idx,
+                     int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  const int ldS = (nb + 3) & ~3;
+  const size_t smem = sizeof(double) * (static_cast<size_t>(ldS) * (kGroup ? 1 + kWarps : 1)) +
+                      sizeof(int) * kWarps * 256;
+  auto kern = select_p_kernel<kGroup>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t NH = kGroup ? static_cast<int64_t>(B) * Hkv : static_cast<int64_t>(B) * Hq;
+  const int64_t grid = NH * ((nb + kWarps - 1) / kWarps);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kSelThreads, smem, st>>>(p, vnorm, B, Hq, Hkv, nb, ldS,
+                                                             plan, cap, metric, sel_idx, sel_cnt,
+                                                             m_out);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_select_p(const float* p, const float* vnorm, int B, int Hq, int Hkv, int nb,
+                            PlanDev plan, int64_t cap, SelMetric metric, int32_t* sel_idx,
+                            int32_t* sel_cnt, float* m_out, cudaStream_t st) {
+  if (B * Hq == 0 || nb == 0) return cudaSuccess;
+  if (metric.group && Hq != Hkv)
+    return launch_p<true>(p, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt, m_out,
+                          st);
+  return launch_p<false>(p, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx, sel_cnt, m_out,
+                         st);
+}
 
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,

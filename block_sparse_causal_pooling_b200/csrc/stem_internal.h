@@ -37,6 +37,23 @@ cudaError_t launch_select(const float* qbar, const float* kbar, const float* vno
                           SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
                           cudaStream_t st);
 
+// Block probabilities by anti-diagonal sampling (antidiag_sm100.cu), bf16 inputs, D 64 or 128,
+// stride | block, stride | S, block/stride a power of two <= 32. p: [B*Hq][nb*(nb+1)/2] rows of
+// p_ij (j <= i); scratch: antidiag_scratch_floats() floats; status as for the attention.
+constexpr int kAdSlots = 148;  // most CTAs the kernel runs (one scratch slot each)
+cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv, int S, int D,
+                            int block, int stride, float* p, float* scratch, int32_t* status,
+                            cudaStream_t st);
+int64_t antidiag_units(int B, int Hq, int S, int stride);
+size_t antidiag_scratch_floats(int B, int Hq, int S, int block, int stride);
+
+// Top-k selection from block probabilities p (select.cu): ranks ln p_ij + ln n_j (product) or
+// ln p_ij + beta * e_j (additive), per query head or summed over a kv-head group like
+// launch_select.
+cudaError_t launch_select_p(const float* p, const float* vnorm, int B, int Hq, int Hkv, int nb,
+                            PlanDev plan, int64_t cap, SelMetric metric, int32_t* sel_idx,
+                            int32_t* sel_cnt, float* m_out, cudaStream_t st);
+
 // Block-sparse attention, bfloat16 inputs on the tensor cores (attn_sm100.cu; block 64 falls to
 // the mma.sync kernel of attn_bf16.cu). `sched` is workspace of pairs_bytes() for the head-pair
 // step schedule (pairs.cu).

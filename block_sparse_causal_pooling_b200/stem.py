@@ -35,6 +35,8 @@ STEM_VSUM_MEAN = 0
 STEM_VSUM_MAX = 1
 STEM_SHARE_HEAD = 0
 STEM_SHARE_GROUP = 1
+STEM_SCORE_POOLED = 0
+STEM_SCORE_ANTIDIAG = 1
 
 
 class StemError(RuntimeError):
@@ -49,16 +51,18 @@ class stem_method_t(ctypes.Structure):
         ("k_start", ctypes.c_float), ("mu", ctypes.c_float), ("k_min", ctypes.c_int32),
         ("metric", ctypes.c_int32), ("beta", ctypes.c_float), ("clamp", ctypes.c_int32),
         ("vsum", ctypes.c_int32), ("share", ctypes.c_int32),
+        ("score", ctypes.c_int32), ("stride", ctypes.c_int32),
     ]
 
 
 def make_method(schedule: str = "exp", rho_min: float = 1.0, tau: float = 1.0,
                 k_start: float = 1.0, mu: float = 1.0, k_min: int = 1, metric: str = "product",
                 beta: float = 0.0, clamp: bool = True, vsum: str = "mean",
-                share: str = "head") -> stem_method_t:
+                share: str = "head", score: str = "pooled", stride: int = 16) -> stem_method_t:
     """Method parameters (stem_method_t): schedule "exp" (rho_min, tau) or "linear" (k_start,
     mu); metric "product" or "additive" (beta, clamp); vsum "mean" or "max"; share "head" or
-    "group" (one selection per kv-head group)."""
+    "group" (one selection per kv-head group); score "pooled" or "antidiag" (block
+    probabilities by anti-diagonal sampling with groups of `stride` tokens)."""
     m = stem_method_t()
     m.schedule = {"exp": STEM_SCHED_EXP, "linear": STEM_SCHED_LINEAR}[schedule]
     m.rho_min, m.tau, m.k_start, m.mu, m.k_min = rho_min, tau, k_start, mu, k_min
@@ -66,6 +70,8 @@ def make_method(schedule: str = "exp", rho_min: float = 1.0, tau: float = 1.0,
     m.beta, m.clamp = beta, int(bool(clamp))
     m.vsum = {"mean": STEM_VSUM_MEAN, "max": STEM_VSUM_MAX}[vsum]
     m.share = {"head": STEM_SHARE_HEAD, "group": STEM_SHARE_GROUP}[share]
+    m.score = {"pooled": STEM_SCORE_POOLED, "antidiag": STEM_SCORE_ANTIDIAG}[score]
+    m.stride = stride
     return m
 
 
@@ -126,6 +132,10 @@ def _load() -> ctypes.CDLL:
         "stem_prefill_varlen": (I, [ctypes.POINTER(stem_varlen_args_t), P]),
         "stem_varlen_workspace_size": (Z, [I, ctypes.POINTER(ctypes.c_int32), I, I, I, I]),
         "stem_varlen_sel_capacity": (ctypes.c_int64, [I, ctypes.POINTER(ctypes.c_int32), I, M]),
+        "stem_workspace_size_m": (Z, [I, I, I, I, I, I, M]),
+        "stem_antidiag_m": (I, [P, P, I, I, I, I, I, I, I, M, P, P, Z, P, P]),
+        "stem_select_p_m": (I, [P, P, I, I, I, I, M, P, P, P, P, Z, P]),
+        "stem_varlen_workspace_size_m": (Z, [I, ctypes.POINTER(ctypes.c_int32), I, I, I, I, M]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -142,7 +152,8 @@ EXPORTED = ("stem_prefill", "stem_prefill_ex", "stem_prefill_host", "stem_budget
             "stem_select", "stem_sparse_attn", "stem_budget_m", "stem_sel_capacity_m",
             "stem_pool_m", "stem_select_m", "stem_sparse_attn_m", "stem_prefill_varlen",
             "stem_varlen_workspace_size", "stem_varlen_sel_capacity", "stem_select_static",
-            "stem_test_withhold_q")
+            "stem_test_withhold_q", "stem_workspace_size_m", "stem_antidiag_m", "stem_select_p_m",
+            "stem_varlen_workspace_size_m")
 
 
 def lib() -> ctypes.CDLL:
@@ -205,7 +216,10 @@ def stem_budget_m(nb: int, method: stem_method_t):
     return k[:nb].clone(), off
 
 
-def stem_workspace_size(B: int, Hq: int, Hkv: int, S: int, D: int, block: int) -> int:
+def stem_workspace_size(B: int, Hq: int, Hkv: int, S: int, D: int, block: int,
+                        method=None) -> int:
+    if method is not None:
+        return int(_lib.stem_workspace_size_m(B, Hq, Hkv, S, D, block, ctypes.byref(method)))
     return int(_lib.stem_workspace_size(B, Hq, Hkv, S, D, block))
 
 
@@ -229,9 +243,9 @@ def alloc_outputs(q: torch.Tensor, k: torch.Tensor, block: int, rho_min: float, 
     return out, sel_idx, sel_cnt
 
 
-def alloc_workspace(q: torch.Tensor, k: torch.Tensor, block: int) -> torch.Tensor:
+def alloc_workspace(q: torch.Tensor, k: torch.Tensor, block: int, method=None) -> torch.Tensor:
     B, Hq, Hkv, S, D = _shape(q, k)
-    n = stem_workspace_size(B, Hq, Hkv, S, D, block)
+    n = stem_workspace_size(B, Hq, Hkv, S, D, block, method)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
 
 
@@ -268,7 +282,7 @@ def stem_prefill_ex(q, k, v, block, rho_min, tau, k_min, out=None, sel_idx=None,
     if out is None or sel_idx is None or sel_cnt is None:
         out, sel_idx, sel_cnt = alloc_outputs(q, k, block, rho_min, tau, k_min, method)
     if workspace is None:
-        workspace = alloc_workspace(q, k, block)
+        workspace = alloc_workspace(q, k, block, method)
     a = make_args(q, k, v, block, rho_min, tau, k_min, out, sel_idx, sel_cnt, workspace, status,
                   events, method)
     _check(_lib.stem_prefill_ex(ctypes.byref(a), _stream(stream)), "stem_prefill_ex")
@@ -363,6 +377,46 @@ def stem_sparse_attn(q, k, v, block, rho_min, tau, k_min, sel_idx, sel_cnt, out=
     return out
 
 
+def stem_antidiag(q, k, block, method, p=None, workspace=None, status=None, stream=None):
+    """Block probabilities by anti-diagonal sampling (bf16 device tensors; groups of
+    method.stride tokens). Returns p [B, Hq, nb*(nb+1)/2] float32, row i at i*(i+1)/2."""
+    B, Hq, Hkv, S, D = _shape(q, k)
+    nb = -(-S // block)
+    if p is None:
+        p = torch.empty((B, Hq, max(nb * (nb + 1) // 2, 1)), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        m = stem_method_t.from_buffer_copy(method)
+        m.score = STEM_SCORE_ANTIDIAG
+        workspace = alloc_workspace(q, k, block, m)
+    _check(_lib.stem_antidiag_m(q.data_ptr(), k.data_ptr(), _dtype_code(q), B, Hq, Hkv, S, D,
+                                block, ctypes.byref(method), p.data_ptr(), workspace.data_ptr(),
+                                workspace.numel(), _ptr(status), _stream(stream)),
+           "stem_antidiag_m")
+    return p
+
+
+def stem_select_p(p, vnorm, Hq, method, with_metric=False, workspace=None, sel_idx=None,
+                  sel_cnt=None, stream=None):
+    """CSR selection from block probabilities p [B, Hq, T] and V magnitudes vnorm [B, Hkv, nb]
+    (float32 device tensors). Returns (sel_idx, sel_cnt, m or None)."""
+    B, Hkv, nb = vnorm.shape
+    dev = p.device
+    cap = stem_sel_capacity(nb, 1.0, 1.0, 1, method)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, Hq, max(cap, 1)), dtype=torch.int32, device=dev)
+        sel_cnt = torch.empty((B, Hq, max(nb, 1)), dtype=torch.int32, device=dev)
+    m = (torch.empty((B, Hq, nb * (nb + 1) // 2), dtype=torch.float32, device=dev)
+         if with_metric else None)
+    if workspace is None:
+        workspace = torch.empty(max(stem_workspace_size(B, Hq, Hkv, nb * 64, 64, 64), 256),
+                                dtype=torch.uint8, device=dev)
+    _check(_lib.stem_select_p_m(p.data_ptr(), vnorm.data_ptr(), B, Hq, Hkv, nb,
+                                ctypes.byref(method), sel_idx.data_ptr(), sel_cnt.data_ptr(),
+                                _ptr(m), workspace.data_ptr(), workspace.numel(),
+                                _stream(stream)), "stem_select_p_m")
+    return sel_idx, sel_cnt, m
+
+
 def stem_select_static(qbar, kbar, vnorm, rho_min, tau, k_min, sel_idx=None, sel_cnt=None,
                        stream=None):
     """stem_select without a workspace or any device allocation by the library: its scratch
@@ -415,7 +469,8 @@ def stem_prefill_varlen(q, k, v, cu_seqlens, Hq, Hkv, D, block, method, out=None
         sel_idx = torch.empty(max(Hq * cap, 1), dtype=torch.int32, device=dev)
         sel_cnt = torch.empty(max(Hq * nbt, 1), dtype=torch.int32, device=dev)
     if workspace is None:
-        nbytes = int(_lib.stem_varlen_workspace_size(n, arr, Hq, Hkv, D, block))
+        nbytes = int(_lib.stem_varlen_workspace_size_m(n, arr, Hq, Hkv, D, block,
+                                                       ctypes.byref(method)))
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
     a = stem_varlen_args_t()
     a.q, a.k, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()

@@ -74,6 +74,8 @@ extern "C" {
 #define STEM_VSUM_MAX 1        /* n_j = largest V-row L2 norm of the block */
 #define STEM_SHARE_HEAD 0      /* one selection per query head (the default) */
 #define STEM_SHARE_GROUP 1     /* one selection per kv-head group, shared by its query heads */
+#define STEM_SCORE_POOLED 0    /* block scores from mean-pooled Q and K (the default) */
+#define STEM_SCORE_ANTIDIAG 1  /* block probabilities by anti-diagonal sampling */
 
 /*
  * Method parameters: budget schedule, block metric and V summary.
@@ -93,7 +95,23 @@ extern "C" {
  *          ranked in log space; additive: sum_h s_hij + G * beta * e_j) and written to each
  *          head's CSR row. The pages are silent on GQA; this is an alternative reading. With
  *          share = GROUP and G > 1, nb beyond 1024 returns STEM_ERR_UNSUPPORTED.
- * Fields the chosen schedule and metric do not use are ignored.
+ *   score: STEM_SCORE_POOLED (s_ij from the pooled Q and K above), or STEM_SCORE_ANTIDIAG: the
+ *          block probability p_ij comes from anti-diagonal sampling ([fr] 2.C step 1: block
+ *          metrics "with anti-diagonal sampling"; the pages give no formula, this is the
+ *          reading used). Tokens form groups of `stride` consecutive tokens; query group u and
+ *          key group w are scored by the mean of the anti-diagonal samples of their
+ *          stride x stride logit sub-tile,
+ *            a_uw = (1/stride) sum_t Q[u*stride+t] . K[w*stride+stride-1-t] / sqrt(D),
+ *          each query group takes a softmax over w <= u, and p_ij is the mass the query groups
+ *          of block i put on the key groups of block j, averaged over those query groups.
+ *          ln p_ij then takes the place of s_ij - logsumexp_j s_ij in the metric (product:
+ *          rank by ln p_ij + ln n_j; additive: ln p_ij + beta * e_j; group share: the summed
+ *          metric as above). Requires bfloat16 inputs (else STEM_ERR_UNSUPPORTED), a power-of-two
+ *          stride with block % stride == 0, block / stride <= 32 and S % stride == 0 (else
+ *          STEM_ERR_ARG). The sampled products run on the tensor cores (bf16 in, fp32
+ *          accumulation); it costs about 1/stride of a dense causal Q K^T.
+ * Fields the chosen schedule and metric do not use are ignored. Zero-initialise the struct
+ * (score 0 = pooled) before setting fields.
  */
 typedef struct stem_method {
   int32_t schedule;
@@ -107,6 +125,8 @@ typedef struct stem_method {
   int32_t clamp;
   int32_t vsum;
   int32_t share;
+  int32_t score;
+  int32_t stride; /* STEM_SCORE_ANTIDIAG only */
 } stem_method_t;
 
 /* Largest number of blocks per sequence (the selection kernel keeps one score row per
@@ -253,6 +273,35 @@ int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, i
                        const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
                        void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
+/* Workspace bytes stem_prefill_ex needs for this shape and method (with STEM_SCORE_ANTIDIAG
+ * it also holds the block probabilities and the estimator's per-CTA scratch, about
+ * 148 * 512 * ceil(S/block) bytes). 0 for an invalid or empty request. Host only. */
+size_t stem_workspace_size_m(int B, int Hq, int Hkv, int S, int D, int block,
+                             const stem_method_t* m);
+
+/*
+ * Block probabilities by anti-diagonal sampling (score STEM_SCORE_ANTIDIAG of stem_method_t;
+ * [fr] 2.C step 1). Reads bfloat16 q [B,Hq,S,D] and k [B,Hkv,S,D] (device, 16-byte aligned)
+ * and writes p (device float32 [B,Hq,nb*(nb+1)/2], row i at offset i*(i+1)/2, p_ij for j <= i;
+ * each row sums to 1 up to rounding). m->stride must satisfy the stem_method_t rules (m->score
+ * is not read). workspace: stem_workspace_size_m bytes for a method with this stride; status
+ * as in stem_args_t.
+ */
+int stem_antidiag_m(const void* q, const void* k, int dtype, int B, int Hq, int Hkv, int S, int D,
+                    int block, const stem_method_t* m, float* p, void* workspace,
+                    size_t workspace_bytes, int32_t* status, void* stream);
+
+/*
+ * Variable-k selection from block probabilities p (layout of stem_antidiag_m) and the V
+ * magnitudes vnorm [B,Hkv,nb] (layout of stem_pool_m): the metric of m (product, additive,
+ * per head or group-shared, see stem_method_t score) ranked in double, ties to the lower block
+ * index. m_out as in stem_select_m: m_ij = p_ij * n_j (product) or M_ij = ln p_ij + beta * e_j
+ * (additive), the group's summed metric under group share. workspace: as for stem_select_m.
+ */
+int stem_select_p_m(const float* p, const float* vnorm, int B, int Hq, int Hkv, int nb,
+                    const stem_method_t* m, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * Variable-length batches. nseq sequences of lengths S_s = cu_seqlens[s+1] - cu_seqlens[s]
  * (cu_seqlens: host int32[nseq+1], cu_seqlens[0] = 0, non-decreasing), packed back to back, each
@@ -284,6 +333,9 @@ int stem_prefill_varlen(const stem_varlen_args_t* a, void* stream);
 /* Workspace bytes for these sequences (the largest sequence's), 0 on invalid input. Host only. */
 size_t stem_varlen_workspace_size(int nseq, const int32_t* cu_seqlens, int Hq, int Hkv, int D,
                                   int block);
+/* The same for a method (needed with STEM_SCORE_ANTIDIAG, whose workspace is larger). */
+size_t stem_varlen_workspace_size_m(int nseq, const int32_t* cu_seqlens, int Hq, int Hkv, int D,
+                                    int block, const stem_method_t* m);
 /* Total CSR entries per query head: sum over the sequences of cap_s; negative STEM_ERR_* on
  * invalid input. Host only. */
 int64_t stem_varlen_sel_capacity(int nseq, const int32_t* cu_seqlens, int block,

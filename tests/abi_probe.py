@@ -153,4 +153,52 @@ res.update({
     "attn_m_bad_block": L.stem_sparse_attn_m(FAKE, FAKE, FAKE, 0, 1, 4, 2, 1000, 128, 96, M(GOOD),
                                           FAKE, FAKE, FAKE, FAKE, 1 << 20, None, None),
 })
+
+# anti-diagonal scoring: stride rules and the estimator's entry points
+AD = S.make_method("exp", rho_min=0.25, tau=4.0, k_min=2, score="antidiag", stride=16)
+def ad(**kw):
+    m = S.stem_method_t.from_buffer_copy(AD)
+    for key, val in kw.items():
+        setattr(m, key, val)
+    return m
+
+
+res.update({
+    "ad_stride_not_pow2": ex(method=ctypes.pointer(ad(stride=12))),
+    "ad_stride_zero": ex(method=ctypes.pointer(ad(stride=0))),
+    "ad_stride_above_block": ex(method=ctypes.pointer(ad(stride=256))),
+    "ad_too_many_groups": ex(method=ctypes.pointer(ad(stride=2))),
+    "ad_S_not_multiple": ex(S=1000, method=ctypes.pointer(ad())),
+    "ad_f32": ex(dtype=1, method=ctypes.pointer(ad())),
+    "ad_bad_score": ex(method=ctypes.pointer(ad(score=5))),
+    # the pooled method's workspace lacks the estimator's regions
+    "ad_small_workspace": ex(workspace_bytes=L.stem_workspace_size(1, 4, 2, 1024, 128, 128),
+                             method=ctypes.pointer(ad())),
+    "ad_host_bad_stride": L.stem_prefill_host(ctypes.byref(base(method=ctypes.pointer(ad(stride=3))))),
+    "ad_varlen_bad_S": varlen([0, 1000], method=ad()),
+    "antidiag_m_null_method": L.stem_antidiag_m(FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, None,
+                                                FAKE, FAKE, 1 << 30, None, None),
+    "antidiag_m_bad_stride": L.stem_antidiag_m(FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128,
+                                               M(ad(stride=48)), FAKE, FAKE, 1 << 30, None, None),
+    "antidiag_m_f32": L.stem_antidiag_m(FAKE, FAKE, 1, 1, 4, 2, 1024, 128, 128, M(AD), FAKE,
+                                        FAKE, 1 << 30, None, None),
+    "antidiag_m_null_p": L.stem_antidiag_m(FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128, M(AD), None,
+                                           FAKE, 1 << 30, None, None),
+    "antidiag_m_small_workspace": L.stem_antidiag_m(FAKE, FAKE, 0, 1, 4, 2, 1024, 128, 128,
+                                                    M(AD), FAKE, FAKE, 4096, None, None),
+    "antidiag_m_q_misaligned": L.stem_antidiag_m(FAKE + 8, FAKE, 0, 1, 4, 2, 1024, 128, 128,
+                                                 M(AD), FAKE, FAKE, 1 << 30, None, None),
+    "antidiag_m_empty": L.stem_antidiag_m(None, None, 0, 1, 4, 2, 0, 128, 128, M(AD), None,
+                                          None, 0, None, None),
+    "select_p_null_method": L.stem_select_p_m(FAKE, FAKE, 1, 4, 2, 8, None, FAKE, FAKE, None,
+                                              FAKE, 1 << 20, None),
+    "select_p_bad_mu": L.stem_select_p_m(FAKE, FAKE, 1, 4, 2, 8, M(BAD_MU), FAKE, FAKE, None,
+                                         FAKE, 1 << 20, None),
+    "select_p_no_workspace": L.stem_select_p_m(FAKE, FAKE, 1, 4, 2, 8, M(AD), FAKE, FAKE, None,
+                                               None, 0, None),
+    "select_p_nb_too_large": L.stem_select_p_m(FAKE, FAKE, 1, 4, 2, S.STEM_MAX_NB + 1, M(AD),
+                                               FAKE, FAKE, None, FAKE, 1 << 30, None),
+    "select_p_null_vnorm": L.stem_select_p_m(FAKE, None, 1, 4, 2, 8, M(AD), FAKE, FAKE, None,
+                                             FAKE, 1 << 20, None),
+})
 print(json.dumps(res))

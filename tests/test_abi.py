@@ -141,6 +141,18 @@ def test_workspace_size_layout():
         S.stem_workspace_size(B, Hq, Hkv, 1024, D, block) > 0
     assert S.stem_workspace_size(B, Hq, Hkv, 1000, 96, block) == 0  # unsupported D
     assert S.stem_workspace_size(0, Hq, Hkv, Sq, D, block) == 0  # empty
+    # anti-diagonal scoring adds p (packed rows) and the estimator's per-CTA scratch:
+    # min(units, 148) slots of (nb + ceil((S/stride)/256)) * 128 floats
+    ad = S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8, score="antidiag", stride=16)
+    assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad.__class__.from_buffer_copy(
+        S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8))) == n
+    na = S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad)
+    p_bytes = 4 * B * Hq * nb * (nb + 1) // 2
+    nred = Sq // 16
+    scratch = 4 * min(B * Hq * (nred // 128), 148) * (nb + nred // 256) * 128
+    assert n + p_bytes + scratch <= na < n + p_bytes + scratch + 1024
+    ad.stride = 24
+    assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad) == 0
 
 
 def test_strerror_covers_every_code():
@@ -172,5 +184,12 @@ def test_argument_validation_rejects_before_any_device_work():
         "group_nb_too_large": S.STEM_ERR_UNSUPPORTED,
         "empty_B": S.STEM_OK,
         "empty_S": S.STEM_OK,
+        "ad_f32": S.STEM_ERR_UNSUPPORTED,
+        "ad_small_workspace": S.STEM_ERR_WORKSPACE,
+        "antidiag_m_f32": S.STEM_ERR_UNSUPPORTED,
+        "antidiag_m_small_workspace": S.STEM_ERR_WORKSPACE,
+        "antidiag_m_empty": S.STEM_OK,
+        "select_p_no_workspace": S.STEM_ERR_WORKSPACE,
+        "select_p_nb_too_large": S.STEM_ERR_UNSUPPORTED,
     })
     assert res == want
