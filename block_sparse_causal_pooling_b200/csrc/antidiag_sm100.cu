@@ -25,12 +25,12 @@
 //   warp 1    allocates the 512 TMEM columns; lane 0 issues tcgen05.mma (M 128, N 256, K 16)
 //             into one of two 256-column fp32 accumulators, so the epilogue of one key tile
 //             overlaps the products of the next.
-//   warps 2-5 epilogue, one query group (TMEM lane) per thread: online softmax over the key
-//             tiles in base 2 (running max m, running sum l); per key block the sum of
-//             exp2(a - m) over its key groups goes to a per-CTA scratch row together with the
-//             m it was taken against. After the unit's last tile each value is rescaled to the
-//             final m and divided by l, the block's query groups are summed with shuffles and
-//             p_ij is written.
+//   warps 2-5 epilogue, one query group (TMEM lane) per thread: online softmax over the
+//             32-column chunks of each key tile in base 2 (running max m, running sum l), one
+//             TMEM read per chunk; per key block the sum of exp2(a - m) over its key groups goes
+//             to a per-CTA scratch row, and each chunk's m (its snapshot) beside it. After the
+//             unit's last tile each value is rescaled to the final m and divided by l, the
+//             block's query groups are summed with shuffles and p_ij is written.
 // Every mbarrier wait is bounded by the global nanosecond timer; on expiry the CTA records
 // STEM_ERR_TIMEOUT, every role leaves its loop, issued products and copies are drained (bounded)
 // and TMEM is freed.
@@ -76,7 +76,7 @@ struct AdParams {
   int64_t units;        // B * Hq * nqt
   float scale_log2;     // log2(e) / (stride * sqrt(D))
   float* p;             // [B*Hq][nb*(nb+1)/2]
-  float* scratch;       // [gridDim.x][nb*128 + nkt_max*128]
+  float* scratch;       // [gridDim.x][nb*128 + 8*nkt_max*128]
   int64_t scratch_per_cta;
   int32_t* status;
 };
@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)));
-      const uint64_t pol = policy_evict_last();
+      // a unit re-reads its Q' tile for every key tile: keep it; K' tiles pass through
+      const uint64_t pol_q = policy_evict_last(), pol_k = policy_evict_normal();
       int64_t f = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x) {
@@ -168,9 +169,9 @@ __global__ void __launch_bounds__(kAThreads, 1)
             mbar_expect_tx(&bars->full[s], kStageBytes);
             const int chunk = ks / P.kparts, part = ks % P.kparts;
             unsigned char* st = smem + s * kStageBytes;
-            tma_load_3d(st, &tm_q, ks * 64, u.qt * kAM, u.bh, &bars->full[s], pol);
+            tma_load_3d(st, &tm_q, ks * 64, u.qt * kAM, u.bh, &bars->full[s], pol_q);
             tma_load_3d(st + kQBox, &tm_k, (P.stride - 1 - chunk) * P.D + part * 64, kt * kAN,
-                        kvh, &bars->full[s], pol);
+                        kvh, &bars->full[s], pol_k);
             ++f;
           }
         }
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t tri = static_cast<int64_t>(P.nb) * (P.nb + 1) / 2;
     float* esc = P.scratch + static_cast<int64_t>(blockIdx.x) * P.scratch_per_cta;  // [nb][128]
-    float* msc = esc + static_cast<int64_t>(P.nb) * kAM;                            // [nkt][128]
+    float* msc = esc + static_cast<int64_t>(P.nb) * kAM;  // [nkt * 8 chunks][128] snapshots
     const int R = P.R;
     int64_t tiles = 0;
     bool ok = true;
@@ -244,49 +245,51 @@ __global__ void __launch_bounds__(kAThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t taddr = tmem + lane_addr + buf * kAN;
-        const int lim = u - kt * kAN;  // columns c <= lim are visible (w <= u)
-        uint32_t r[32];
-        float tmax = -INFINITY;
+        // One pass per 32-column chunk: the exact running max over the columns seen so far,
+        // exp2 against it, sums by tree. Each chunk's sums are stored with the max they were
+        // taken against (its snapshot), so no column is read twice.
 #pragma unroll 1
         for (int ch = 0; ch < kAN / 32; ++ch) {
+          uint32_t r[32];
           TC_LD32(taddr + ch * 32, r);
           tc_wait_ld();
+          const int lim = u - kt * kAN - ch * 32;  // columns c <= lim are visible (w <= u)
+          float x[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (ch * 32 + c <= lim) tmax = fmaxf(tmax, __uint_as_float(r[c]));
-        }
-        const float m_new = fmaxf(m_run, tmax * P.scale_log2);
-        l_run *= ex2(m_run - m_new);  // m_run = -inf on the first tile: l_run is 0 either way
-        const int jbase = kt * (kAN / R);  // first key block of the tile
-#pragma unroll 1
-        for (int ch = 0; ch < kAN / 32; ++ch) {
-          TC_LD32(taddr + ch * 32, r);
-          tc_wait_ld();
+          for (int c = 0; c < 32; ++c) x[c] = c <= lim ? __uint_as_float(r[c]) : -INFINITY;
+          float mx[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) mx[c] = fmaxf(x[c], x[c + 16]);
+#pragma unroll
+          for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+            for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+          // every row sees column 0 of its first chunk, so m_new is finite from there on
+          const float m_new = fmaxf(m_run, mx[0] * P.scale_log2);
+          l_run *= ex2(m_run - m_new);  // m_run = -inf before the first chunk: l_run stays 0
           float e[32];
-          float part = 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            e[c] = ch * 32 + c <= lim ? ex2(fmaf(__uint_as_float(r[c]), P.scale_log2, -m_new))
-                                      : 0.f;
-            part += e[c];
-          }
-          l_run += part;
-          // segmented sums over the R consecutive columns of each key block (R | 32)
+          for (int c = 0; c < 32; ++c) e[c] = ex2(fmaf(x[c], P.scale_log2, -m_new));  // -inf -> 0
+          // tree sums: at level R the partial sums are the per-key-block sums (R | 32)
+          const int jb = (kt * kAN + ch * 32) / R;  // key block of column 0 of the chunk
 #pragma unroll
-          for (int lv = 1; lv < 32; lv <<= 1) {
-            if (lv < R) {
+          for (int lv = 1; lv <= 32; lv <<= 1) {
+            if (lv == R) {
+#pragma unroll
+              for (int c = 0; c < 32; c += lv) {
+                const int j = jb + c / lv;  // the last tile may reach past block nb-1
+                if (j < P.nb) esc[static_cast<int64_t>(j) * kAM + row] = e[c];
+              }
+            }
+            if (lv < 32) {
 #pragma unroll
               for (int c = 0; c < 32; c += 2 * lv) e[c] += e[c + lv];
             }
           }
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int j = jbase + (ch * 32 + c) / R;  // the last tile may reach past block nb-1
-            if ((c & (R - 1)) == 0 && j < P.nb) esc[static_cast<int64_t>(j) * kAM + row] = e[c];
-          }
+          l_run += e[0];
+          msc[(kt * (kAN / 32) + ch) * kAM + row] = m_new;
+          m_run = m_new;
         }
-        msc[kt * kAM + row] = m_new;
-        m_run = m_new;
         tc_fence_before();
         mbar_arrive(&bars->acc_empty[buf]);
         ++tiles;
@@ -299,14 +302,24 @@ __global__ void __launch_bounds__(kAThreads, 1)
       const float inv_l = 1.f / l_run;
       const int i_hi = min(P.nb - 1, (un.qt * kAM + quarter * 32 + 31) / R);  // warp's last block
       float* prow = P.p + static_cast<int64_t>(un.bh) * tri + static_cast<int64_t>(i) * (i + 1) / 2;
-      for (int j = 0; j <= i_hi; ++j) {
-        float val = 0.f;
-        if (valid && j <= i) {
-          const int ktj = j * R / kAN;
-          val = esc[static_cast<int64_t>(j) * kAM + row] * ex2(msc[ktj * kAM + row] - m_run) * inv_l;
+      const float inv_n = 1.f / static_cast<float>(n_i);
+      // eight key blocks per step, their loads issued together; every j <= i_hi lies in a tile
+      // this unit processed, so the scratch entries read here are this unit's
+      for (int j0 = 0; j0 <= i_hi; j0 += 8) {
+        float ev[8], sv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int j = min(j0 + t, i_hi);
+          ev[t] = esc[static_cast<int64_t>(j) * kAM + row];
+          sv[t] = msc[((j * R) >> 5) * kAM + row];  // snapshot of the chunk holding block j
         }
-        for (int o = 1; o < R; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
-        if (valid && j <= i && (lane & (R - 1)) == 0) prow[j] = val / static_cast<float>(n_i);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int j = j0 + t;
+          float val = valid && j <= i ? ev[t] * ex2(sv[t] - m_run) * inv_l : 0.f;
+          for (int o = 1; o < R; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
+          if (valid && j <= i && (lane & (R - 1)) == 0) prow[j] = val * inv_n;
+        }
       }
     }
   }
@@ -350,7 +363,7 @@ size_t antidiag_scratch_floats(int B, int Hq, int S, int block, int stride) {
   const int64_t nred = S / stride;
   const int64_t nkt = (nred + kAN - 1) / kAN;
   const int64_t slots = std::min<int64_t>(antidiag_units(B, Hq, S, stride), kAdSlots);
-  return static_cast<size_t>(slots * (nb + nkt) * kAM);
+  return static_cast<size_t>(slots * (nb + (kAN / 32) * nkt) * kAM);
 }
 
 cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv, int S, int D,
@@ -375,7 +388,7 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   P.scale_log2 = static_cast<float>(1.4426950408889634 / (stride * std::sqrt(static_cast<double>(D))));
   P.p = p;
   P.scratch = scratch;
-  P.scratch_per_cta = static_cast<int64_t>(P.nb + (P.nred + kAN - 1) / kAN) * kAM;
+  P.scratch_per_cta = static_cast<int64_t>(P.nb + (kAN / 32) * ((P.nred + kAN - 1) / kAN)) * kAM;
   P.status = status;
   CUtensorMap tq, tk;
   if (!make_group_map(&tq, q, static_cast<uint64_t>(B) * Hq, S, D, stride, kAM) ||
