@@ -18,19 +18,21 @@
 // the inputs: no copy is made. The reversal costs nothing: the k-step that reads chunk t of Q'
 // reads chunk sigma-1-t of K', which is only a different TMA box coordinate.
 //
-// Persistent kernel, one CTA per SM, 6 warps. Work unit: (b, h, 128 consecutive query groups).
+// Persistent kernel, one CTA per SM, 10 warps. Work unit: (b, h, 128 consecutive query groups).
 //   warp 0    TMA producer: for every key tile (256 key groups, up to the unit's causal end) and
 //             every k-step (64 of the sigma*D columns), the Q' box (128 x 64) and the K' box
 //             (256 x 64) into a 4-stage ring of 128B-swizzled shared-memory tiles.
 //   warp 1    allocates the 512 TMEM columns; lane 0 issues tcgen05.mma (M 128, N 256, K 16)
 //             into one of two 256-column fp32 accumulators, so the epilogue of one key tile
 //             overlaps the products of the next.
-//   warps 2-5 epilogue, one query group (TMEM lane) per thread: online softmax over the
+//   warps 2-5 tile epilogue, one query group (TMEM lane) per thread: online softmax over the
 //             32-column chunks of each key tile in base 2 (running max m, running sum l), one
 //             TMEM read per chunk; per key block the sum of exp2(a - m) over its key groups goes
-//             to a per-CTA scratch row, and each chunk's m (its snapshot) beside it. After the
-//             unit's last tile each value is rescaled to the final m and divided by l, the
-//             block's query groups are summed with shuffles and p_ij is written.
+//             to a scratch row, and each chunk's m (its snapshot) beside it. At the unit's end
+//             m and l go to shared memory and the unit's scratch slot is handed over.
+//   warps 6-9 fixup, while warps 2-5 work on the next unit (two scratch slots per CTA): each
+//             value is rescaled to its row's final m and divided by l, the block's query groups
+//             are summed with shuffles and p_ij is written.
 // Every mbarrier wait is bounded by the global nanosecond timer; on expiry the CTA records
 // STEM_ERR_TIMEOUT, every role leaves its loop, issued products and copies are drained (bounded)
 // and TMEM is freed.
@@ -53,8 +55,9 @@ using namespace sm100;
 constexpr int kAM = 128;              // query groups per tile (MMA M)
 constexpr int kAN = 256;              // key groups per tile (MMA N)
 constexpr int kStages = 4;            // shared-memory ring
-constexpr int kAThreads = 192;        // 6 warps
+constexpr int kAThreads = 320;        // 10 warps
 constexpr int kEpiThreads = 128;      // warps 2-5
+constexpr int kFixThreads = 128;      // warps 6-9
 constexpr uint32_t kQBox = kAM * 128;  // 128 rows x 64 bf16
 constexpr uint32_t kKBox = kAN * 128;  // 256 rows x 64 bf16
 constexpr uint32_t kStageBytes = kQBox + kKBox;
@@ -63,9 +66,11 @@ constexpr uint32_t kTmemCols = 512;
 struct __align__(8) ABars {
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t unit_done[2], fix_done[2];  // per scratch slot: tiles done -> fixup done
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
+  float ml[2][2][kAM];  // [slot][running max m, running sum l][query group of the tile]
 };
 
 struct AdParams {
@@ -76,8 +81,8 @@ struct AdParams {
   int64_t units;        // B * Hq * nqt
   float scale_log2;     // log2(e) / (stride * sqrt(D))
   float* p;             // [B*Hq][nb*(nb+1)/2]
-  float* scratch;       // [gridDim.x][nb*128 + 8*nkt_max*128]
-  int64_t scratch_per_cta;
+  float* scratch;       // [gridDim.x][2 slots][nb*128 + 8*nkt_max*128]
+  int64_t scratch_per_slot;
   int32_t* status;
 };
 
@@ -131,6 +136,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->acc_full[s], 1);
       mbar_init(&bars->acc_empty[s], kEpiThreads);
+      mbar_init(&bars->unit_done[s], kEpiThreads);
+      mbar_init(&bars->fix_done[s], kFixThreads);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -220,19 +227,24 @@ __global__ void __launch_bounds__(kAThreads, 1)
       tc_commit(&bars->drain);  // every issued product completes before TMEM is released
       drain_bar(&bars->drain, 0);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ tile epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const int64_t tri = static_cast<int64_t>(P.nb) * (P.nb + 1) / 2;
-    float* esc = P.scratch + static_cast<int64_t>(blockIdx.x) * P.scratch_per_cta;  // [nb][128]
-    float* msc = esc + static_cast<int64_t>(P.nb) * kAM;  // [nkt * 8 chunks][128] snapshots
     const int R = P.R;
-    int64_t tiles = 0;
+    int64_t tiles = 0, n = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x) {
+    for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x, ++n) {
       const AUnit un = ad_unit(t, P, BH);
+      const int slot = static_cast<int>(n & 1);
+      // the slot's previous unit (n - 2) must be through its fixup before it is overwritten
+      ok = __all_sync(0xffffffffu, ad_wait(&bars->fix_done[slot],
+                                           static_cast<uint32_t>(((n >> 1) & 1) ^ 1), bars,
+                                           P.status));
+      if (!ok) break;
+      float* esc = P.scratch + (2 * static_cast<int64_t>(blockIdx.x) + slot) * P.scratch_per_slot;
+      float* msc = esc + static_cast<int64_t>(P.nb) * kAM;  // [nkt * 8 chunks][128] snapshots
       const int u = un.qt * kAM + row;  // this thread's query group
       float m_run = -INFINITY, l_run = 0.f;
       for (int kt = 0; kt < un.nkt; ++kt) {
@@ -295,12 +307,37 @@ __global__ void __launch_bounds__(kAThreads, 1)
         ++tiles;
       }
       if (!ok) break;
-      // ---- the unit's block probabilities
+      bars->ml[slot][0][row] = m_run;
+      bars->ml[slot][1][row] = l_run;
+      mbar_arrive(&bars->unit_done[slot]);  // releases the slot's scratch and m, l
+    }
+  } else {
+    // ------------------------------------------------------------ fixup (warps 6-9)
+    // The unit's block probabilities from its scratch slot, while the other warps work on the
+    // next unit: each value is rescaled to its row's final m and divided by l, the block's
+    // query groups are summed with shuffles and p_ij is written.
+    const int fw = warp - 6;
+    const int row = fw * 32 + lane;
+    const int R = P.R;
+    const int64_t tri = static_cast<int64_t>(P.nb) * (P.nb + 1) / 2;
+    int64_t n = 0;
+    for (int64_t t = blockIdx.x; t < P.units; t += gridDim.x, ++n) {
+      const AUnit un = ad_unit(t, P, BH);
+      const int slot = static_cast<int>(n & 1);
+      if (!__all_sync(0xffffffffu, ad_wait(&bars->unit_done[slot],
+                                           static_cast<uint32_t>((n >> 1) & 1), bars,
+                                           P.status)))
+        break;
+      const float* esc =
+          P.scratch + (2 * static_cast<int64_t>(blockIdx.x) + slot) * P.scratch_per_slot;
+      const float* msc = esc + static_cast<int64_t>(P.nb) * kAM;
+      const float m_run = bars->ml[slot][0][row], l_run = bars->ml[slot][1][row];
+      const int u = un.qt * kAM + row;
       const bool valid = u < P.nred;
       const int i = u / R;                         // query block of this group
       const int n_i = min(R, P.nred - i * R);      // its query groups
       const float inv_l = 1.f / l_run;
-      const int i_hi = min(P.nb - 1, (un.qt * kAM + quarter * 32 + 31) / R);  // warp's last block
+      const int i_hi = min(P.nb - 1, (un.qt * kAM + fw * 32 + 31) / R);  // warp's last block
       float* prow = P.p + static_cast<int64_t>(un.bh) * tri + static_cast<int64_t>(i) * (i + 1) / 2;
       const float inv_n = 1.f / static_cast<float>(n_i);
       // eight key blocks per step, their loads issued together; every j <= i_hi lies in a tile
@@ -308,19 +345,20 @@ __global__ void __launch_bounds__(kAThreads, 1)
       for (int j0 = 0; j0 <= i_hi; j0 += 8) {
         float ev[8], sv[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int j = min(j0 + t, i_hi);
-          ev[t] = esc[static_cast<int64_t>(j) * kAM + row];
-          sv[t] = msc[((j * R) >> 5) * kAM + row];  // snapshot of the chunk holding block j
+        for (int q = 0; q < 8; ++q) {
+          const int j = min(j0 + q, i_hi);
+          ev[q] = esc[static_cast<int64_t>(j) * kAM + row];
+          sv[q] = msc[((j * R) >> 5) * kAM + row];  // snapshot of the chunk holding block j
         }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int j = j0 + t;
-          float val = valid && j <= i ? ev[t] * ex2(sv[t] - m_run) * inv_l : 0.f;
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + q;
+          float val = valid && j <= i ? ev[q] * ex2(sv[q] - m_run) * inv_l : 0.f;
           for (int o = 1; o < R; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
           if (valid && j <= i && (lane & (R - 1)) == 0) prow[j] = val * inv_n;
         }
       }
+      mbar_arrive(&bars->fix_done[slot]);  // the slot may be overwritten
     }
   }
 
@@ -363,7 +401,7 @@ size_t antidiag_scratch_floats(int B, int Hq, int S, int block, int stride) {
   const int64_t nred = S / stride;
   const int64_t nkt = (nred + kAN - 1) / kAN;
   const int64_t slots = std::min<int64_t>(antidiag_units(B, Hq, S, stride), kAdSlots);
-  return static_cast<size_t>(slots * (nb + (kAN / 32) * nkt) * kAM);
+  return static_cast<size_t>(slots * 2 * (nb + (kAN / 32) * nkt) * kAM);  // two slots per CTA
 }
 
 cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv, int S, int D,
@@ -388,7 +426,7 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   P.scale_log2 = static_cast<float>(1.4426950408889634 / (stride * std::sqrt(static_cast<double>(D))));
   P.p = p;
   P.scratch = scratch;
-  P.scratch_per_cta = static_cast<int64_t>(P.nb + (kAN / 32) * ((P.nred + kAN - 1) / kAN)) * kAM;
+  P.scratch_per_slot = static_cast<int64_t>(P.nb + (kAN / 32) * ((P.nred + kAN - 1) / kAN)) * kAM;
   P.status = status;
   CUtensorMap tq, tk;
   if (!make_group_map(&tq, q, static_cast<uint64_t>(B) * Hq, S, D, stride, kAM) ||

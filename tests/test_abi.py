@@ -142,14 +142,14 @@ def test_workspace_size_layout():
     assert S.stem_workspace_size(B, Hq, Hkv, 1000, 96, block) == 0  # unsupported D
     assert S.stem_workspace_size(0, Hq, Hkv, Sq, D, block) == 0  # empty
     # anti-diagonal scoring adds p (packed rows) and the estimator's per-CTA scratch:
-    # min(units, 148) slots of (nb + 8 * ceil((S/stride)/256)) * 128 floats
+    # min(units, 148) CTAs x 2 slots of (nb + 8 * ceil((S/stride)/256)) * 128 floats
     ad = S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8, score="antidiag", stride=16)
     assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad.__class__.from_buffer_copy(
         S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8))) == n
     na = S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad)
     p_bytes = 4 * B * Hq * nb * (nb + 1) // 2
     nred = Sq // 16
-    scratch = 4 * min(B * Hq * (nred // 128), 148) * (nb + 8 * (nred // 256)) * 128
+    scratch = 4 * min(B * Hq * (nred // 128), 148) * 2 * (nb + 8 * (nred // 256)) * 128
     assert n + p_bytes + scratch <= na < n + p_bytes + scratch + 1024
     ad.stride = 24
     assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad) == 0
