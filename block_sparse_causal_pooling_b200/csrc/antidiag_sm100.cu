@@ -18,7 +18,9 @@
 // the inputs: no copy is made. The reversal costs nothing: the k-step that reads chunk t of Q'
 // reads chunk sigma-1-t of K', which is only a different TMA box coordinate.
 //
-// Persistent kernel, one CTA per SM, 10 warps. Work unit: (b, h, 128 consecutive query groups).
+// Persistent kernel, one CTA per SM, 10 warps. Work unit: (b, h, 128 consecutive query groups),
+// claimed from a global counter in kv-head-major order (the units in flight share one kv head's
+// K', which stays in L2) and handed to the other roles through a ring in shared memory.
 //   warp 0    TMA producer: for every key tile (256 key groups, up to the unit's causal end) and
 //             every k-step (64 of the sigma*D columns), the Q' box (128 x 64) and the K' box
 //             (256 x 64) into a 4-stage ring of 128B-swizzled shared-memory tiles.
@@ -33,6 +35,8 @@
 //   warps 6-9 fixup, while warps 2-5 work on the next unit (two scratch slots per CTA): each
 //             value is rescaled to its row's final m and divided by l, the block's query groups
 //             are summed with shuffles and p_ij is written.
+// Q' tiles load with evict_last (a unit re-reads its Q' tile for every key tile); scratch and p
+// move with streaming loads and stores, so that they do not push Q' and K' out of L2.
 // Every mbarrier wait is bounded by the global nanosecond timer; on expiry the CTA records
 // STEM_ERR_TIMEOUT, every role leaves its loop, issued products and copies are drained (bounded)
 // and TMEM is freed.
@@ -62,12 +66,16 @@ constexpr uint32_t kQBox = kAM * 128;  // 128 rows x 64 bf16
 constexpr uint32_t kKBox = kAN * 128;  // 256 rows x 64 bf16
 constexpr uint32_t kStageBytes = kQBox + kKBox;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kUnitRing = 8;          // unit indices handed from the producer to the other roles
+constexpr int kUnitReaders = 1 + kEpiThreads + kFixThreads;  // MMA thread, warps 2-9
 
 struct __align__(8) ABars {
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t unit_done[2], fix_done[2];  // per scratch slot: tiles done -> fixup done
+  uint64_t uq_full[kUnitRing], uq_empty[kUnitRing];
   uint64_t drain;
+  int64_t uq[kUnitRing];  // unit index, or -1: no more units
   uint32_t tmem_base;
   volatile int abort;
   float ml[2][2][kAM];  // [slot][running max m, running sum l][query group of the tile]
@@ -81,6 +89,7 @@ struct AdParams {
   int64_t units;        // B * Hq * nqt
   float scale_log2;     // log2(e) / (stride * sqrt(D))
   float* p;             // [B*Hq][nb*(nb+1)/2]
+  unsigned long long* next_unit;  // work counter, 0 at launch
   float* scratch;       // [gridDim.x][2 slots][nb*128 + 8*nkt_max*128]
   int64_t scratch_per_slot;
   int32_t* status;
@@ -104,17 +113,36 @@ __device__ __forceinline__ bool ad_wait(uint64_t* b, uint32_t parity, ABars* bar
   return mbar_try(b, parity) || ad_wait_slow(b, parity, bars, status);
 }
 
-// Unit t -> (bh, qt): heaviest query tiles first (a tile's key range grows with qt).
+// Unit t -> (bh, qt). kv-head-major, so that the units in flight share one kv head's K' (which
+// then stays in L2); inside a kv head the heaviest query tiles first (a tile's key range grows
+// with qt), the G query heads of a tile next to each other. CTAs take units from a global
+// counter, so the order is the order of issue, not a fixed assignment.
 struct AUnit {
-  int bh, qt, nkt;
+  int bh, qt, nkt, kvh;
 };
-__device__ __forceinline__ AUnit ad_unit(int64_t t, const AdParams& P, int BH) {
+__device__ __forceinline__ AUnit ad_unit(int64_t t, const AdParams& P) {
+  const int G = P.Hq / P.Hkv;
+  const int64_t per_kv = static_cast<int64_t>(G) * P.nqt;
+  const int kvh = static_cast<int>(t / per_kv);  // b * Hkv + kv head
+  const int r = static_cast<int>(t % per_kv);
   AUnit u;
-  u.qt = P.nqt - 1 - static_cast<int>(t / BH);
-  u.bh = static_cast<int>(t % BH);
+  u.kvh = kvh;
+  u.qt = P.nqt - 1 - r / G;
+  u.bh = (kvh / P.Hkv) * P.Hq + (kvh % P.Hkv) * G + r % G;
   const int last = min(P.nred - 1, u.qt * kAM + kAM - 1);  // last query group of the tile
   u.nkt = last / kAN + 1;                                   // key tiles 0 .. (last / 256)
   return u;
+}
+
+// The n-th unit of this CTA from the ring (every reader calls this once per unit, in order).
+__device__ __forceinline__ bool ad_next_unit(ABars* bars, int64_t n, int32_t* status,
+                                             int64_t* t) {
+  const int q = static_cast<int>(n % kUnitRing);
+  if (!ad_wait(&bars->uq_full[q], static_cast<uint32_t>((n / kUnitRing) & 1), bars, status))
+    return false;
+  *t = bars->uq[q];
+  mbar_arrive(&bars->uq_empty[q]);
+  return true;
 }
 
 __global__ void __launch_bounds__(kAThreads, 1)
@@ -125,8 +153,6 @@ __global__ void __launch_bounds__(kAThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   ABars* bars = reinterpret_cast<ABars*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = static_cast<int>(P.units / P.nqt);
-  const int G = P.Hq / P.Hkv;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -138,6 +164,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
       mbar_init(&bars->acc_empty[s], kEpiThreads);
       mbar_init(&bars->unit_done[s], kEpiThreads);
       mbar_init(&bars->fix_done[s], kFixThreads);
+    }
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(&bars->uq_full[s], 1);
+      mbar_init(&bars->uq_empty[s], kUnitReaders);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -163,9 +193,19 @@ __global__ void __launch_bounds__(kAThreads, 1)
       const uint64_t pol_q = policy_evict_last(), pol_k = policy_evict_normal();
       int64_t f = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x) {
-        const AUnit u = ad_unit(t, P, BH);
-        const int kvh = (u.bh / P.Hq) * P.Hkv + (u.bh % P.Hq) / G;
+      for (int64_t n = 0; ok; ++n) {
+        // claim the next unit and publish it to the other roles (-1: none left)
+        int64_t t = static_cast<int64_t>(atomicAdd(P.next_unit, 1ull));
+        if (t >= P.units) t = -1;
+        const int q = static_cast<int>(n % kUnitRing);
+        if (!(ok = ad_wait(&bars->uq_empty[q], static_cast<uint32_t>(((n / kUnitRing) & 1) ^ 1),
+                           bars, P.status)))
+          break;
+        bars->uq[q] = t;
+        mbar_arrive(&bars->uq_full[q]);
+        if (t < 0) break;
+        const AUnit u = ad_unit(t, P);
+        const int kvh = u.kvh;
         for (int kt = 0; kt < u.nkt && ok; ++kt) {
           for (int ks = 0; ks < P.ksteps; ++ks) {
             const int s = static_cast<int>(f % kStages);
@@ -195,8 +235,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
       const uint32_t base = su32(smem);
       int64_t f = 0, tiles = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x) {
-        const AUnit u = ad_unit(t, P, BH);
+      for (int64_t n = 0; ok; ++n) {
+        int64_t t;
+        if (!(ok = ad_next_unit(bars, n, P.status, &t)) || t < 0) break;
+        const AUnit u = ad_unit(t, P);
         for (int kt = 0; kt < u.nkt && ok; ++kt) {
           const int buf = static_cast<int>(tiles & 1);
           const int64_t use = tiles >> 1;
@@ -235,8 +277,11 @@ __global__ void __launch_bounds__(kAThreads, 1)
     const int R = P.R;
     int64_t tiles = 0, n = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < P.units && ok; t += gridDim.x, ++n) {
-      const AUnit un = ad_unit(t, P, BH);
+    for (; ok; ++n) {
+      int64_t t;
+      ok = __all_sync(0xffffffffu, ad_next_unit(bars, n, P.status, &t));
+      if (!ok || t < 0) break;
+      const AUnit un = ad_unit(t, P);
       const int slot = static_cast<int>(n & 1);
       // the slot's previous unit (n - 2) must be through its fixup before it is overwritten
       ok = __all_sync(0xffffffffu, ad_wait(&bars->fix_done[slot],
@@ -290,7 +335,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
 #pragma unroll
               for (int c = 0; c < 32; c += lv) {
                 const int j = jb + c / lv;  // the last tile may reach past block nb-1
-                if (j < P.nb) esc[static_cast<int64_t>(j) * kAM + row] = e[c];
+                if (j < P.nb) __stcs(esc + static_cast<int64_t>(j) * kAM + row, e[c]);
               }
             }
             if (lv < 32) {
@@ -299,7 +344,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
             }
           }
           l_run += e[0];
-          msc[(kt * (kAN / 32) + ch) * kAM + row] = m_new;
+          __stcs(msc + (kt * (kAN / 32) + ch) * kAM + row, m_new);
           m_run = m_new;
         }
         tc_fence_before();
@@ -321,8 +366,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
     const int R = P.R;
     const int64_t tri = static_cast<int64_t>(P.nb) * (P.nb + 1) / 2;
     int64_t n = 0;
-    for (int64_t t = blockIdx.x; t < P.units; t += gridDim.x, ++n) {
-      const AUnit un = ad_unit(t, P, BH);
+    for (;; ++n) {
+      int64_t t;
+      if (!__all_sync(0xffffffffu, ad_next_unit(bars, n, P.status, &t)) || t < 0) break;
+      const AUnit un = ad_unit(t, P);
       const int slot = static_cast<int>(n & 1);
       if (!__all_sync(0xffffffffu, ad_wait(&bars->unit_done[slot],
                                            static_cast<uint32_t>((n >> 1) & 1), bars,
@@ -347,15 +394,15 @@ __global__ void __launch_bounds__(kAThreads, 1)
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int j = min(j0 + q, i_hi);
-          ev[q] = esc[static_cast<int64_t>(j) * kAM + row];
-          sv[q] = msc[((j * R) >> 5) * kAM + row];  // snapshot of the chunk holding block j
+          ev[q] = __ldcs(esc + static_cast<int64_t>(j) * kAM + row);
+          sv[q] = __ldcs(msc + ((j * R) >> 5) * kAM + row);  // snapshot of block j's chunk
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int j = j0 + q;
           float val = valid && j <= i ? ev[q] * ex2(sv[q] - m_run) * inv_l : 0.f;
           for (int o = 1; o < R; o <<= 1) val += __shfl_xor_sync(0xffffffffu, val, o);
-          if (valid && j <= i && (lane & (R - 1)) == 0) prow[j] = val * inv_n;
+          if (valid && j <= i && (lane & (R - 1)) == 0) __stcs(prow + j, val * inv_n);
         }
       }
       mbar_arrive(&bars->fix_done[slot]);  // the slot may be overwritten
@@ -401,7 +448,8 @@ size_t antidiag_scratch_floats(int B, int Hq, int S, int block, int stride) {
   const int64_t nred = S / stride;
   const int64_t nkt = (nred + kAN - 1) / kAN;
   const int64_t slots = std::min<int64_t>(antidiag_units(B, Hq, S, stride), kAdSlots);
-  return static_cast<size_t>(slots * 2 * (nb + (kAN / 32) * nkt) * kAM);  // two slots per CTA
+  // the work counter (64 floats, keeping the rest 256-byte aligned), then two slots per CTA
+  return static_cast<size_t>(64 + slots * 2 * (nb + (kAN / 32) * nkt) * kAM);
 }
 
 cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv, int S, int D,
@@ -425,7 +473,8 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   P.units = antidiag_units(B, Hq, S, stride);
   P.scale_log2 = static_cast<float>(1.4426950408889634 / (stride * std::sqrt(static_cast<double>(D))));
   P.p = p;
-  P.scratch = scratch;
+  P.next_unit = reinterpret_cast<unsigned long long*>(scratch);
+  P.scratch = scratch + 64;
   P.scratch_per_slot = static_cast<int64_t>(P.nb + (kAN / 32) * ((P.nred + kAN - 1) / kAN)) * kAM;
   P.status = status;
   CUtensorMap tq, tk;
@@ -439,6 +488,8 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>({P.units, static_cast<int64_t>(sm_count()),
                                           static_cast<int64_t>(kAdSlots)});
+  e = cudaMemsetAsync(P.next_unit, 0, sizeof(unsigned long long), st);
+  if (e != cudaSuccess) return e;
   antidiag_sm100_kernel<<<static_cast<unsigned>(grid), kAThreads, smem, st>>>(tq, tk, P);
   return cudaGetLastError();
 }
