@@ -44,8 +44,12 @@ KERNELS_PER_STEP = 4
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615536128 + 1023997440,
-                "sources_sha256": "01d0c89698de2d0b5e9e849b14c3e348330e4c12402f65143710731da57d4678"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1618323968 + 1024240384,
+                "sources_sha256": "d648f7134bd5690aab5e67e2830f8500fd66fcb87e487bfd9aa37a2ca9632376"}
+# The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
+# profiles/antidiag_sm100_llama3-8b-128k.md.
+AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,
+              "sources_sha256": "a170d26289c250b936c431969e85cbcdbe77282f17e7f2640721f48784d9b454"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -70,15 +74,28 @@ def parse():
     return p.parse_args()
 
 
-def attn_traffic(workload_name):
+def _sources_sha(files):
     import hashlib
 
     h = hashlib.sha256()
-    for f in ("attn_sm100.cu", "pairs.cu", "sm100.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "block_sparse_causal_pooling_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    if workload_name == ATTN_TRAFFIC["workload"] and h.hexdigest() == ATTN_TRAFFIC["sources_sha256"]:
+    return h.hexdigest()
+
+
+def attn_traffic(workload_name):
+    if (workload_name == ATTN_TRAFFIC["workload"] and
+            _sources_sha(("attn_sm100.cu", "pairs.cu", "sm100.cuh")) ==
+            ATTN_TRAFFIC["sources_sha256"]):
         return ATTN_TRAFFIC["bytes"]
+    return None
+
+
+def antidiag_traffic(workload_name, stride):
+    if (workload_name == AD_TRAFFIC["workload"] and stride == AD_TRAFFIC["stride"] and
+            _sources_sha(("antidiag_sm100.cu", "sm100.cuh")) == AD_TRAFFIC["sources_sha256"]):
+        return AD_TRAFFIC["bytes"]
     return None
 
 
@@ -476,7 +493,10 @@ def run_ours(args, world, rank, local):
         ad_tf = ad_flop / (sel_ms * 1e-3) / 1e12
         line["kernels"]["select"].update({
             "what": "antidiag estimator + selection from p", "bound": "tensor",
-            "estimator_tflop": ad_flop / 1e12, "tflops": ad_tf, "frac": ad_tf / peak_tf})
+            "estimator_tflop": ad_flop / 1e12, "tflops": ad_tf, "frac": ad_tf / peak_tf,
+            "estimator_traffic": antidiag_traffic(w.name, mp["stride"]),
+            "estimator_algorithmic_bytes": 2 * w.B * (w.Hq + w.Hkv) * w.S * w.D +
+                                           4 * w.B * w.Hq * w.nb * (w.nb + 1) // 2})
         line["gpu_launches"] = (KERNELS_PER_STEP + 1) * K
     if e2e is not None:
         line["e2e"] = e2e
