@@ -190,3 +190,72 @@ def test_select_p_metric_output():
             np.testing.assert_allclose(mgd, mref, rtol=0, atol=2e-5 * max(1.0, np.abs(mref).max()))
         else:
             np.testing.assert_allclose(mgd, mref, rtol=2e-6, atol=1e-35)
+
+
+def _full_rows(w, seed=11, n_random=9):
+    import random
+
+    rng = random.Random(seed)
+    rows = {(0, 0, 0), (0, 0, 1), (0, w.Hq - 1, w.nb - 1), (w.B - 1, 0, w.nb - 1)}
+    while len(rows) < 4 + n_random:
+        rows.add((rng.randrange(w.B), rng.randrange(w.Hq), rng.randrange(w.nb)))
+    return sorted(rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("w", [wl.LLAMA_128K, wl.QWEN_64K], ids=lambda w: w.name)
+def test_full_size_sampled(w):
+    """The bench's workloads at full size, in its launch configuration (stem_prefill_ex with a
+    caller workspace on torch's stream): every row of p sums to 1; sampled rows of p, their
+    selections and their outputs against the oracle computed row by row."""
+    stride = 16
+    m = method(w, stride)
+    q, k, v = wl.make_inputs(w, DEV)
+    out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min, m)
+    ws = S.alloc_workspace(q, k, w.block, m)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S.stem_prefill_ex(q, k, v, w.block, 0.0, 0.0, 0, out, sel_idx, sel_cnt, ws, status,
+                      method=m)
+    p = S.stem_antidiag(q, k, w.block, m)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    # row sums, every row (a float32 sum of up to nb values each)
+    tri_i = torch.repeat_interleave(torch.arange(w.nb, device=DEV),
+                                    torch.arange(1, w.nb + 1, device=DEV))
+    sums = torch.zeros((w.B, w.Hq, w.nb), dtype=torch.float64, device=DEV)
+    sums.index_add_(2, tri_i, p.double())
+    assert float((sums - 1.0).abs().max()) < 1e-4
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    rows = _full_rows(w)
+    pref = oracle.antidiag(qc, kc, w.block, stride, rows=rows)
+    tol = p_rel_tol(qc, kc, stride)
+    pc = p.cpu().double().numpy()
+    # selection of the sampled rows from the oracle's p rows (other rows: placeholders)
+    _, _, vn = oracle.pool(qc, kc, vc, w.block)
+    kk, off = oracle.budget(w.nb, w.rho_min, w.tau, w.k_min)
+    pp = np.ones((w.B, w.Hq, w.nb * (w.nb + 1) // 2))
+    for (b, h, i), r in zip(rows, pref):
+        lo = i * (i + 1) // 2
+        got = pc[b, h, lo:lo + i + 1]
+        assert np.all(np.abs(got - r[:i + 1]) <= tol * r[:i + 1] + 1e-12), (b, h, i)
+        pp[b, h, lo:lo + i + 1] = r[:i + 1]
+    mref = oracle.metric_from_p(pp, vn)
+    ref_idx, ref_cnt = oracle.select(mref, kk, off)
+    si = sel_idx.cpu().numpy()
+    rel = _sel_rel((qc, kc), stride, False)
+    keep = []
+    for (b, h, i) in rows:
+        assert int(sel_cnt[b, h, i]) == int(kk[i])
+        g = si[b, h, off[i]:off[i + 1]]
+        r = ref_idx[b, h, off[i]:off[i + 1]]
+        if np.array_equal(g, r):
+            keep.append((b, h, i))
+            continue
+        extra, missing = np.setdiff1d(g, r), np.setdiff1d(r, g)
+        mrow = oracle.metric_row(mref, b, h, i)
+        hi, lo_ = mrow[missing].max(), mrow[extra].min()
+        assert hi - lo_ <= rel * hi, ((b, h, i), extra, missing)
+    assert len(keep) >= len(rows) - 2
+    ref_out = oracle.attention(qc, kc, vc, w.block, ref_idx, ref_cnt, off, keep)
+    parity.assert_out_close(parity.out_rows(out, keep, w.block), ref_out, w.torch_dtype,
+                            f"antidiag/{w.name}")
