@@ -492,11 +492,15 @@ int stem_prefill(const void* q, const void* k, const void* v, int B, int Hq, int
   return run_prefill(&a, nullptr);
 }
 
-// Host buffers: the problem splits into B*Hkv independent chunks (batch b, kv-head group g: the
-// group's G query heads, its K and V head, their outputs and CSR rows, each contiguous). Chunk
-// c's inputs go up on one stream, its kernels run on a second once they have arrived, and its
-// results come down on a third once its kernels are done, so the copies of one chunk overlap
-// the kernels of the others and the two PCIe directions overlap each other.
+// Host buffers: the problem splits into independent pieces, each a pair of query heads of one
+// (batch b, kv-head group g) with the group's K and V (the whole group when the selection is
+// shared by the group). Piece c's inputs go up on one stream (K and V with the group's first
+// piece), its kernels run on a second once they have arrived, and its results come down on a
+// third once its kernels are done, so the copies of one piece overlap the kernels of the others
+// and the two PCIe directions overlap each other; small pieces keep the pipeline's fill (the
+// first piece's upload) and drain (the last piece's kernels and download) short. Each head's
+// results are those of the device-buffer path: selection and attention are per head, and the
+// pieces keep the attention kernel's head pairs.
 int stem_prefill_host(const stem_args_t* h) {
   if (h == nullptr) return STEM_ERR_ARG;
   int rc = check_shape(h->B, h->Hq, h->Hkv, h->S, h->D, h->block, h->dtype);
@@ -510,26 +514,29 @@ int stem_prefill_host(const stem_args_t* h) {
   if (is_empty(h->B, h->S)) return STEM_OK;
   if (!h->q || !h->k || !h->v || !h->out || !h->sel_idx || !h->sel_cnt) return STEM_ERR_ARG;
   const int G = h->Hq / h->Hkv;
-  const int nc = h->B * h->Hkv;  // chunks
+  const int hp = (m.share == STEM_SHARE_GROUP || G < 2) ? G : 2;  // query heads per piece
+  const int per_group = (G + hp - 1) / hp;
+  const int np = h->B * h->Hkv * per_group;  // pieces
   const size_t es = elem_size(h->dtype);
   const int64_t cap = capacity(nb, m);
-  const size_t qcb = es * static_cast<size_t>(G) * h->S * h->D;  // per chunk
-  const size_t kvcb = es * static_cast<size_t>(h->S) * h->D;
-  const size_t sicb = sizeof(int32_t) * static_cast<size_t>(G) * cap;
-  const size_t sccb = sizeof(int32_t) * static_cast<size_t>(G) * nb;
-  const Layout Lc = layout(1, G, 1, nb, h->D, &m, h->S, h->block);  // one chunk's workspace
+  const size_t hb = es * static_cast<size_t>(h->S) * h->D;  // one head of q, k, v or out
+  const size_t sih = sizeof(int32_t) * static_cast<size_t>(cap);  // one head's CSR
+  const size_t sch = sizeof(int32_t) * static_cast<size_t>(nb);   // one head's counts
+  const size_t nq = static_cast<size_t>(h->B) * h->Hq, nkv = static_cast<size_t>(h->B) * h->Hkv;
+  const Layout Lc = layout(1, hp, 1, nb, h->D, &m, h->S, h->block);  // one piece's workspace
   const Plan* plan = get_plan(nb, m);
   if (plan == nullptr) return STEM_ERR_CUDA;
-  // device arena: chunk status words | the plan | chunk workspaces | q | k | v | out | sel_idx |
-  // sel_cnt. The plan and the cleared status words go up first on the input stream: a copy
-  // issued on the compute stream would wait in the copy engine behind every chunk's inputs.
-  const size_t o_plan = align_up(sizeof(int32_t) * nc);
+  // device arena: piece status words | the plan | piece workspaces | q | k | v | out | sel_idx |
+  // sel_cnt (the tensors in their host layout). The plan and the cleared status words go up
+  // first on the input stream: a copy issued on the compute stream would wait in the copy
+  // engine behind every piece's inputs.
+  const size_t o_plan = align_up(sizeof(int32_t) * np);
   const size_t o_ws = o_plan + plan_bytes(nb);
   const size_t wsb = align_up(Lc.total);
-  const size_t o_q = o_ws + wsb * nc, o_k = o_q + align_up(qcb * nc),
-               o_v = o_k + align_up(kvcb * nc), o_out = o_v + align_up(kvcb * nc),
-               o_si = o_out + align_up(qcb * nc), o_sc = o_si + align_up(sicb * nc),
-               total = o_sc + align_up(sccb * nc);
+  const size_t o_q = o_ws + wsb * np, o_k = o_q + align_up(hb * nq),
+               o_v = o_k + align_up(hb * nkv), o_out = o_v + align_up(hb * nkv),
+               o_si = o_out + align_up(hb * nq), o_sc = o_si + align_up(sih * nq),
+               total = o_sc + align_up(sch * nq);
   static std::mutex host_mu;  // host-buffer calls share one arena: one at a time
   std::lock_guard<std::mutex> lock(host_mu);
   void* arena = nullptr;
@@ -537,7 +544,7 @@ int stem_prefill_host(const stem_args_t* h) {
   if (rc != STEM_OK) return rc;
   auto* base = static_cast<unsigned char*>(arena);
   cudaStream_t sin = nullptr, srun = nullptr, sout = nullptr;
-  std::vector<cudaEvent_t> ev(2 * static_cast<size_t>(nc), nullptr);
+  std::vector<cudaEvent_t> ev(2 * static_cast<size_t>(np), nullptr);
   cudaError_t e = cudaSuccess;
   auto cleanup = [&]() {
     for (cudaStream_t s : {sin, srun, sout})
@@ -547,6 +554,12 @@ int stem_prefill_host(const stem_args_t* h) {
     for (cudaStream_t s : {sin, srun, sout})
       if (s) cudaStreamDestroy(s);
   };
+  auto up = [&](size_t off, const void* src, size_t bytes) {
+    return cudaMemcpyAsync(base + off, src, bytes, cudaMemcpyHostToDevice, sin);
+  };
+  auto down = [&](void* dst, size_t off, size_t bytes) {
+    return cudaMemcpyAsync(dst, base + off, bytes, cudaMemcpyDeviceToHost, sout);
+  };
   do {
     if ((e = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking))) break;
     if ((e = cudaStreamCreateWithFlags(&srun, cudaStreamNonBlocking))) break;
@@ -554,55 +567,57 @@ int stem_prefill_host(const stem_args_t* h) {
     for (auto& x : ev)
       if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming))) break;
     if (e) break;
-    if ((e = cudaMemsetAsync(base, 0, sizeof(int32_t) * nc, sin))) break;
+    if ((e = cudaMemsetAsync(base, 0, sizeof(int32_t) * np, sin))) break;
     if ((e = cudaMemcpyAsync(base + o_plan, plan->host, plan->bytes, cudaMemcpyHostToDevice, sin)))
       break;
     PlanDev pd;
     pd.k = reinterpret_cast<const int32_t*>(base + o_plan);
     pd.off = pd.k + nb;
     pd.order = pd.k + 2 * nb + 1;
-    for (int c = 0; c < nc && rc == STEM_OK && e == cudaSuccess; ++c) {
-      const auto* hq = static_cast<const unsigned char*>(h->q) + qcb * c;
-      const auto* hk = static_cast<const unsigned char*>(h->k) + kvcb * c;
-      const auto* hv = static_cast<const unsigned char*>(h->v) + kvcb * c;
+    for (int c = 0; c < np && rc == STEM_OK && e == cudaSuccess; ++c) {
+      const int bg = c / per_group, pi = c % per_group;
+      const int nh = std::min(hp, G - pi * hp);
+      const size_t qh0 = static_cast<size_t>(bg) * G + static_cast<size_t>(pi) * hp;  // 1st head
+      if (pi == 0) {  // the group's K and V go up with its first piece
+        if ((e = up(o_k + hb * bg, static_cast<const unsigned char*>(h->k) + hb * bg, hb))) break;
+        if ((e = up(o_v + hb * bg, static_cast<const unsigned char*>(h->v) + hb * bg, hb))) break;
+      }
+      if ((e = up(o_q + hb * qh0, static_cast<const unsigned char*>(h->q) + hb * qh0, hb * nh)))
+        break;
       stem_args_t d = *h;
       d.B = 1;
-      d.Hq = G;
+      d.Hq = nh;
       d.Hkv = 1;
-      d.q = base + o_q + qcb * c;
-      d.k = base + o_k + kvcb * c;
-      d.v = base + o_v + kvcb * c;
-      d.out = base + o_out + qcb * c;
-      d.sel_idx = reinterpret_cast<int32_t*>(base + o_si + sicb * c);
-      d.sel_cnt = reinterpret_cast<int32_t*>(base + o_sc + sccb * c);
+      d.q = base + o_q + hb * qh0;
+      d.k = base + o_k + hb * bg;
+      d.v = base + o_v + hb * bg;
+      d.out = base + o_out + hb * qh0;
+      d.sel_idx = reinterpret_cast<int32_t*>(base + o_si + sih * qh0);
+      d.sel_cnt = reinterpret_cast<int32_t*>(base + o_sc + sch * qh0);
       d.workspace = base + o_ws + wsb * c;
       d.workspace_bytes = Lc.total;
       d.status = reinterpret_cast<int32_t*>(base) + c;
       d.events = nullptr;
-      if ((e = cudaMemcpyAsync(const_cast<void*>(d.q), hq, qcb, cudaMemcpyHostToDevice, sin))) break;
-      if ((e = cudaMemcpyAsync(const_cast<void*>(d.k), hk, kvcb, cudaMemcpyHostToDevice, sin))) break;
-      if ((e = cudaMemcpyAsync(const_cast<void*>(d.v), hv, kvcb, cudaMemcpyHostToDevice, sin))) break;
       if ((e = cudaEventRecord(ev[2 * c], sin))) break;
       if ((e = cudaStreamWaitEvent(srun, ev[2 * c], 0))) break;
       if ((rc = enqueue_kernels(&d, m, nb, plan->cap, pd, srun)) != STEM_OK) break;
       if ((e = cudaEventRecord(ev[2 * c + 1], srun))) break;
       if ((e = cudaStreamWaitEvent(sout, ev[2 * c + 1], 0))) break;
-      if ((e = cudaMemcpyAsync(static_cast<unsigned char*>(h->out) + qcb * c, d.out, qcb,
-                               cudaMemcpyDeviceToHost, sout)))
+      if ((e = down(static_cast<unsigned char*>(h->out) + hb * qh0, o_out + hb * qh0, hb * nh)))
         break;
-      if ((e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(h->sel_idx) + sicb * c,
-                               d.sel_idx, sicb, cudaMemcpyDeviceToHost, sout)))
+      if ((e = down(reinterpret_cast<unsigned char*>(h->sel_idx) + sih * qh0, o_si + sih * qh0,
+                    sih * nh)))
         break;
-      if ((e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(h->sel_cnt) + sccb * c,
-                               d.sel_cnt, sccb, cudaMemcpyDeviceToHost, sout)))
+      if ((e = down(reinterpret_cast<unsigned char*>(h->sel_cnt) + sch * qh0, o_sc + sch * qh0,
+                    sch * nh)))
         break;
     }
   } while (false);
   cleanup();
   if (rc != STEM_OK) return rc;
   if (e != cudaSuccess) return cuda_err(e);
-  std::vector<int32_t> status(nc, 0);
-  e = cudaMemcpy(status.data(), base, sizeof(int32_t) * nc, cudaMemcpyDeviceToHost);
+  std::vector<int32_t> status(np, 0);
+  e = cudaMemcpy(status.data(), base, sizeof(int32_t) * np, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_err(e);
   for (int32_t x : status)
     if (x < 0) return x;
