@@ -93,6 +93,7 @@ struct AdParams {
   float* scratch;       // [gridDim.x][2 slots][nb*128 + 8*nkt_max*128]
   int64_t scratch_per_slot;
   int32_t* status;
+  int withhold;         // test switch: the first stage's copies are never sent
 };
 
 __device__ __noinline__ bool ad_wait_slow(uint64_t* b, uint32_t parity, ABars* bars,
@@ -214,6 +215,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
                                P.status)))
               break;
             mbar_expect_tx(&bars->full[s], kStageBytes);
+            if (P.withhold && f == 0) {  // test switch: the stage's bytes never arrive
+              ++f;
+              continue;
+            }
             const int chunk = ks / P.kparts, part = ks % P.kparts;
             unsigned char* st = smem + s * kStageBytes;
             tma_load_3d(st, &tm_q, ks * 64, u.qt * kAM, u.bh, &bars->full[s], pol_q);
@@ -477,6 +482,7 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   P.scratch = scratch + 64;
   P.scratch_per_slot = static_cast<int64_t>(P.nb + (kAN / 32) * ((P.nred + kAN - 1) / kAN)) * kAM;
   P.status = status;
+  P.withhold = g_withhold_q.load();
   CUtensorMap tq, tk;
   if (!make_group_map(&tq, q, static_cast<uint64_t>(B) * Hq, S, D, stride, kAM) ||
       !make_group_map(&tk, k, static_cast<uint64_t>(B) * Hkv, S, D, stride, kAN))

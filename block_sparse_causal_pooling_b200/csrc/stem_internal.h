@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace stem {
 
 // Device view of the budget plan (int32 arrays inside the workspace).
@@ -76,5 +78,8 @@ cudaError_t launch_attn_f32(const float* q, const float* k, const float* v, int 
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// Test switch of stem_test_withhold_q (attn_sm100.cu): read by the tensor-core kernels' launchers.
+extern std::atomic<int> g_withhold_q;
 
 }  // namespace stem

@@ -361,12 +361,13 @@ int stem_select_static(const float* qbar, const float* kbar, const float* vnorm,
 
 /*
  * stem_test_withhold_q: TEST ONLY. With on != 0, later launches of the bfloat16 block-128
- * attention kernel (stem_prefill*, stem_sparse_attn*) skip each CTA's first Q tile, so the
- * kernel's bounded wait for it expires (after about 2 s): the kernel then records
- * STEM_ERR_TIMEOUT in the status word, every role leaves its loop, issued copies and products
- * are drained, TMEM is freed and the kernel returns, leaving the CUDA context usable. It exists
- * to exercise that path; the outputs of such a call are undefined. Process-wide; returns the
- * previous setting (0 or 1). The paper has no counterpart.
+ * attention kernel (stem_prefill*, stem_sparse_attn*) skip each CTA's first Q tile, and later
+ * launches of the anti-diagonal estimator (score STEM_SCORE_ANTIDIAG, stem_antidiag_m) skip each
+ * CTA's first stage of copies, so the kernel's bounded wait for them expires (after about 2 s):
+ * the kernel then records STEM_ERR_TIMEOUT in the status word, every role leaves its loop, issued
+ * copies and products are drained, TMEM is freed and the kernel returns, leaving the CUDA
+ * context usable. It exists to exercise that path; the outputs of such a call are undefined.
+ * Process-wide; returns the previous setting (0 or 1). The paper has no counterpart.
  */
 int stem_test_withhold_q(int on);
 
