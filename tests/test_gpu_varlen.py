@@ -9,7 +9,7 @@ import torch
 import oracle
 from block_sparse_causal_pooling_b200 import stem as S
 from block_sparse_causal_pooling_b200 import workloads as wl
-from tests import parity
+from tests import parity, test_gpu_antidiag
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +25,10 @@ CASES = {
                    dict(schedule="exp", rho_min=0.3, tau=4.0, k_min=2)),
     "f32": (wl.TINY.replace(name="varlen", Hq=4, Hkv=2, D=128, block=128), [900, 130],
             dict(schedule="exp", rho_min=0.3, tau=4.0, k_min=2)),
+    # block scores by anti-diagonal sampling (every length a multiple of the 16-token group)
+    "bf16-antidiag": (wl.LLAMA_32K.replace(name="varlen", Hq=8, Hkv=2), [2048, 80, 0, 1600],
+                      dict(schedule="exp", rho_min=0.2, tau=6.0, k_min=3, score="antidiag",
+                           stride=16)),
 }
 
 
@@ -49,7 +53,8 @@ def test_varlen_matches_each_sequence(name):
     okw = dict(rho_min=md.get("rho_min", 1.0), tau=md.get("tau", 1.0), k_min=md["k_min"],
                schedule=md["schedule"], k_start=md.get("k_start", 0.0), mu=md.get("mu", 1.0),
                metric_form=md.get("metric", "product"), beta=md.get("beta", 0.0),
-               vsum=md.get("vsum", "mean"))
+               vsum=md.get("vsum", "mean"), score=md.get("score", "pooled"),
+               stride=md.get("stride", 16))
     for (qs, ks, vs), L, t0 in zip(seqs, lengths, cu[:-1]):
         if L == 0:
             continue
@@ -59,8 +64,11 @@ def test_varlen_matches_each_sequence(name):
         g_out = out[w.Hq * w.D * t0: w.Hq * w.D * (t0 + L)].view(1, w.Hq, L, w.D)
         g_si = si[w.Hq * capo: w.Hq * (capo + cap)].view(1, w.Hq, cap)
         g_sc = sc[w.Hq * nbo: w.Hq * (nbo + nb)].view(1, w.Hq, nb)
+        # anti-diagonal scores: near-ties within the bound derived from their arithmetic
+        rel = (2.0 * test_gpu_antidiag.p_rel_tol(qs, ks, md["stride"])
+               if md.get("score") == "antidiag" else parity.REL_TIE)
         res = parity.compare_selection(g_si, g_sc, ref["sel_idx"], ref["sel_cnt"], ref["m"],
-                                       ref["k"], ref["off"],
+                                       ref["k"], ref["off"], rel=rel,
                                        additive=md.get("metric") == "additive")
         assert not res["violations"], (L, res["violations"][:5])
         swapped = set(res["rows_bad"])
