@@ -71,6 +71,8 @@ def parse():
                         "antidiag: the default with block probabilities by anti-diagonal "
                         "sampling (--stride tokens per group)")
     p.add_argument("--stride", type=int, default=16)
+    p.add_argument("--no-context", action="store_true",
+                   help="skip the context timing of dense causal attention (torch SDPA)")
     return p.parse_args()
 
 
@@ -469,6 +471,7 @@ def run_ours(args, world, rank, local):
                 f"x{w.sink_scale}, {w.n_v_outliers()} V rows per kv-head x{w.v_outlier_scale}, "
                 f"heavy-tail fraction {w.heavy_tail_frac})",
         "config": dict(config_of(w, mp), kept_pairs=pairs, effective_tflop=flop / 1e12,
+                       causal_exact_tflop=causal_exact_flops(w, kk) / 1e12,
                        causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
@@ -500,9 +503,48 @@ def run_ours(args, world, rank, local):
         line["gpu_launches"] = (KERNELS_PER_STEP + 1) * K
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_context:
+        line["context"] = dense_context(q, k, v, ms)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, mp)
+        line["cpu_baseline"]["extrapolated_full_workload_s"] = (
+            flop / (line["cpu_baseline"]["value"] * 1e12))
     print(json.dumps(line), flush=True)
+
+
+def causal_exact_flops(w, kk):
+    """FLOPs of the kept pairs counting only causal (query, key) token pairs: the diagonal
+    block of every row is half a tile plus its diagonal; a partial last block counts its rows."""
+    full = wl.effective_flops(1, w.block, w.D)  # one whole tile
+    total = 0.0
+    for i in range(w.nb):
+        n = min(w.block, w.S - i * w.block)
+        off_diag = int(kk[i]) - 1
+        total += off_diag * full * n / w.block + full * n * (n + 1) / 2 / (w.block * w.block)
+    return w.B * w.Hq * total
+
+
+def dense_context(q, k, v, sparse_ms):
+    """Context, not a target: dense causal attention by torch's scaled_dot_product_attention
+    (a library kernel) at the same shape, against the step time."""
+    try:
+        G = q.shape[1] // k.shape[1]
+        fn = torch.nn.functional.scaled_dot_product_attention
+        run = lambda: fn(q, k, v, is_causal=True, enable_gqa=G > 1)  # noqa: E731
+        run()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(3):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        dense_ms = a.elapsed_time(b) / 3
+        return {"dense_causal_sdpa_ms": dense_ms, "speedup_vs_dense": dense_ms / sparse_ms,
+                "what": "torch scaled_dot_product_attention, is_causal, same Q/K/V (library "
+                        "kernel; not a baseline of this metric)"}
+    except Exception as e:  # noqa: BLE001
+        return {"dense_causal_sdpa_ms": None, "error": str(e)[:200]}
 
 
 def cpu_baseline(w, mp=None):
