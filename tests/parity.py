@@ -109,6 +109,12 @@ def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what:
     if dtype == torch.bfloat16 and ref.size:
         bound = np.maximum(t["max_abs"], np.abs(ref) * 2.0 ** -7)
         e["n_bound_above_max_abs"] = int((np.abs(ref) * 2.0 ** -7 > t["max_abs"]).sum())
+        # reported, not asserted: the error against the oracle rounded to bf16 (what an exact
+        # bf16 kernel would return) and how many outputs exceed 8 in magnitude (where a bf16
+        # half-ulp alone is 0.031)
+        ref_b = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+        e["max_abs_vs_bf16_ref"] = float(np.abs(gpu - ref_b).max())
+        e["n_ref_above_8"] = int((np.abs(ref) > 8).sum())
     worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
     assert worst <= 0 and e["mean_abs"] <= t["mean_abs"], (what, e, t)
     return e
