@@ -273,9 +273,10 @@ int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, i
                        const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
                        void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
-/* Workspace bytes stem_prefill_ex needs for this shape and method (with STEM_SCORE_ANTIDIAG
- * it also holds the block probabilities and the estimator's per-CTA scratch, about
- * 148 * 512 * ceil(S/block) bytes). 0 for an invalid or empty request. Host only. */
+/* Workspace bytes stem_prefill_ex needs for this shape and method. With STEM_SCORE_ANTIDIAG it
+ * also holds the block probabilities (4 * B * Hq * nb * (nb+1) / 2 bytes) and the estimator's
+ * scratch: up to 148 CTAs x 2 slots x (nb + 8 * ceil(S / (256 * stride))) x 512 bytes (about
+ * 194 MB at S = 131072, block 128, stride 16). 0 for an invalid or empty request. Host only. */
 size_t stem_workspace_size_m(int B, int Hq, int Hkv, int S, int D, int block,
                              const stem_method_t* m);
 
