@@ -10,7 +10,8 @@ max(1, |M|): |M_a - M_b| <= REL_TIE * max(1, |M_a|, |M_b|).
 Attention output: max-abs error <= 2e-2 and mean-abs error <= 1e-3 against the oracle's
 double-precision result for bfloat16 inputs (float32 accumulation); tighter for float32 inputs.
 For bfloat16 the per-element max-abs bound grows as 2^-7 |reference| above |reference| = 2.56
-(the bfloat16 rounding of P and of the output; see assert_out_close).
+(the bfloat16 rounding of P and of the output; see assert_out_close), and the mean-abs bound by
+the mean of 2^-8 |reference| over those elements.
 """
 
 from __future__ import annotations
@@ -116,5 +117,13 @@ def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what:
         e["max_abs_vs_bf16_ref"] = float(np.abs(gpu - ref_b).max())
         e["n_ref_above_8"] = int((np.abs(ref) > 8).sum())
     worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
-    assert worst <= 0 and e["mean_abs"] <= t["mean_abs"], (what, e, t)
+    # the mean bound grows the same way: elements above |reference| = 2.56 add their own share
+    # of the bf16 rounding, 2^-8 |reference| each (0 for the named workloads, whose outputs stay
+    # below 2.56)
+    mean_bound = t["mean_abs"]
+    if dtype == torch.bfloat16 and ref.size:
+        big = np.abs(ref) > 2.56
+        mean_bound += float((np.abs(ref) * 2.0 ** -8 * big).mean())
+        e["mean_bound"] = mean_bound
+    assert worst <= 0 and e["mean_abs"] <= mean_bound, (what, e, t)
     return e
