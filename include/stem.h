@@ -42,6 +42,11 @@
  *     Faults surface at the caller's next synchronisation. The library never prints or aborts.
  *   - Arguments are validated before anything is enqueued; on a negative return nothing was
  *     launched and no buffer was written.
+ *   - Host state: the budget plan of each distinct (nb, schedule parameters, k_min) is built on
+ *     first use and kept in pinned host memory for the life of the process (3*nb + 1 int32 per
+ *     plan, shared by all threads under a lock). Plans are never freed, since a copy enqueued
+ *     from one may still be in flight; a caller with many distinct sequence lengths holds one
+ *     plan per length.
  */
 #ifndef STEM_H
 #define STEM_H
