@@ -357,10 +357,19 @@ class RawEvents:
         self.made = []
 
 
+L2_BYTES = 126 * 2 ** 20
+
+
 def config_of(w, mp=None):
+    elt = 2 if w.dtype == "bf16" else 4
+    in_bytes = w.B * (w.Hq + 2 * w.Hkv) * w.S * w.D * elt
+    l2 = (f"inputs (Q+K+V, {in_bytes / 1e6:.0f} MB) larger than the 126 MB L2; no flush"
+          if in_bytes > L2_BYTES else
+          f"inputs (Q+K+V, {in_bytes / 1e6:.1f} MB) fit in L2; not flushed (a parity-size "
+          f"workload, not a timing one)")
     c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "D": w.D,
          "block": w.block, "rho_min": w.rho_min, "tau": w.tau, "k_min": w.k_min,
-         "input_dtype": w.dtype, "l2": "inputs (Q+K+V) larger than L2; no flush"}
+         "input_dtype": w.dtype, "l2": l2}
     if mp is not None:
         c.pop("rho_min")
         c.pop("tau")
