@@ -44,8 +44,8 @@ KERNELS_PER_STEP = 4
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1618323968 + 1024240384,
-                "sources_sha256": "d648f7134bd5690aab5e67e2830f8500fd66fcb87e487bfd9aa37a2ca9632376"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615505920 + 1023842304,
+                "sources_sha256": "99bf71cdd8604193e2a52d3c5b933240922d06a42cb1fc3c842d78552a79e9c5"}
 # The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,

@@ -216,6 +216,7 @@ struct Seq {
   int n, j, cnt;
   Item it;
   const uint32_t* row;
+  uint32_t e_next;  // schedule entry of the coming step, loaded one call ahead
   __device__ __forceinline__ void init(int64_t items_, int G_, int nb_, int Hkv_, int Hq_,
                                        int64_t cap_, PlanDev plan_, const uint32_t* sched_) {
     t = blockIdx.x;
@@ -232,12 +233,17 @@ struct Seq {
       cnt = plan.k[it.i];
       j = 0;
       row = sched_row(sched, it, Hkv, G, cap, plan);
+      e_next = row[0];
     }
+    // the entry of this step was loaded by the previous call; the next one is loaded now, so
+    // its latency overlaps a step's work instead of stalling the caller
+    const uint32_t e = e_next;
+    if (j + 1 < cnt) e_next = row[j + 1];
     s.n = n;
     s.first = (j == 0);
     s.last = (j == cnt - 1);
     s.it = it;
-    sched_step(row[j], it.i, s.ba, s.bb);
+    sched_step(e, it.i, s.ba, s.bb);
     ++j;
     return true;
   }
@@ -648,10 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode(t, G, nb, Hkv, plan.order);
       const int cnt = plan.k[it.i];
       const uint32_t* srow = sched_row(sched, it, Hkv, G, cap, plan);
+      uint32_t e_next = srow[0];  // loaded one step ahead, as in Seq
       for (int j = 0; j < cnt && ok; ++j) {
+        const uint32_t e = e_next;
+        if (j + 1 < cnt) e_next = srow[j + 1];
         Step x;
         x.it = it;
-        sched_step(srow[j], it.i, x.ba, x.bb);
+        sched_step(e, it.i, x.ba, x.bb);
         const bool has_b = x.has_b(), shared = x.shared();
         if (have_prev) order.v_a();
         order.k_a();
