@@ -44,8 +44,8 @@ KERNELS_PER_STEP = 4
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615505920 + 1023842304,
-                "sources_sha256": "99bf71cdd8604193e2a52d3c5b933240922d06a42cb1fc3c842d78552a79e9c5"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615398912 + 1023005184,
+                "sources_sha256": "1441e55fb9487896d62f3b2102b2ee71d65da1e8c83734d6fe9433e1b85f8c55"}
 # The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,

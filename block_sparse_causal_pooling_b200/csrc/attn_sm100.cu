@@ -158,6 +158,58 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Eight products of one group issued back to back from one asm block, their descriptors
+// computed beforehand: one predicate for the first product's accumulate flag and a
+// constant-true one for the other seven. The issuing thread's instructions between products
+// leave the tensor pipe idle (the MMA queue does not hide them), so they are kept to none.
+// operands: %0 d, %1..%8 a[0..7], %9..%16 b[0..7], %17 acc0, %18 idesc
+__device__ __forceinline__ void mma_ss8(uint32_t d, const uint64_t* a, const uint64_t* b,
+                                        uint32_t idesc, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t"
+      "setp.ne.b32 p0, %17, 0;\n\t"
+      "setp.eq.b32 p1, %17, %17;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %18, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %18, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %18, p1;\n\t}" ::"r"(d),
+      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]),
+      "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]),
+      "r"(acc0), "r"(idesc)
+      : "memory");
+}
+// The same with A from TMEM: product k reads P at column a0 + 8k.
+// operands: %0 d, %1 a0, %2..%9 b[0..7], %10 acc0, %11 idesc
+__device__ __forceinline__ void mma_ts8(uint32_t d, uint32_t a0, const uint64_t* b,
+                                        uint32_t idesc, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 p0, %10, 0;\n\t"
+      "setp.eq.b32 p1, %10, %10;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %11, p0;\n\t"
+      "add.u32 a, %1, 8;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %3, %11, p1;\n\t"
+      "add.u32 a, %1, 16;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %4, %11, p1;\n\t"
+      "add.u32 a, %1, 24;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %5, %11, p1;\n\t"
+      "add.u32 a, %1, 32;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %6, %11, p1;\n\t"
+      "add.u32 a, %1, 40;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %7, %11, p1;\n\t"
+      "add.u32 a, %1, 48;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %8, %11, p1;\n\t"
+      "add.u32 a, %1, 56;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %9, %11, p1;\n\t}" ::"r"(d),
+      "r"(a0), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
+      "l"(b[7]), "r"(acc0), "r"(idesc)
+      : "memory");
+}
+
 // Work item t -> (b, g, i, head pair): kv-head-group-major, query blocks in the plan's
 // heavy-first order, the ceil(G/2) head pairs of a group adjacent. Tile A is head g*G + 2p,
 // tile B head g*G + 2p + 1 (absent when G is odd and this is the group's last pair).
@@ -410,11 +462,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t qa = q_base + tl * C::kTile;
         const uint32_t ka = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
+        static_assert(C::kKSteps == 8 || C::kKSteps == 4, "group of 8 (D 128) or 4 (D 64)");
+        if constexpr (C::kKSteps == 8) {
+          uint64_t ad[8], bd[8];
 #pragma unroll
-        for (int kk = 0; kk < C::kKSteps; ++kk) {
-          const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
-          mma_ss(tmem + tl * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
+            ad[kk] = smem_desc(qa + off, 16, 1024);
+            bd[kk] = smem_desc(ka + off, 16, 1024);
+          }
+          mma_ss8(tmem + tl * 128, ad, bd, idesc_s, 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
+            mma_ss(tmem + tl * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
+                   idesc_s, kk > 0 ? 1u : 0u);
+          }
         }
         tc_commit(&bars->s_full[tl]);
         return true;
@@ -436,11 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t vaddr = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
         const uint32_t o_tm = tmem + 256 + tl * 128, p_tm = tmem + tl * 128;
-#pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
+        {
           // B = V rows kk*16 .. +15 (keys), MN-major: 64-column boxes kN*128 bytes apart
-          const uint64_t bd = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
-          mma_ts(o_tm, p_tm + kk * 8, bd, idesc_o, (st.first && kk == 0) ? 0u : 1u);
+          uint64_t bd[8];
+#pragma unroll
+          for (int kk = 0; kk < kN / 16; ++kk)
+            bd[kk] = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
+          mma_ts8(o_tm, p_tm, bd, idesc_o, st.first ? 0u : 1u);
         }
         if (tl == 1 && !next_has_b) tc_commit(&bars->kv_empty[f % kSlots]);
         if (st.last) {
