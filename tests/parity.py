@@ -9,9 +9,17 @@ max(1, |M|): |M_a - M_b| <= REL_TIE * max(1, |M_a|, |M_b|).
 
 Attention output: max-abs error <= 2e-2 and mean-abs error <= 1e-3 against the oracle's
 double-precision result for bfloat16 inputs (float32 accumulation); tighter for float32 inputs.
-For bfloat16 the per-element max-abs bound grows as 2^-7 |reference| above |reference| = 2.56
-(the bfloat16 rounding of P and of the output; see assert_out_close), and the mean-abs bound by
-the mean of 2^-8 |reference| over those elements.
+These bounds hold for every element of every named workload and of the small cases drawn with
+their value recipes; the tests assert that no element there needs more.
+
+One exception, for synthetic cases built to have very large outputs (many x5 V outliers in a
+short sequence, or key blocks scaled far above the sink): where |reference| >= 8 a bfloat16
+output cannot be within 2e-2 of it, since half a bfloat16 ulp there is 2^-5 or more. For those
+elements alone, and only in cases that declare outliers=True, the bound adds that half-ulp.
+
+Rows whose kept set differs from the oracle's by a tie swap are compared with the oracle's
+attention over the GPU's own kept set (several selections are correct there, and each has its
+own exact output), under the same bounds.
 """
 
 from __future__ import annotations
@@ -98,32 +106,70 @@ def out_error(gpu: np.ndarray, ref: np.ndarray):
                 max_ref=float(np.abs(ref).max()) if ref.size else 0.0)
 
 
-def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
-    """Max-abs and mean-abs error against the oracle. For bfloat16 the per-element bound is
-    max(max_abs, 2^-7 |reference|): P enters P V rounded to bfloat16 (relative error <= 2^-9)
-    and the output is rounded to bfloat16 (<= 2^-8 relative), so where one key dominates a
-    large output the error of any such kernel approaches 2^-7 |out|. Up to |out| = 2.56 the
-    bound is max_abs itself."""
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half a bfloat16 ulp at |x| (8 significant bits): 2^(floor(log2|x|) - 8), for x != 0."""
+    ax = np.maximum(np.abs(x), np.finfo(np.float64).tiny)
+    return np.ldexp(1.0, np.floor(np.log2(ax)).astype(np.int64) - 8)
+
+
+def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = "",
+                     outliers: bool = False):
+    """Max-abs and mean-abs error against the oracle, element by element.
+
+    bfloat16: every element within 2e-2, mean within 1e-3. With outliers=True (synthetic cases
+    only) elements with |reference| >= 8 may also be off by half a bfloat16 ulp of the
+    reference (the output format's own rounding there exceeds 2e-2), and the mean bound grows
+    by the mean of those half-ulps. Without it, no element may use the widened bound."""
     e = out_error(gpu, ref)
     t = tol_for(dtype)
-    bound = t["max_abs"]
-    if dtype == torch.bfloat16 and ref.size:
-        bound = np.maximum(t["max_abs"], np.abs(ref) * 2.0 ** -7)
-        e["n_bound_above_max_abs"] = int((np.abs(ref) * 2.0 ** -7 > t["max_abs"]).sum())
-        # reported, not asserted: the error against the oracle rounded to bf16 (what an exact
-        # bf16 kernel would return) and how many outputs exceed 8 in magnitude (where a bf16
-        # half-ulp alone is 0.031)
-        ref_b = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
-        e["max_abs_vs_bf16_ref"] = float(np.abs(gpu - ref_b).max())
-        e["n_ref_above_8"] = int((np.abs(ref) > 8).sum())
-    worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
-    # the mean bound grows the same way: elements above |reference| = 2.56 add their own share
-    # of the bf16 rounding, 2^-8 |reference| each (0 for the named workloads, whose outputs stay
-    # below 2.56)
+    bound = np.full(ref.shape, t["max_abs"])
     mean_bound = t["mean_abs"]
     if dtype == torch.bfloat16 and ref.size:
-        big = np.abs(ref) > 2.56
-        mean_bound += float((np.abs(ref) * 2.0 ** -8 * big).mean())
+        big = np.abs(ref) >= 8.0
+        e["n_ref_at_least_8"] = int(big.sum())
+        if outliers:
+            extra = np.where(big, bf16_half_ulp(ref), 0.0)
+            bound = bound + extra
+            mean_bound += float(extra.mean())
         e["mean_bound"] = mean_bound
+        # elements whose error needed more than the plain 2e-2
+        e["n_bound_above_max_abs"] = int((np.abs(gpu - ref) > t["max_abs"]).sum())
+        ref_b = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+        e["max_abs_vs_bf16_ref"] = float(np.abs(gpu - ref_b).max())
+    worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
     assert worst <= 0 and e["mean_abs"] <= mean_bound, (what, e, t)
+    if dtype == torch.bfloat16 and not outliers:
+        assert e["n_bound_above_max_abs"] == 0, (what, e)
     return e
+
+
+def gpu_csr(sel_idx, sel_cnt, B: int, Hq: int, nb: int, cap: int):
+    """The GPU's CSR as int32 numpy arrays [B, Hq, cap] and [B, Hq, nb]."""
+    gi = np.asarray(sel_idx.cpu() if torch.is_tensor(sel_idx) else sel_idx, dtype=np.int32)
+    gc = np.asarray(sel_cnt.cpu() if torch.is_tensor(sel_cnt) else sel_cnt, dtype=np.int32)
+    return (np.ascontiguousarray(gi.reshape(B, Hq, -1)[:, :, :cap]),
+            np.ascontiguousarray(gc.reshape(B, Hq, -1)[:, :, :nb]))
+
+
+def assert_prefill_out(out: torch.Tensor, cpu_inputs, block: int, ref_out: np.ndarray,
+                       ref_rows, res: dict, sel_idx, sel_cnt, off, dtype: torch.dtype,
+                       what: str = "", outliers: bool = False):
+    """Output check of an end-to-end call. ref_out[t] is the oracle's output for ref_rows[t]
+    on the oracle's selection. Rows whose GPU selection is a tie swap of the oracle's (listed
+    in res["rows_bad"] by compare_selection) are instead compared with the oracle's attention
+    over the GPU's own kept blocks. Returns (error on agreeing rows, error on swapped rows)."""
+    swapped = set(res["rows_bad"])
+    keep = [t for t, r in enumerate(ref_rows) if r not in swapped]
+    e1 = assert_out_close(out_rows(out, [ref_rows[t] for t in keep], block), ref_out[keep],
+                          dtype, what, outliers)
+    sw = [r for r in ref_rows if r in swapped]
+    e2 = None
+    if sw:
+        q, k, v = cpu_inputs
+        B, Hq, S_, _ = q.shape
+        nb = -(-S_ // block)
+        gi, gc = gpu_csr(sel_idx, sel_cnt, B, Hq, nb, int(off[nb]))
+        ref_sw = oracle.attention(q, k, v, block, gi, gc, off, sw)
+        e2 = assert_out_close(out_rows(out, sw, block), ref_sw, dtype, what + " (tie rows)",
+                              outliers)
+    return e1, e2

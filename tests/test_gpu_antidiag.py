@@ -134,11 +134,9 @@ def test_end_to_end(wname, stride, kw):
         si = sel_idx.cpu().numpy()[:, :, :int(ref["off"][-1])]
         for h in range(w.Hq):
             assert np.array_equal(si[:, h], si[:, (h // G) * G])
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, f"antidiag/{wname}")
+    parity.assert_prefill_out(out, cpu, w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, f"antidiag/{wname}")
 
 
 def test_stage_calls_match_the_full_path():
@@ -259,3 +257,10 @@ def test_full_size_sampled(w):
     ref_out = oracle.attention(qc, kc, vc, w.block, ref_idx, ref_cnt, off, keep)
     parity.assert_out_close(parity.out_rows(out, keep, w.block), ref_out, w.torch_dtype,
                             f"antidiag/{w.name}")
+    # rows whose selection is a near-tie swap: the oracle's attention over the GPU's own list
+    swapped = [r for r in rows if r not in set(keep)]
+    if swapped:
+        gi, gc = parity.gpu_csr(sel_idx, sel_cnt, w.B, w.Hq, w.nb, int(off[w.nb]))
+        ref_sw = oracle.attention(qc, kc, vc, w.block, gi, gc, off, swapped)
+        parity.assert_out_close(parity.out_rows(out, swapped, w.block), ref_sw, w.torch_dtype,
+                                f"antidiag/{w.name} (tie rows)")

@@ -152,11 +152,9 @@ def test_end_to_end(mname, wname):
                                    additive=_oracle_kwargs(mname)["metric_form"] == "additive")
     assert not res["violations"], res["violations"][:5]
     assert res["tie_swaps"] <= max(1, res["rows"] // 100), res
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, f"{mname}/{wname}")
+    parity.assert_prefill_out(out, cpu, w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, f"{mname}/{wname}")
 
 
 def test_stage_calls_with_method_match_the_full_path():

@@ -118,11 +118,9 @@ def test_end_to_end(name):
                                    ref["k"], ref["off"])
     assert not res["violations"], res["violations"][:5]
     assert res["tie_swaps"] <= max(1, res["rows"] // 100), res
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, name)
+    parity.assert_prefill_out(out, cpu, w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, name)
 
 
 @pytest.mark.parametrize("rho_min", [0.2, 1.0])
@@ -149,11 +147,10 @@ def test_scores_growing_after_the_first_block(rho_min):
     kept = [bool({16, 17} & set(oracle.row_list(ref["sel_idx"], ref["off"], ref["k"], 0, h, i)))
             for h in range(w.Hq) for i in range(18, w.nb)]
     assert sum(kept) >= (len(kept) if rho_min == 1.0 else len(kept) // 4), sum(kept)
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, "growth")
+    # synthetic large outputs: key blocks x6 with no sink make rows peaked on single x5 V rows
+    parity.assert_prefill_out(out, (q, k, v), w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, "growth", outliers=True)
 
 
 def test_dense_budget_matches_torch_sdpa():

@@ -82,8 +82,8 @@ def test_random_case(seed):
                                    ref["k"], ref["off"], rel=rel, additive=additive)
     assert not res["violations"], (w, md, res["violations"][:5])
     assert res["tie_swaps"] <= max(1, res["rows"] // 20), res
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, f"{w} {md}")
+    # the tiny workload's recipe: 16 x5 V rows per kv head in sequences of a few hundred
+    # tokens, so rows peaked on one outlier reach |out| > 8 (synthetic large outputs)
+    parity.assert_prefill_out(out, (q, k, v), w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, f"{w} {md}", outliers=True)

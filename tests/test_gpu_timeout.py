@@ -45,11 +45,9 @@ def test_expired_wait_reports_timeout_and_the_context_survives():
     res = parity.compare_selection(sel_idx, sel_cnt, ref["sel_idx"], ref["sel_cnt"], ref["m"],
                                    ref["k"], ref["off"])
     assert not res["violations"], res["violations"][:5]
-    swapped = set(res["rows_bad"])
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    keep = [t for t, r in enumerate(rows) if r not in swapped]
-    got = parity.out_rows(out, [rows[t] for t in keep], w.block)
-    parity.assert_out_close(got, ref["out"][keep], w.torch_dtype, "after timeout")
+    parity.assert_prefill_out(out, (q, k, v), w.block, ref["out"], rows, res, sel_idx, sel_cnt,
+                              ref["off"], w.torch_dtype, "after timeout")
 
 
 def test_estimator_expired_wait_reports_timeout_and_the_context_survives():

@@ -71,11 +71,9 @@ def test_varlen_matches_each_sequence(name):
                                        ref["k"], ref["off"], rel=rel,
                                        additive=md.get("metric") == "additive")
         assert not res["violations"], (L, res["violations"][:5])
-        swapped = set(res["rows_bad"])
         rows = [(0, h, i) for h in range(w.Hq) for i in range(nb)]
-        keep = [t for t, r in enumerate(rows) if r not in swapped]
-        parity.assert_out_close(parity.out_rows(g_out, [rows[t] for t in keep], w.block),
-                                ref["out"][keep], w.torch_dtype, f"{name} L={L}")
+        parity.assert_prefill_out(g_out, (qs, ks, vs), w.block, ref["out"], rows, res, g_si,
+                                  g_sc, ref["off"], w.torch_dtype, f"{name} L={L}")
         # bit for bit the single-sequence call
         o1, s1, c1 = S.stem_prefill_ex(qs.to(DEV), ks.to(DEV), vs.to(DEV), w.block, 0.0, 0.0, 0,
                                        method=m)
