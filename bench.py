@@ -14,8 +14,12 @@ both sides of exactly K timed steps, max over ranks. Inputs (1.61 GB) are larger
 126 MB L2, so no flush runs between steps. Per-stage durations come from four events the
 library records around its kernels inside the timed steps.
 
-N > 1 (torchrun): each rank runs its own independent problem (seed + rank) on its own GPU; no
-data-path collective (the path partitions by (batch, kv-head group)); weak scaling.
+N > 1 (torchrun): one problem split across the ranks by (batch, kv-head group) (partition.py):
+every rank builds the same seeded inputs and runs only its contiguous share of the (b, kv head)
+units, through the same C-ABI call on views of its heads; no data-path collective (a query
+head's pooling, selection and attention read only its own kv head); strong scaling, value =
+the whole problem's effective FLOPs over the slowest rank's time. --replicas instead runs an
+independent problem per rank (seed + rank), weak scaling.
 
 --impl reference: the CPU oracle (oracle/), as it stands, on this host's cores, on a bounded
 sample of the same workload per step (rank 0 only).
@@ -71,6 +75,9 @@ def parse():
                         "antidiag: the default with block probabilities by anti-diagonal "
                         "sampling (--stride tokens per group)")
     p.add_argument("--stride", type=int, default=16)
+    p.add_argument("--replicas", action="store_true",
+                   help="N > 1: an independent problem per rank (weak scaling) instead of one "
+                        "problem split across the ranks by kv-head group")
     p.add_argument("--no-context", action="store_true",
                    help="skip the context timing of dense causal attention (torch SDPA)")
     return p.parse_args()
@@ -303,8 +310,17 @@ def run_reference(args, world, rank):
 
 
 def rank_workload(w, rank: int):
-    """Each rank runs its own independent problem of the same shape (weak scaling)."""
+    """--replicas: each rank runs its own independent problem of the same shape (weak
+    scaling)."""
     return w.replace(seed=w.seed + rank)
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:
@@ -317,7 +333,8 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
 
 
 def whole_job_tflops(flop_per_rank: float, world: int, seconds: float) -> float:
-    """Throughput of the whole job: every rank's effective FLOPs over the slowest rank's time."""
+    """Throughput of the whole job: every rank's effective FLOPs over the slowest rank's time
+    (replicas: every rank does flop_per_rank)."""
     return world * flop_per_rank / seconds / 1e12
 
 
@@ -385,31 +402,40 @@ def run_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     mp = method_params(w, args.method, args.stride)
     meth = None if mp is None else S.make_method(**mp)
-    q, k, v = wl.make_inputs(rank_workload(w, rank), dev)
+    from block_sparse_causal_pooling_b200 import partition
+
+    replicas = args.replicas and world > 1
+    q, k, v = wl.make_inputs(rank_workload(w, rank) if replicas else w, dev)
     out, sel_idx, sel_cnt = S.alloc_outputs(q, k, w.block, w.rho_min, w.tau, w.k_min, meth)
-    ws = S.alloc_workspace(q, k, w.block, meth)
+    ws = S.alloc_workspace(q, k, w.block, meth)  # large enough for any segment of the problem
     if meth is None:
         kk, _ = S.stem_budget(w.nb, w.rho_min, w.tau, w.k_min)
     else:
         kk, _ = S.stem_budget_m(w.nb, meth)
     pairs = w.B * w.Hq * int(kk.sum())
-    flop = wl.effective_flops(pairs, w.block, w.D)
+    flop = wl.effective_flops(pairs, w.block, w.D)  # the whole problem
+    # this rank's calls: the whole problem (one rank, or replicas), else its segments
+    views = ([(q, k, v, out, sel_idx, sel_cnt)] if (world == 1 or replicas) else
+             list(partition.rank_views(q, k, v, out, sel_idx, sel_cnt, rank, world)))
+    rank_pairs = sum(t[0].shape[0] * t[0].shape[1] for t in views) * int(kk.sum())
     stream = torch.cuda.current_stream(dev)
 
     K, W = args.steps, args.warmup
     raw = RawEvents()
-    ev = [[raw.create() for _ in range(4)] for _ in range(K)]
-    args_warm = S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
-                            ws, method=meth)
-    call_args = [S.make_args(q, k, v, w.block, w.rho_min, w.tau, w.k_min, out, sel_idx, sel_cnt,
-                             ws, events=ev[s], method=meth) for s in range(K)]
+    ev = [[[raw.create() for _ in range(4)] for _ in views] for _ in range(K)]
+    args_warm = [S.make_args(*t[:3], w.block, w.rho_min, w.tau, w.k_min, *t[3:], ws, method=meth)
+                 for t in views]
+    call_args = [[S.make_args(*t[:3], w.block, w.rho_min, w.tau, w.k_min, *t[3:], ws,
+                              events=ev[s][c], method=meth) for c, t in enumerate(views)]
+                 for s in range(K)]
     lib = S.lib()
     hstream = S.ctypes.c_void_p(stream.cuda_stream)
 
-    def step(a):
-        rc = lib.stem_prefill_ex(S.ctypes.byref(a), hstream)
-        if rc != 0:
-            raise S.StemError(rc, "stem_prefill_ex")
+    def step(calls):
+        for a in calls:
+            rc = lib.stem_prefill_ex(S.ctypes.byref(a), hstream)
+            if rc != 0:
+                raise S.StemError(rc, "stem_prefill_ex")
 
     for _ in range(W):
         step(args_warm)
@@ -429,35 +455,45 @@ def run_ours(args, world, rank, local):
         torch.distributed.barrier()
     total_ms = start.elapsed_time(stop)
     stage_ms = {"pool": [], "select": [], "attn": []}
-    for s in range(K):
-        e = ev[s]
-        stage_ms["pool"].append(raw.elapsed_ms(e[0], e[1]))
-        stage_ms["select"].append(raw.elapsed_ms(e[1], e[2]))
-        stage_ms["attn"].append(raw.elapsed_ms(e[2], e[3]))
+    for s in range(K):  # a step's stage time: summed over this rank's calls
+        stage_ms["pool"].append(sum(raw.elapsed_ms(e[0], e[1]) for e in ev[s]))
+        stage_ms["select"].append(sum(raw.elapsed_ms(e[1], e[2]) for e in ev[s]))
+        stage_ms["attn"].append(sum(raw.elapsed_ms(e[2], e[3]) for e in ev[s]))
     raw.destroy()
     ms = max_over_ranks(total_ms / K, world, dev)
     clk = clocks.summary()
+    # the pooling kernel alone with a cold L2 (a 256 MB buffer written before each launch), so
+    # its bandwidth counts no bytes left in L2 by the previous step's attention
+    pool_cold_ms = pool_cold(S, views, w, meth, stream)
 
-    # end to end through the host-buffer entry point: pinned inputs in, output + CSR back
+    # end to end through the host-buffer entry point: pinned inputs in, output + CSR back (this
+    # rank's share of the problem)
     e2e = None
     if args.e2e_steps > 0:
-        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-        hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-        hsi = torch.empty(sel_idx.shape, dtype=torch.int32).pin_memory()
-        hsc = torch.empty(sel_cnt.shape, dtype=torch.int32).pin_memory()
-        S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc,
-                            method=meth)
+        hviews = [tuple(t.cpu().pin_memory() for t in vs[:3]) +
+                  (torch.empty(vs[3].shape, dtype=q.dtype).pin_memory(),
+                   torch.empty(vs[4].shape, dtype=torch.int32).pin_memory(),
+                   torch.empty(vs[5].shape, dtype=torch.int32).pin_memory()) for vs in views]
+
+        def host_step():
+            for hq, hk, hv, hout, hsi, hsc in hviews:
+                S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi,
+                                    hsc, method=meth)
+
+        host_step()
         if world > 1:
             torch.distributed.barrier()
         t0 = time.perf_counter()
         for _ in range(args.e2e_steps):
-            S.stem_prefill_host(hq, hk, hv, w.block, w.rho_min, w.tau, w.k_min, hout, hsi, hsc,
-                                method=meth)
+            host_step()
         e2e_s = max_over_ranks((time.perf_counter() - t0) / args.e2e_steps, world, dev)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-        d2h = sum(t.numel() * t.element_size() for t in (hout, hsi, hsc))
-        e2e = {"value": whole_job_tflops(flop, world, e2e_s), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        h2d = sum_over_ranks(sum(t.numel() * t.element_size() for hv_ in hviews
+                                 for t in hv_[:3]), world, dev)
+        d2h = sum_over_ranks(sum(t.numel() * t.element_size() for hv_ in hviews
+                                 for t in hv_[3:]), world, dev)
+        e2e = {"value": (whole_job_tflops(flop, world, e2e_s) if replicas else
+                         flop / e2e_s / 1e12), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": 1e3 * e2e_s}
 
     if rank != 0:
@@ -468,18 +504,26 @@ def run_ours(args, world, rank, local):
     sel_ms = statistics.mean(stage_ms["select"])
     long_region = total_ms > 1000.0
     peak_tf = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
-    achieved = flop / (attn_ms * 1e-3) / 1e12
+    # the dominant kernel's rate on this rank: its own share of the kept pairs
+    achieved = wl.effective_flops(rank_pairs, w.block, w.D) / (attn_ms * 1e-3) / 1e12
     elt = 2 if w.dtype == "bf16" else 4
-    pool_bytes = (w.B * (w.Hq + 2 * w.Hkv) * w.S * w.D * elt +
-                  4 * (w.B * (w.Hq + w.Hkv) * w.nb * w.D + w.B * w.Hkv * w.nb))
+    share = rank_pairs / pairs  # this rank's fraction of the (b, head) units
+    pool_bytes = share * (w.B * (w.Hq + 2 * w.Hkv) * w.S * w.D * elt +
+                          4 * (w.B * (w.Hq + w.Hkv) * w.nb * w.D + w.B * w.Hkv * w.nb))
     line = {
-        "metric": METRIC, "value": whole_job_tflops(flop, world, ms * 1e-3), "unit": "TFLOP/s",
+        "metric": METRIC,
+        "value": (whole_job_tflops(flop, world, ms * 1e-3) if replicas else
+                  flop / (ms * 1e-3) / 1e12), "unit": "TFLOP/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "scaling": "weak" if (replicas or world == 1) else "strong", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": f"synthetic, seeded ({w.name}: N(0,1) Q/K/V, RoPE theta {w.rope_theta}, K row 0 "
                 f"x{w.sink_scale}, {w.n_v_outliers()} V rows per kv-head x{w.v_outlier_scale}, "
                 f"heavy-tail fraction {w.heavy_tail_frac})",
         "config": dict(config_of(w, mp), kept_pairs=pairs, effective_tflop=flop / 1e12,
+                       parallelism=(f"replicas x{world}" if replicas else
+                                    f"kv-head-group partition over {world} rank(s), "
+                                    f"{len(views)} call(s) per step on rank 0"),
                        causal_exact_tflop=causal_exact_flops(w, kk) / 1e12,
                        causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
@@ -490,18 +534,24 @@ def run_ours(args, world, rank, local):
         "kernels": {
             "pool": {"ms": pool_ms, "bound": "hbm", "bytes": pool_bytes,
                      "GB/s": pool_bytes / (pool_ms * 1e-3) / 1e9,
-                     "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
-            "select": {"ms": sel_ms},
+                     "frac": pool_bytes / (pool_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "cold_l2": {"ms": pool_cold_ms,
+                                 "GB/s": pool_bytes / (pool_cold_ms * 1e-3) / 1e9,
+                                 "frac": pool_bytes / (pool_cold_ms * 1e-3) / 1e9 /
+                                 pk["hbm_gbs"],
+                                 "how": f"stem_pool alone, {POOL_COLD_REPS} launches, each "
+                                        "after writing a 256 MB buffer (L2 is 126 MB)"}},
+            "select": select_roofline(w, sel_ms, share, kk, clk, pk),
             "attn": {"ms": attn_ms, "tflops": achieved},
         },
         "clocks": clk,
-        "gpu_launches": KERNELS_PER_STEP * K,
+        "gpu_launches": KERNELS_PER_STEP * len(views) * K,
     }
     if mp is not None and mp.get("score") == "antidiag":
         # the estimator: 2 * stride*D FLOP per causal (query group, key group) pair; its time is
         # the "select" stage, which also holds the selection from p (a lower bound on its rate)
         nred = w.S // mp["stride"]
-        ad_flop = w.B * w.Hq * 2.0 * mp["stride"] * w.D * nred * (nred + 1) / 2
+        ad_flop = share * w.B * w.Hq * 2.0 * mp["stride"] * w.D * nred * (nred + 1) / 2
         ad_tf = ad_flop / (sel_ms * 1e-3) / 1e12
         line["kernels"]["select"].update({
             "what": "antidiag estimator + selection from p", "bound": "tensor",
@@ -509,7 +559,7 @@ def run_ours(args, world, rank, local):
             "estimator_traffic": antidiag_traffic(w.name, mp["stride"]),
             "estimator_algorithmic_bytes": 2 * w.B * (w.Hq + w.Hkv) * w.S * w.D +
                                            4 * w.B * w.Hq * w.nb * (w.nb + 1) // 2})
-        line["gpu_launches"] = (KERNELS_PER_STEP + 1) * K
+        line["gpu_launches"] = (KERNELS_PER_STEP + 1) * len(views) * K
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_context:
@@ -519,6 +569,53 @@ def run_ours(args, world, rank, local):
         line["cpu_baseline"]["extrapolated_full_workload_s"] = (
             flop / (line["cpu_baseline"]["value"] * 1e12))
     print(json.dumps(line), flush=True)
+
+
+POOL_COLD_REPS = 5
+# fp32 lanes per SM (4 sub-partitions x 32) and FLOP per fused multiply-add
+FP32_LANES_PER_SM = 128
+SM_COUNT = 148
+
+
+def pool_cold(S, views, w, meth, stream):
+    """Mean duration (ms) of the pooling stage of this rank's calls with L2 flushed first."""
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=stream.device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    bufs = [S.stem_pool(*vs[:3], w.block, stream=stream, method=meth) for vs in views]
+    times = []
+    for _ in range(POOL_COLD_REPS):
+        t = 0.0
+        for vs, b in zip(views, bufs):
+            flush.fill_(1)
+            e0.record(stream)
+            S.stem_pool(*vs[:3], w.block, *b, stream=stream, method=meth)
+            e1.record(stream)
+            torch.cuda.synchronize(stream.device)
+            t += e0.elapsed_time(e1)
+        times.append(t)
+    return statistics.mean(times)
+
+
+def select_roofline(w, sel_ms, share, kk, clk, pk):
+    """Roofline entry of the metric + top-k stage. Its arithmetic is the pooled score, 2*D FLOP
+    per causal (query block, key block) pair per query head, on the fp32 lanes (the bound the
+    kernel is designed against); the peak is 2 FLOP x 128 lanes x 148 SMs x the median SM clock
+    under load. Its bytes are the pooled inputs read and the CSR written."""
+    pairs_causal = share * w.B * w.Hq * w.nb * (w.nb + 1) / 2
+    flop = 2.0 * w.D * pairs_causal
+    cap = int(kk.sum())
+    bytes_ = share * (4 * w.B * (w.Hq + w.Hkv) * w.nb * w.D + 4 * w.B * w.Hkv * w.nb +
+                      4 * w.B * w.Hq * (cap + w.nb))
+    mhz = clk.get("sm_mhz") or 1965.0
+    peak = 2.0 * FP32_LANES_PER_SM * SM_COUNT * mhz * 1e6 / 1e12
+    tf = flop / (sel_ms * 1e-3) / 1e12
+    gbs = bytes_ / (sel_ms * 1e-3) / 1e9
+    return {"ms": sel_ms, "bound": "alu", "flop": flop, "tflops": tf,
+            "peak": peak, "peak_unit": "TFLOP/s fp32 FMA", "frac": tf / peak,
+            "bytes": bytes_, "GB/s": gbs, "hbm_frac": gbs / pk["hbm_gbs"],
+            "peak_derivation": f"2 x {FP32_LANES_PER_SM} fp32 lanes x {SM_COUNT} SMs x "
+                               f"{mhz:.0f} MHz (median SM clock under load)"}
 
 
 def causal_exact_flops(w, kk):

@@ -46,7 +46,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_agree_on_slowest_time_and_whole_job_value():
     world, port = 2, _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
