@@ -13,6 +13,8 @@ from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
+from oracle import build as oracle_build
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "stem_oracle.c")
 
@@ -92,8 +94,8 @@ def _check(mutant, tmp):
     lib = os.path.join(d, "libm.so")
     with open(csrc, "w") as f:
         f.write(src.replace(old, new))
-    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-w", "-o", lib, csrc, "-lm"],
-                   check=True)
+    flags = [f for f in oracle_build.CFLAGS if not f.startswith("-W")]  # as the oracle itself
+    subprocess.run(["gcc"] + flags + ["-w", "-o", lib, csrc, "-lm"], check=True)
     env = dict(os.environ, STEM_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-c", "from tests import pins; pins.run_all()"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
