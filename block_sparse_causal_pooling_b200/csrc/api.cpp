@@ -324,8 +324,10 @@ int enqueue_kernels(const stem_args_t* a, const stem_method_t& m, int nb, int64_
     rc = cuda_err(launch_select_p(p, vnorm, a->B, a->Hq, a->Hkv, nb, pd, cap, sel_metric(m),
                                   a->sel_idx, a->sel_cnt, nullptr, st));
   } else {
+    // the score triangles go to the schedule region, which the attention stage fills later
     rc = cuda_err(launch_select(qbar, kbar, vnorm, a->B, a->Hq, a->Hkv, nb, a->D, pd, cap,
-                                sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st));
+                                sel_metric(m), a->sel_idx, a->sel_cnt, nullptr, st,
+                                reinterpret_cast<float*>(ws + L.sched), L.sched_end - L.sched));
   }
   if (rc != STEM_OK) return rc;
   if ((rc = mark(2)) != STEM_OK) return rc;
@@ -670,8 +672,17 @@ int stem_select_m(const float* qbar, const float* kbar, const float* vnorm, int 
   PlanDev pd;
   rc = upload_plan(plan, workspace, L, st, &pd);
   if (rc != STEM_OK) return rc;
+  // a workspace of stem_workspace_size has room for score triangles after the plan; a smaller
+  // one (the plan only) runs the fused kernel, with the same selection
+  float* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (workspace_bytes >= L.sched_end) {
+    scratch = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + L.sched);
+    scratch_bytes = L.sched_end - L.sched;
+  }
   return cuda_err(launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, plan->cap,
-                                sel_metric(*m), sel_idx, sel_cnt, m_out, st));
+                                sel_metric(*m), sel_idx, sel_cnt, m_out, st, scratch,
+                                scratch_bytes));
 }
 
 int stem_antidiag_m(const void* q, const void* k, int dtype, int B, int Hq, int Hkv, int S, int D,

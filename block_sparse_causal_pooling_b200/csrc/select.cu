@@ -19,15 +19,22 @@
 // Kept set of row i: {0, i} plus the k(i)-2 largest key_ij over j in [1, i-1], larger first,
 // equal keys to the lower j. Written ascending into the CSR slot of row (b, h, i).
 //
-// Design: one CTA (8 warps) per (b, h, R consecutive query blocks).
-//   phase 1 - s for the R rows and every j < i0+R: a float32 SIMT tile product (kbar tiles of
-//             64 blocks staged in shared memory, qbar rows broadcast), kept in shared memory;
-//   phase 2 - one warp per row: an exact radix select on the 64-bit order-preserving image of
-//             key_ij (8-bit digits, starting at the highest bit where the row's keys differ),
-//             then an ascending ballot compaction that takes the threshold ties lowest-j first.
-// Rows never touch HBM except for the CSR they write (and m_out when requested).
+// Two designs compute the same selection from the same scores:
+//   split (the path's default, given scratch): score_tri_kernel writes s for the lower triangle
+//     of a chunk of heads into scratch (a tiled float32 SIMT product, 64 x 64 tiles, 4 x 4
+//     scores per thread), then select_s_kernel selects each row with one warp per row at high
+//     occupancy; the chunk's triangle (tens of MB) stays in L2 between the two;
+//   fused (no scratch; the allocation-free entry point): select_kernel, one CTA (8 warps) per
+//     (b, h, R consecutive query blocks): phase 1 computes s for its R rows into shared memory,
+//     phase 2 selects each row with one warp.
+// Every score is the same float32 multiply-add chain over d ascending in both, so both designs
+// select identically. The selection of a row: an exact radix select on the 64-bit
+// order-preserving image of key_ij (8-bit digits, starting at the highest bit where the row's
+// keys differ), then an ascending ballot compaction that takes the threshold ties lowest-j first.
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "stem_internal.h"
 
@@ -313,6 +320,147 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
     };
     select_row(i, kk, key_bits, hist, lane, dst, 0, 1);
   }
+}
+
+// ---- split design, step 1: pooled scores s_ij = qbar_i . kbar_j / sqrt(D) for j <= i of heads
+// [h0, h0 + nh) of the B*Hq, into tri[(head - h0) * nb(nb+1)/2 + i(i+1)/2 + j]. One CTA per 64 x 64
+// tile of (i, j) with the j tile at most the i tile; each thread holds the 4 x 4 scores of rows
+// ty + 16a and columns tx + 16b (a, b < 4) of the tile, both tiles' pooled rows staged in shared
+// memory (row stride D + 4 floats: the 16 columns a warp reads at one d fall in distinct banks).
+constexpr int kScT = 64;
+
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) score_tri_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar, int Hq, int Hkv, int nb,
+    int h0, int tiles_per_head, float* __restrict__ tri) {
+  constexpr int LD = D + 4;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qs = reinterpret_cast<float*>(smem_raw);
+  float* ks = qs + kScT * LD;
+  const int hl = static_cast<int>(blockIdx.x) / tiles_per_head;
+  const int t = static_cast<int>(blockIdx.x) % tiles_per_head;
+  // t -> (ti, tj), tj <= ti, tiles of the lower triangle numbered row by row
+  int ti = static_cast<int>((sqrtf(8.0f * static_cast<float>(t) + 1.0f) - 1.0f) * 0.5f);
+  while (ti * (ti + 1) / 2 > t) --ti;
+  while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+  const int tj = t - ti * (ti + 1) / 2;
+  const int64_t bh = static_cast<int64_t>(h0) + hl;
+  const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
+  const int G = Hq / Hkv;
+  const float* qsrc = qbar + bh * nb * D;
+  const float* ksrc = kbar + (static_cast<int64_t>(b) * Hkv + h / G) * nb * D;
+  const int i0 = ti * kScT, j0 = tj * kScT;
+  for (int idx = threadIdx.x; idx < kScT * D / 4; idx += kSelThreads) {
+    const int r = idx / (D / 4), c4 = idx % (D / 4);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+    if (i0 + r < nb) a = reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(i0 + r) * D)[c4];
+    if (j0 + r < nb) c = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j0 + r) * D)[c4];
+    *reinterpret_cast<float4*>(qs + r * LD + 4 * c4) = a;
+    *reinterpret_cast<float4*>(ks + r * LD + 4 * c4) = c;
+  }
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 2
+  for (int d = 0; d < D; d += 4) {
+    float4 qv[4], kv[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qs + (ty + 16 * a) * LD + d);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(ks + (tx + 16 * c) * LD + d);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[a][c] = fmaf(qv[a].x, kv[c].x, acc[a][c]);
+        acc[a][c] = fmaf(qv[a].y, kv[c].y, acc[a][c]);
+        acc[a][c] = fmaf(qv[a].z, kv[c].z, acc[a][c]);
+        acc[a][c] = fmaf(qv[a].w, kv[c].w, acc[a][c]);
+      }
+  }
+  const float scale = rsqrtf(static_cast<float>(D));  // as in select_kernel
+  float* dst = tri + static_cast<int64_t>(hl) * (static_cast<int64_t>(nb) * (nb + 1) / 2);
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty + 16 * a;
+    if (i >= nb) continue;
+    const int64_t rowoff = static_cast<int64_t>(i) * (i + 1) / 2;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + tx + 16 * c;
+      if (j <= i) dst[rowoff + j] = acc[a][c] * scale;
+    }
+  }
+}
+
+// ---- split design, step 2: the selection of every row of heads [h0, h0 + nh) from their score
+// rows in tri (written by score_tri_kernel). One CTA (8 warps) per (head, 8 consecutive query
+// blocks), heaviest rows first, one row per warp; the per-column term of the key (ln n_j, or
+// beta * e_j for the additive form) in shared memory. m_out as select_kernel writes it.
+__global__ void __launch_bounds__(kSelThreads) select_s_kernel(
+    const float* __restrict__ tri, const float* __restrict__ vnorm, int Hq, int Hkv, int nb,
+    int h0, int nh, PlanDev plan, int64_t cap, SelMetric metric, int32_t* __restrict__ sel_idx,
+    int32_t* __restrict__ sel_cnt, float* __restrict__ m_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int ldS = (nb + 3) & ~3;
+  double* lnn = reinterpret_cast<double*>(smem_raw);                      // [ldS]
+  int* hist_all = reinterpret_cast<int*>(lnn + ldS);                      // [kWarps][256]
+  const int ntiles = (nb + kWarps - 1) / kWarps;
+  const int tile = ntiles - 1 - static_cast<int>(blockIdx.x / nh);  // heaviest rows first
+  const int sh = static_cast<int>(blockIdx.x % nh);
+  const int64_t bh = static_cast<int64_t>(h0) + sh;
+  const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
+  const int G = Hq / Hkv;
+  const int i0 = tile * kWarps;
+  const int rows = min(kWarps, nb - i0);
+  const int jend = i0 + rows;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const float* nsrc = vnorm + (static_cast<int64_t>(b) * Hkv + h / G) * nb;
+  const int64_t trisz = static_cast<int64_t>(nb) * (nb + 1) / 2;
+  for (int j = t; j < jend; j += kSelThreads) {
+    double c;
+    if (!metric.additive) {
+      c = log(static_cast<double>(nsrc[j]));
+    } else if (metric.beta == 0.f) {
+      c = 0.0;
+    } else {
+      double e = 2.0 * log(static_cast<double>(nsrc[j]));
+      if (metric.clamp && e < 0.0) e = 0.0;
+      c = static_cast<double>(metric.beta) * e;
+    }
+    lnn[j] = c;
+  }
+  __syncthreads();
+  if (warp >= rows) return;  // no __syncthreads below
+  const int i = i0 + warp;
+  const int kk = plan.k[i];
+  const int64_t rowoff = static_cast<int64_t>(i) * (i + 1) / 2;
+  const float* srow = tri + static_cast<int64_t>(sh) * trisz + rowoff;
+  int* hist = hist_all + warp * 256;
+  if (lane == 0) sel_cnt[bh * nb + i] = kk;
+  if (m_out != nullptr && metric.additive) {  // diagnostic metric row: M_ij = s_ij + beta e_j
+    for (int j = lane; j <= i; j += 32)
+      m_out[bh * trisz + rowoff + j] = static_cast<float>(static_cast<double>(srow[j]) + lnn[j]);
+  } else if (m_out != nullptr) {  // diagnostic metric row, float32 softmax
+    float mx = -INFINITY;
+    for (int j = lane; j <= i; j += 32) mx = fmaxf(mx, srow[j]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float z = 0.f;
+    for (int j = lane; j <= i; j += 32) z += expf(srow[j] - mx);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    for (int j = lane; j <= i; j += 32)
+      m_out[bh * trisz + rowoff + j] = expf(srow[j] - mx) / z * nsrc[j];
+  }
+  auto key_bits = [&](int j) -> uint64_t {
+    return order_bits(static_cast<double>(__ldg(srow + j)) + lnn[j]);
+  };
+  select_row(i, kk, key_bits, hist, lane, sel_idx + bh * cap + plan.off[i], 0, 1);
 }
 
 // ---- GQA-group-shared selection: one kept list per (b, kv-head group, query block), chosen by
@@ -650,11 +798,54 @@ cudaError_t launch_select_p(const float* p, const float* vnorm, int B, int Hq, i
                          st);
 }
 
+// The split design over chunks of heads whose score triangles fit the scratch.
+template <int D>
+cudaError_t launch_split(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
+                         int Hkv, int nb, PlanDev plan, int64_t cap, SelMetric metric,
+                         int32_t* sel_idx, int32_t* sel_cnt, float* m_out, float* scratch,
+                         int chunk, cudaStream_t st) {
+  const int nt = (nb + kScT - 1) / kScT;
+  const int tiles = nt * (nt + 1) / 2;
+  const size_t smem1 = sizeof(float) * 2 * kScT * (D + 4);
+  const size_t smem2 = sizeof(double) * ((nb + 3) & ~3) + sizeof(int) * kWarps * 256;
+  cudaError_t e = cudaFuncSetAttribute(score_tri_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem1));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(select_s_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem2));
+  if (e != cudaSuccess) return e;
+  const int heads = B * Hq;
+  for (int h0 = 0; h0 < heads; h0 += chunk) {
+    const int nh = std::min(chunk, heads - h0);
+    const int64_t g1 = static_cast<int64_t>(nh) * tiles;
+    const int64_t g2 = static_cast<int64_t>(nh) * ((nb + kWarps - 1) / kWarps);
+    if (g1 > 0x7fffffff || g2 > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    score_tri_kernel<D><<<static_cast<unsigned>(g1), kSelThreads, smem1, st>>>(
+        qbar, kbar, Hq, Hkv, nb, h0, tiles, scratch);
+    select_s_kernel<<<static_cast<unsigned>(g2), kSelThreads, smem2, st>>>(
+        scratch, vnorm, Hq, Hkv, nb, h0, nh, plan, cap, metric, sel_idx, sel_cnt, m_out);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
                           SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* scratch, size_t scratch_bytes) {
   if (B * Hq == 0 || nb == 0) return cudaSuccess;
+  const size_t tri_bytes = sizeof(float) * (static_cast<size_t>(nb) * (nb + 1) / 2);
+  const int64_t chunk = scratch ? static_cast<int64_t>(scratch_bytes / tri_bytes) : 0;
+  if (!(metric.group && Hq != Hkv) && chunk >= 1) {
+    const int c = static_cast<int>(std::min<int64_t>(chunk, static_cast<int64_t>(B) * Hq));
+    if (D == 128)
+      return launch_split<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                               sel_cnt, m_out, scratch, c, st);
+    if (D == 64)
+      return launch_split<64>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,
+                              sel_cnt, m_out, scratch, c, st);
+    return cudaErrorInvalidValue;
+  }
   if (metric.group && Hq != Hkv) {
     if (D == 128)
       return launch_group<128>(qbar, kbar, vnorm, B, Hq, Hkv, nb, plan, cap, metric, sel_idx,

@@ -33,11 +33,14 @@ struct SelMetric {
 // Largest nb the group-shared selection supports (its per-CTA key rows live in shared memory).
 constexpr int kGroupMaxNb = 1024;
 
-// Metric + top-k selection (select.cu).
+// Metric + top-k selection (select.cu). With scratch (at least one head's score triangle,
+// 4*nb*(nb+1)/2 bytes) and per-head selection it runs as two kernels, scores then selection,
+// over chunks of heads; otherwise (scratch NULL, or group share) as one fused kernel. Both give
+// the same selection.
 cudaError_t launch_select(const float* qbar, const float* kbar, const float* vnorm, int B,
                           int Hq, int Hkv, int nb, int D, PlanDev plan, int64_t cap,
                           SelMetric metric, int32_t* sel_idx, int32_t* sel_cnt, float* m_out,
-                          cudaStream_t st);
+                          cudaStream_t st, float* scratch = nullptr, size_t scratch_bytes = 0);
 
 // Block probabilities by anti-diagonal sampling (antidiag_sm100.cu), bf16 inputs, D 64 or 128,
 // stride | block, stride | S, block/stride a power of two <= 32. p: [B*Hq][nb*(nb+1)/2] rows of
