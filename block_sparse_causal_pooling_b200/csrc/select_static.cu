@@ -12,9 +12,17 @@
 // needs 49,156 bytes); larger requests are rejected with STEM_ERR_UNSUPPORTED.
 //
 // The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
-// that device current; that first call should come before any stream capture. Every call
-// shares the array and rewrites the whole plan it uses (nothing needs to start at zero), so
-// calls whose kernels overlap on the GPU race on it: issue them in stream order.
+// that device current; that first call should come before any stream capture. The address is
+// looked up again only when the device's context changes (after a cudaDeviceReset the module
+// is loaded anew and the array has a new address). Every call shares the array and rewrites
+// the whole plan it uses (nothing needs to start at zero), so calls whose kernels overlap on
+// the GPU race on it: issue them in stream order.
+//
+// The plan reaches the array without a host-to-device copy: the host builds it and passes it
+// by value as the parameters of a small kernel (at most two launches of 32,000 bytes), which
+// writes it into the array. Launch parameters are copied when the launch is made, so nothing a
+// later call does on the host can change what an earlier call's kernels read.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -31,10 +39,55 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) int32_t g_static_plan[kStaticPlanBytes / sizeof(int32_t)];
 
+// One launch's share of the plan, passed by value (kernel parameters may take 32,764 bytes).
+constexpr int kChunkInts = 8000;
+struct PlanChunk {
+  int32_t v[kChunkInts];
+};
+static_assert(sizeof(PlanChunk) + 2 * sizeof(int) <= 32764, "kernel parameter limit");
+
+__global__ void write_plan_kernel(const PlanChunk c, int start, int n) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x)
+    g_static_plan[start + t] = c.v[t];
+}
+
 std::mutex g_static_mu;
+// per device: the array's address and the unique ID of the context it was looked up in
 void* g_static_addr[kMaxDevices] = {nullptr};
-// host image of the plan, rebuilt under the mutex by every call
-int32_t g_host_plan[kStaticPlanBytes / sizeof(int32_t)];
+unsigned long long g_static_ctx[kMaxDevices] = {0};
+// host scratch of the plan (3 * STEM_MAX_NB + 1 int32 fit in two chunks), rebuilt under the
+// mutex by every call; its bytes travel in the launch parameters
+PlanChunk g_host_chunks[2];
+static_assert(2 * kChunkInts >= 3 * STEM_MAX_NB + 1, "plan fits two chunks");
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID (for the life of the process) of the calling thread's current context; 0 if the
+// driver cannot say.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 bool aligned_to(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
 
@@ -67,34 +120,38 @@ extern "C" int stem_select_static(const float* qbar, const float* kbar, const fl
     return STEM_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_addr[dev] == nullptr) {  // once per device, with that device current
+  const unsigned long long ctx = current_ctx_id();  // 0 before the runtime made one current
+  if (g_static_addr[dev] == nullptr || ctx == 0 || ctx != g_static_ctx[dev]) {
+    // once per device (and again after its context changed), with that device current
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_plan) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
       return STEM_ERR_CUDA;
     }
     g_static_addr[dev] = p;
+    g_static_ctx[dev] = current_ctx_id();  // the lookup made the device's context current
   }
-  int32_t* k = g_host_plan;
+  // the plan in the two host chunks, as one array: k | off | order
+  int32_t plan[2 * kChunkInts];
+  int32_t* k = plan;
   int32_t* off = k + nb;
   int32_t* order = off + nb + 1;
   if (stem_budget(nb, rho_min, tau, k_min, k, off) != STEM_OK) return STEM_ERR_ARG;
   for (int i = 0; i < nb; ++i) order[i] = i;
   // heaviest rows first; equal budgets: later rows first (a total order: no ties)
   std::sort(order, order + nb, [&](int a, int b) { return k[a] != k[b] ? k[a] > k[b] : a > b; });
-
+  const int n_ints = 3 * nb + 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // pageable source: the call returns after the bytes are staged, so the host image is free
-  // for the next call as soon as this one returns
-  if (cudaMemcpyAsync(g_static_addr[dev], g_host_plan, plan_bytes, cudaMemcpyHostToDevice, st) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return STEM_ERR_CUDA;
+  for (int start = 0, c = 0; start < n_ints; start += kChunkInts, ++c) {
+    const int n = std::min(kChunkInts, n_ints - start);
+    std::copy(plan + start, plan + start + n, g_host_chunks[c].v);
+    write_plan_kernel<<<(n + 255) / 256, 256, 0, st>>>(g_host_chunks[c], start, n);
+    if (cudaGetLastError() != cudaSuccess) return STEM_ERR_CUDA;
   }
   const int32_t* dk = static_cast<const int32_t*>(g_static_addr[dev]);
   PlanDev pd{dk, dk + nb, dk + 2 * nb + 1};
-  const cudaError_t e = launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, cap, SelMetric{}, sel_idx,
-                                      sel_cnt, nullptr, st);
+  const cudaError_t e = launch_select(qbar, kbar, vnorm, B, Hq, Hkv, nb, D, pd, cap,
+                                      SelMetric{}, sel_idx, sel_cnt, nullptr, st);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return STEM_ERR_CUDA;

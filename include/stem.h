@@ -239,7 +239,11 @@ int stem_pool(const void* q, const void* k, const void* v, int dtype, int B, int
  * in double; ties go to the lower block index.
  * m_out: optional (NULL to skip) float32 [B,Hq,nb*(nb+1)/2], row i at offset i*(i+1)/2, the
  * metric m_ij for j <= i (softmax over j <= i in float32).
- * workspace: as for stem_prefill_ex (only the plan region is used).
+ * workspace: as for stem_prefill_ex. Given stem_workspace_size bytes, the scores s_ij of the
+ * lower triangle are written to the workspace region after the plan (a chunk of heads at a
+ * time) and the rows are selected from there by a second kernel; given only the plan region
+ * (smaller workspaces down to that size are accepted), one fused kernel computes the same
+ * scores in shared memory. Both select identically.
  */
 int stem_select(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
                 int Hkv, int nb, int D, float rho_min, float tau, int k_min, int32_t* sel_idx,
@@ -357,9 +361,13 @@ int64_t stem_varlen_sel_capacity(int nseq, const int32_t* cu_seqlens, int block,
  * kernel's scratch, the budget plan (3*nb+1 int32), lives in a 64 KiB file-scope device array
  * that every GPU loading the library holds until the process exits. Inputs and outputs are
  * those of stem_select (no m_out). nb beyond STEM_MAX_NB returns STEM_ERR_UNSUPPORTED.
- * The first call on a device looks the array up (with that device current); make it before
- * any stream capture. All calls share the array: calls whose kernels overlap on the GPU race,
- * so issue them in stream order. Same errors as stem_select, except that there is no workspace.
+ * The first call on a device looks the array up (with that device current), and so does the
+ * first call after the device's context changed (a cudaDeviceReset loads the library's device
+ * code anew); make such a call before any stream capture. The plan goes to the array as the
+ * launch parameters of a small kernel (no host-to-device copy, so no host buffer that a later
+ * call could rewrite). All calls share the device array: calls whose kernels overlap on the GPU
+ * race, so issue them in stream order. Same errors as stem_select, except that there is no
+ * workspace.
  */
 int stem_select_static(const float* qbar, const float* kbar, const float* vnorm, int B, int Hq,
                        int Hkv, int nb, int D, float rho_min, float tau, int k_min,
