@@ -63,6 +63,9 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float bf16r(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -209,8 +212,9 @@ __global__ void __launch_bounds__(BLOCK * 2) attn_bf16_mma_kernel(
       float sum = 0.f;
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
-        const float p0 = ex2(s[n][2 * hr] * sl2 - muse);
-        const float p1 = ex2(s[n][2 * hr + 1] * sl2 - muse);
+        // P rounded to bf16 here, so the row sum takes the same values that enter P V
+        const float p0 = bf16r(ex2(s[n][2 * hr] * sl2 - muse));
+        const float p1 = bf16r(ex2(s[n][2 * hr + 1] * sl2 - muse));
         s[n][2 * hr] = p0;
         s[n][2 * hr + 1] = p1;
         sum += p0 + p1;

@@ -138,6 +138,19 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// tcgen05.wait::ld that also names the 32 registers of a TC_LD32 as read and written, so the
+// compiler cannot move a use of them above the wait (the load writes them asynchronously).
+__device__ __forceinline__ void tc_wait_ld_r32(uint32_t* r) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 __device__ __forceinline__ void tc_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -156,6 +169,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
   d |= 1ull << 46;
   d |= 2ull << 61;
   return d;
+}
+// The same descriptor split into its two 32-bit words: the low word holds the start address
+// and the leading byte offset, the high word the stride byte offset, the version and the
+// layout. Adding a multiple of 16 bytes to an address adds (bytes >> 4) to the low word, with
+// no carry while the address stays below 256 KB (all of shared memory).
+__host__ __device__ constexpr uint32_t smem_desc_lo(uint32_t addr, uint32_t lbo) {
+  return ((addr >> 4) & 0x3fffu) | (((lbo >> 4) & 0x3fffu) << 16);
+}
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3fffu) | (1u << 14) | (2u << 29);
 }
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, A K-major, B K- or MN-major.
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool b_mn_major) {
