@@ -43,13 +43,15 @@ sys.path.insert(0, ROOT)
 from block_sparse_causal_pooling_b200 import workloads as wl  # noqa: E402
 
 METRIC = "Stem prefill attention latency (ms) & effective TFLOP/s at S=128K, % of BF16 peak"
-# library kernels per step: pooling, metric + selection, head-pair schedule, attention
-KERNELS_PER_STEP = 4
+# library kernels per call: pooling, head-pair schedule, attention, and two per chunk of heads for
+# the selection (scores, then the selection from them); select_chunks() counts the chunks
+KERNELS_PER_CALL = 3
+SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615398912 + 1023005184,
-                "sources_sha256": "1441e55fb9487896d62f3b2102b2ee71d65da1e8c83734d6fe9433e1b85f8c55"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615687168 + 1021676032,
+                "sources_sha256": "1f6e9fcd47619c5d4f09c6ecdb805e5904cdfe10ffad7825983ebd96bfeaab5c"}
 # The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,
@@ -309,6 +311,32 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ multi-rank helpers
 
 
+def select_chunks(B: int, Hq: int, Hkv: int, nb: int) -> int:
+    """Chunks of heads the selection stage runs in: the workspace region it shares with the
+    head-pair schedule holds every head's score triangle up to SCORE_CAP bytes, and at least
+    the schedule's size (as laid out by the library's stem_workspace_size)."""
+    tri = 4 * nb * (nb + 1) // 2
+    G = Hq // Hkv
+    sched = 256 + 4 * B * Hkv * ((G + 1) // 2) * (nb * (nb + 1) // 2)
+    region = -(-max(sched, min(tri * B * Hq, SCORE_CAP)) // 256) * 256
+    per = max(1, region // tri)
+    return -(-(B * Hq) // per)
+
+
+def launches_per_call(w, views, mp=None) -> int:
+    """Library kernels one stem_prefill_ex call launches, per segment view."""
+    n = 0
+    for vs in views:
+        B, Hq, Hkv = vs[0].shape[0], vs[0].shape[1], vs[1].shape[1]
+        if mp is not None and mp.get("score") == "antidiag":
+            n += KERNELS_PER_CALL + 2  # estimator + selection from p
+        elif mp is not None and mp.get("share") == "group" and Hq != Hkv:
+            n += KERNELS_PER_CALL + 1  # one fused group-selection kernel
+        else:
+            n += KERNELS_PER_CALL + 2 * select_chunks(B, Hq, Hkv, w.nb)
+    return n
+
+
 def rank_workload(w, rank: int):
     """--replicas: each rank runs its own independent problem of the same shape (weak
     scaling)."""
@@ -545,7 +573,7 @@ def run_ours(args, world, rank, local):
             "attn": {"ms": attn_ms, "tflops": achieved},
         },
         "clocks": clk,
-        "gpu_launches": KERNELS_PER_STEP * len(views) * K,
+        "gpu_launches": launches_per_call(w, views, mp) * K,
     }
     if mp is not None and mp.get("score") == "antidiag":
         # the estimator: 2 * stride*D FLOP per causal (query group, key group) pair; its time is
@@ -559,7 +587,7 @@ def run_ours(args, world, rank, local):
             "estimator_traffic": antidiag_traffic(w.name, mp["stride"]),
             "estimator_algorithmic_bytes": 2 * w.B * (w.Hq + w.Hkv) * w.S * w.D +
                                            4 * w.B * w.Hq * w.nb * (w.nb + 1) // 2})
-        line["gpu_launches"] = (KERNELS_PER_STEP + 1) * len(views) * K
+
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_context:

@@ -24,6 +24,7 @@ namespace stem {
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr size_t kScoreCap = 128ull << 20;  // most bytes of score triangles in the workspace
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ budget
@@ -172,8 +173,13 @@ Layout layout(int B, int Hq, int Hkv, int nb, int D, const stem_method_t* m = nu
   o += kAlign;
   L.plan = o;
   o += plan_bytes(nb);
+  // The head-pair schedule (attention stage) and the selection's score triangles (selection
+  // stage, before it) share one region: every head's triangle up to 128 MB, at least the
+  // schedule's size (the selection then runs over chunks of heads).
   L.sched = o;
-  o += align_up(pairs_bytes(B, Hq, Hkv, nb));
+  const size_t tri = sizeof(float) * static_cast<size_t>(nb) * (nb + 1) / 2;
+  const size_t scores = std::min(tri * static_cast<size_t>(B) * Hq, kScoreCap);
+  o += align_up(std::max(pairs_bytes(B, Hq, Hkv, nb), scores));
   L.sched_end = o;
   L.qbar = o;
   o += align_up(sizeof(float) * static_cast<size_t>(B) * Hq * nb * D);

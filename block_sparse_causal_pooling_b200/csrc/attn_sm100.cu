@@ -10,10 +10,12 @@
 // Work item: two GQA sibling heads A and B at one query block, which keep the same number of key
 // blocks; a step schedule (pairs.cu) pairs their lists so a block both keep is one K/V tile.
 //
-// Persistent kernel, one CTA per SM, 10 warps:
-//   warp 0      TMA producer: Q_A, Q_B (one tile each) and K/V tiles into a 4-slot ring of
-//               128B-swizzled shared-memory tiles (boxes of 128 rows x 64 columns), filled in the
-//               order the products first use them.
+// Persistent kernel, one CTA per SM, 10 warps. Work items are claimed at run time from a global
+// counter in heavy-first order (the producer claims, the other roles read the claimed indices
+// from a ring in shared memory), so the CTAs finish together.
+//   warp 0      TMA producer: claims items; Q_A, Q_B (one tile each) and K/V tiles into a 4-slot
+//               ring of 128B-swizzled shared-memory tiles (boxes of 128 rows x 64 columns),
+//               filled in the order the products first use them.
 //   warp 1      allocates the 512 TMEM columns; lane 0 issues every tcgen05.mma:
 //                 S_T = Q_T K^T     (M 128, N 128, K = D; A and B K-major in shared memory)
 //                 O_T += P_T V      (A = P read from TMEM over the first half of S_T, B = V
@@ -24,9 +26,9 @@
 //               32*(w%4).. and take 64 columns each; tcgen05.ld 32x32b): row max (halves
 //               exchanged through shared memory at a barrier of the warp pair that also makes
 //               both warps agree on going on, so an abort cannot strand one), exp2 with the
-//               1/sqrt(D) scale folded in, per-thread partial row sums in fp32 (f32x2
-//               arithmetic); P packed to bf16 and stored over the first half of S_T
-//               (tcgen05.st). Only an item's first step takes the exact row max; later steps
+//               1/sqrt(D) scale folded in; P packed to bf16 and stored over the first half of
+//               S_T (tcgen05.st); the per-thread partial row sums add the bf16 values that
+//               enter P V, in fp32. Only an item's first step takes the exact row max; later steps
 //               use it as the reference and fall back to the exact max, an O rescale in TMEM
 //               and a recompute only when a partial row sum reaches 2^16 (exact: the final
 //               1/l uses the same reference as P). At an item's end: O * (1/l) -> bf16 ->
@@ -43,12 +45,14 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <atomic>
 #include <mutex>
 
 #include "sm100.cuh"
 #include "stem.h"
 #include "stem_internal.h"
+
 
 namespace stem {
 
@@ -70,6 +74,8 @@ constexpr int kSlots = 4;           // K/V ring slots
 constexpr int kThreads = 320;       // 10 warps
 constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kItemRing = 8;                       // claimed work items in flight
+constexpr int kItemReaders = 1 + kSoftmaxThreads;  // MMA thread and softmax threads
 
 template <int D>
 struct Cfg {
@@ -83,6 +89,8 @@ struct __align__(8) Bars {
   uint64_t kv_full[kSlots], kv_empty[kSlots];
   uint64_t s_full[2], p_full[2];             // per tile
   uint64_t o_full[2], o_empty[2];            // per tile
+  uint64_t iq_full[kItemRing], iq_empty[kItemRing];  // claimed items, producer -> readers
+  int64_t iq[kItemRing];                     // item index, or -1: none left
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
@@ -139,15 +147,6 @@ __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return r;
 }
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  f2 r;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
-}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -158,57 +157,62 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Eight products of one group issued back to back from one asm block, their descriptors
-// computed beforehand: one predicate for the first product's accumulate flag and a
-// constant-true one for the other seven. The issuing thread's instructions between products
-// leave the tensor pipe idle (the MMA queue does not hide them), so they are kept to none.
-// operands: %0 d, %1..%8 a[0..7], %9..%16 b[0..7], %17 acc0, %18 idesc
-__device__ __forceinline__ void mma_ss8(uint32_t d, const uint64_t* a, const uint64_t* b,
-                                        uint32_t idesc, uint32_t acc0) {
+// Products of one group issued back to back from one asm block. Every descriptor is a base
+// word plus an immediate offset, so the issuing thread spends one add per product between
+// tcgen05.mma instructions: its instructions between products leave the tensor pipe idle (the
+// MMA queue does not hide them), so they are kept to these.
+//
+// S group: S = Q K^T over the D/16 k-steps, both operands K-major 128B-swizzled tiles in shared
+// memory (boxes of 128 rows x 64 columns, 16 KB apart; a k-step is 32 bytes): k-step kk is at
+// descriptor offset (kk / 4) * 1024 + (kk % 4) * 2. The first product overwrites D.
+// operands: %0 d, %1 a_lo, %2 b_lo, %3 hi, %4 idesc
+#define STEM_MMA_SS(OFF)                                                                   \
+  "add.u32 x, %1, " #OFF ";\n\tadd.u32 y, %2, " #OFF ";\n\t"                               \
+  "mov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"                                        \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, pt;\n\t"
+__device__ __forceinline__ void mma_s8(uint32_t d, uint32_t alo, uint32_t blo, uint32_t hi,
+                                       uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p0, p1;\n\t"
-      "setp.ne.b32 p0, %17, 0;\n\t"
-      "setp.eq.b32 p1, %17, %17;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %18, p0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %18, p1;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %18, p1;\n\t}" ::"r"(d),
-      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]),
-      "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]),
-      "r"(acc0), "r"(idesc)
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 x, y;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 pf, %4, %4;\n\tsetp.eq.b32 pt, %4, %4;\n\t"
+      "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, pf;\n\t"
+      STEM_MMA_SS(2) STEM_MMA_SS(4) STEM_MMA_SS(6) STEM_MMA_SS(1024) STEM_MMA_SS(1026)
+      STEM_MMA_SS(1028) STEM_MMA_SS(1030) "}" ::"r"(d), "r"(alo), "r"(blo), "r"(hi), "r"(idesc)
       : "memory");
 }
-// The same with A from TMEM: product k reads P at column a0 + 8k.
-// operands: %0 d, %1 a0, %2..%9 b[0..7], %10 acc0, %11 idesc
-__device__ __forceinline__ void mma_ts8(uint32_t d, uint32_t a0, const uint64_t* b,
-                                        uint32_t idesc, uint32_t acc0) {
+__device__ __forceinline__ void mma_s4(uint32_t d, uint32_t alo, uint32_t blo, uint32_t hi,
+                                       uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 a;\n\t"
-      "setp.ne.b32 p0, %10, 0;\n\t"
-      "setp.eq.b32 p1, %10, %10;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %11, p0;\n\t"
-      "add.u32 a, %1, 8;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %3, %11, p1;\n\t"
-      "add.u32 a, %1, 16;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %4, %11, p1;\n\t"
-      "add.u32 a, %1, 24;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %5, %11, p1;\n\t"
-      "add.u32 a, %1, 32;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %6, %11, p1;\n\t"
-      "add.u32 a, %1, 40;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %7, %11, p1;\n\t"
-      "add.u32 a, %1, 48;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %8, %11, p1;\n\t"
-      "add.u32 a, %1, 56;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], %9, %11, p1;\n\t}" ::"r"(d),
-      "r"(a0), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]),
-      "l"(b[7]), "r"(acc0), "r"(idesc)
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 x, y;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 pf, %4, %4;\n\tsetp.eq.b32 pt, %4, %4;\n\t"
+      "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, pf;\n\t"
+      STEM_MMA_SS(2) STEM_MMA_SS(4) STEM_MMA_SS(6) "}" ::"r"(d), "r"(alo), "r"(blo), "r"(hi),
+      "r"(idesc)
       : "memory");
 }
+#undef STEM_MMA_SS
+// P V group: O += P V over the 128 keys, A = P from TMEM (bf16 pairs, 8 columns per k-step of
+// 16 keys: keys 16kk.. at column a0 + kPCol[kk]), B = V MN-major in shared memory (16 key rows
+// of 128 bytes per k-step: descriptor offset kk * 128). acc0 = 0 starts O afresh.
+// operands: %0 d, %1 a0, %2 b_lo, %3 hi, %4 idesc, %5 acc0
+#define STEM_MMA_TS(COL, OFF)                                                              \
+  "add.u32 x, %1, " #COL ";\n\tadd.u32 y, %2, " #OFF ";\n\tmov.b64 b, {y, %3};\n\t"       \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %4, pt;\n\t"
+__device__ __forceinline__ void mma_pv8(uint32_t d, uint32_t a0, uint32_t blo, uint32_t hi,
+                                        uint32_t idesc, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, pt;\n\t.reg .b32 x, y;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 pt, %4, %4;\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p0;\n\t"
+      STEM_MMA_TS(8, 128) STEM_MMA_TS(16, 256) STEM_MMA_TS(24, 384) STEM_MMA_TS(32, 512)
+      STEM_MMA_TS(40, 640) STEM_MMA_TS(48, 768) STEM_MMA_TS(56, 896)
+      "}" ::"r"(d), "r"(a0), "r"(blo), "r"(hi), "r"(idesc), "r"(acc0)
+      : "memory");
+}
+#undef STEM_MMA_TS
 
 // Work item t -> (b, g, i, head pair): kv-head-group-major, query blocks in the plan's
 // heavy-first order, the ceil(G/2) head pairs of a group adjacent. Tile A is head g*G + 2p,
@@ -259,27 +263,68 @@ struct Step {
   __device__ __forceinline__ bool has_b() const { return it.hB >= 0; }
   __device__ __forceinline__ bool shared() const { return bb == ba; }
 };
+// Work items are claimed at run time, in the heavy-first order of their indices: the producer
+// takes the next index from a global counter (set to 0 by the pairing kernel) when it starts
+// an item and hands it to the MMA thread and the softmax threads through a ring in shared
+// memory (-1: none left). A CTA that finishes its items early takes more, so the CTAs end
+// together instead of by a fixed round-robin share.
+__device__ __forceinline__ bool claim_item(Bars* bars, unsigned long long* counter,
+                                           int64_t items, int64_t n, int32_t* status,
+                                           int64_t* t) {
+  int64_t v = static_cast<int64_t>(atomicAdd(counter, 1ull));
+  if (v >= items) v = -1;
+  const int q = static_cast<int>(n % kItemRing);
+  if (!wait_bar(&bars->iq_empty[q], static_cast<uint32_t>(((n / kItemRing) & 1) ^ 1), bars,
+                status))
+    return false;
+  bars->iq[q] = v;
+  mbar_arrive(&bars->iq_full[q]);
+  *t = v;
+  return true;
+}
+// The n-th claimed item of this CTA (every reader calls this once per item, in order).
+__device__ __forceinline__ bool read_item(Bars* bars, int64_t n, int32_t* status, int64_t* t) {
+  const int q = static_cast<int>(n % kItemRing);
+  if (!wait_bar(&bars->iq_full[q], static_cast<uint32_t>((n / kItemRing) & 1), bars, status))
+    return false;
+  *t = bars->iq[q];
+  mbar_arrive(&bars->iq_empty[q]);
+  return true;
+}
+
 struct Seq {
   int64_t t, items;
   int G, nb, Hkv, Hq;
   int64_t cap;
   PlanDev plan;
   const uint32_t* sched;
+  Bars* bars;
+  unsigned long long* counter;  // non-null: this walker claims items (the producer)
+  int32_t* status;
+  bool failed;  // a bounded wait on the item ring expired
   int n, j, cnt;
   Item it;
   const uint32_t* row;
   uint32_t e_next;  // schedule entry of the coming step, loaded one call ahead
   __device__ __forceinline__ void init(int64_t items_, int G_, int nb_, int Hkv_, int Hq_,
-                                       int64_t cap_, PlanDev plan_, const uint32_t* sched_) {
-    t = blockIdx.x;
+                                       int64_t cap_, PlanDev plan_, const uint32_t* sched_,
+                                       Bars* bars_, unsigned long long* counter_,
+                                       int32_t* status_) {
     items = items_; G = G_; nb = nb_; Hkv = Hkv_; Hq = Hq_; cap = cap_; plan = plan_;
-    sched = sched_;
+    sched = sched_; bars = bars_; counter = counter_; status = status_;
+    failed = false;
     n = -1; j = 0; cnt = 0;
   }
   __device__ __forceinline__ bool next(Step& s) {
     if (j >= cnt) {
-      if (n >= 0) t += gridDim.x;
-      if (t >= items) return false;
+      const int64_t ord = n + 1;
+      const bool ok = counter ? claim_item(bars, counter, items, ord, status, &t)
+                              : read_item(bars, ord, status, &t);
+      if (!ok) {
+        failed = true;
+        return false;
+      }
+      if (t < 0) return false;
       ++n;
       it = decode(t, G, nb, Hkv, plan.order);
       cnt = plan.k[it.i];
@@ -306,8 +351,8 @@ struct Seq {
 // A block both heads keep is one tile. The MMA thread (which takes the tiles) and the release
 // thread (which frees them) run this same recurrence, so both agree on every slot.
 struct TileOrder {
-  int64_t next = 0;
-  int64_t kA = 0, kB = 0, vA = 0, vB = 0;  // tiles of the latest S_A, S_B, PV_A, PV_B
+  int32_t next = 0;
+  int32_t kA = 0, kB = 0, vA = 0, vB = 0;  // tiles of the latest S_A, S_B, PV_A, PV_B
   // call in issue order: k_a(x0), k_b(x0); then per step c: v_a(), k_a(x), v_b(c), k_b(x)
   __device__ __forceinline__ void k_a() { kA = next++; }
   __device__ __forceinline__ void k_b(bool shared) { kB = shared ? kA : next++; }
@@ -320,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, int Hq, int Hkv, int S, int nb,
-                      int64_t items, PlanDev plan, int64_t cap,
+                      int64_t items, PlanDev plan, int64_t cap, unsigned long long* counter,
                       const uint32_t* __restrict__ sched, __nv_bfloat16* __restrict__ out,
                       int32_t* status, int withhold_q) {
   using C = Cfg<D>;
@@ -346,6 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int s = 0; s < kItemRing; ++s) {
+      mbar_init(&bars->iq_full[s], 1);
+      mbar_init(&bars->iq_empty[s], kItemReaders);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -411,9 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return fill(&tm_k, st, st.ba);
       };
       Seq seq;
-      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched);
+      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched, bars, counter, status);
       Step x;
       bool have = seq.next(x);
+      if (seq.failed) ok = false;
       if (have) {
         ok = start_step(x);
         if (ok && x.has_b() && !x.shared()) ok = fill(&tm_k, x, x.bb);
@@ -421,6 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (have && ok) {
         const Step c = x;
         have = seq.next(x);
+        if (seq.failed) {
+          ok = false;
+          break;
+        }
         if (!(ok = fill(&tm_v, c, c.ba))) break;
         if (have && !(ok = start_step(x))) break;
         if (c.has_b() && !c.shared() && !(ok = fill(&tm_v, c, c.bb))) break;
@@ -435,114 +489,148 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per head step T of step c (lookahead x): the waits for P_T(c) and the V tile of c (and,
+    // at an item's first step, the epilogue's release of O_T) are tested together, so their
+    // latencies overlap, then P V_T(c) goes out; then the wait for the K tile of x (and, when
+    // x starts an item, its Q tile) and S_T(x), with one commit after the S group. Bookkeeping
+    // is 32-bit: phase bits and tile numbers (tile f sits in slot f % kSlots, fill round
+    // f / kSlots).
     if (lane == 0) {
       constexpr uint32_t idesc_s = instr_desc(kM, kN, false);
       constexpr uint32_t idesc_o = instr_desc(kM, D, true);
-      const uint32_t q_base = su32(q_tiles), kv_base = su32(kv_tiles);
-      int64_t q_uses[2] = {0, 0};  // Q tiles consumed per tile
-      int64_t steps[2] = {0, 0};   // PV issued per tile (p_full parity)
-      int64_t outs[2] = {0, 0};    // items finished per tile (o_empty parity)
+      constexpr uint32_t kTileU = C::kTile >> 4;  // a tile's size in descriptor units
+      const uint32_t hi = smem_desc_hi(1024);
+      const uint32_t q_lo = smem_desc_lo(su32(q_tiles), 16);
+      const uint32_t k_lo = smem_desc_lo(su32(kv_tiles), 16);
+      const uint32_t v_lo = smem_desc_lo(su32(kv_tiles), kN * 128);
+      uint32_t qph = 0;  // bit T: parity of the next q_full[T] wait
+      uint32_t pph = 0;  // bit T: parity of the next p_full[T] wait
+      uint32_t oph = 0;  // bit T: items finished on tile T, mod 2 (o_empty waits take the other)
       bool ok = true;
       TileOrder order;
-      auto wait_tile = [&](int64_t f) -> bool {
-        return wait_bar(&bars->kv_full[f % kSlots], static_cast<uint32_t>((f / kSlots) & 1), bars,
+      auto kv_try = [&](int32_t f) {
+        return mbar_try(&bars->kv_full[f % kSlots], static_cast<uint32_t>(f / kSlots) & 1u);
+      };
+      auto kv_wait = [&](int32_t f) {
+        return wait_bar(&bars->kv_full[f % kSlots], static_cast<uint32_t>(f / kSlots) & 1u, bars,
                         status);
       };
-      // S_T(x) = Q_T K^T into S_T; one commit, to s_full[T]. Every release (K and V slots, Q)
-      // is done by the softmax release thread when it sees that commit: a commit covers every
-      // earlier product of this thread.
-      auto issue_s = [&](const Step& st, int tl) -> bool {
-        if (st.first) {
-          const int64_t r = q_uses[tl]++;
-          if (!wait_bar(&bars->q_full[tl], static_cast<uint32_t>(r & 1), bars, status))
-            return false;
-        }
-        const int64_t f = tl == 0 ? order.kA : order.kB;
-        if (!(tl == 1 && st.shared()) && !wait_tile(f)) return false;
-        tc_fence_after();
-        const uint32_t qa = q_base + tl * C::kTile;
-        const uint32_t ka = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
-        static_assert(C::kKSteps == 8 || C::kKSteps == 4, "group of 8 (D 128) or 4 (D 64)");
+      auto s_group = [&](int tl, int32_t f) {
+        const uint32_t a = q_lo + tl * kTileU, b = k_lo + static_cast<uint32_t>(f % kSlots) * kTileU;
         if constexpr (C::kKSteps == 8) {
-          uint64_t ad[8], bd[8];
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
-            ad[kk] = smem_desc(qa + off, 16, 1024);
-            bd[kk] = smem_desc(ka + off, 16, 1024);
-          }
-          mma_ss8(tmem + tl * 128, ad, bd, idesc_s, 0u);
+          mma_s8(tmem + tl * 128, a, b, hi, idesc_s);
         } else {
-#pragma unroll
-          for (int kk = 0; kk < C::kKSteps; ++kk) {
-            const uint32_t off = (kk >> 2) * (kM * 128) + (kk & 3) * 32;
-            mma_ss(tmem + tl * 128, smem_desc(qa + off, 16, 1024), smem_desc(ka + off, 16, 1024),
-                   idesc_s, kk > 0 ? 1u : 0u);
-          }
+          static_assert(C::kKSteps == 4, "D 128 or 64");
+          mma_s4(tmem + tl * 128, a, b, hi, idesc_s);
         }
         tc_commit(&bars->s_full[tl]);
-        return true;
       };
-      // O_T += P_T V (P from TMEM over the first half of S_T). No commit: the next S_T commit
-      // covers it; o_full at the item's end; and when head B has no next step (the next item
-      // has a single head, or the sequence ends), its V slot is released here.
-      auto issue_pv = [&](const Step& st, int tl, bool next_has_b) -> bool {
-        if (st.first) {
-          const int64_t r = outs[tl];
-          if (!wait_bar(&bars->o_empty[tl], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
-            return false;
-        }
-        const int64_t r = steps[tl]++;
-        if (!wait_bar(&bars->p_full[tl], static_cast<uint32_t>(r & 1), bars, status))
-          return false;
-        const int64_t f = tl == 0 ? order.vA : order.vB;
-        if (!(tl == 1 && st.shared()) && !wait_tile(f)) return false;
-        tc_fence_after();
-        const uint32_t vaddr = kv_base + static_cast<uint32_t>(f % kSlots) * C::kTile;
-        const uint32_t o_tm = tmem + 256 + tl * 128, p_tm = tmem + tl * 128;
-        {
-          // B = V rows kk*16 .. +15 (keys), MN-major: 64-column boxes kN*128 bytes apart
-          uint64_t bd[8];
-#pragma unroll
-          for (int kk = 0; kk < kN / 16; ++kk)
-            bd[kk] = smem_desc(vaddr + kk * 16 * 128, kN * 128, 1024);
-          mma_ts8(o_tm, p_tm, bd, idesc_o, st.first ? 0u : 1u);
-        }
-        if (tl == 1 && !next_has_b) tc_commit(&bars->kv_empty[f % kSlots]);
-        if (st.last) {
-          tc_commit(&bars->o_full[tl]);
-          ++outs[tl];
-        }
-        return true;
+      auto pv_group = [&](int tl, int32_t f, bool first) {
+        static_assert(kN / 16 == 8, "one P V group is 8 products of 16 keys");
+        mma_pv8(tmem + 256 + tl * 128, tmem + tl * 128,
+                v_lo + static_cast<uint32_t>(f % kSlots) * kTileU, hi, idesc_o, first ? 0u : 1u);
       };
       Seq seq;
-      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched);
+      seq.init(items, G, nb, Hkv, Hq, cap, plan, sched, bars, nullptr, status);
       Step x;
       bool have = seq.next(x);
-      if (have) {
+      if (seq.failed) ok = false;
+      if (have) {  // S of the first step
         order.k_a();
-        ok = issue_s(x, 0);
+        ok = wait_bar(&bars->q_full[0], 0, bars, status) && kv_wait(order.kA);
+        if (ok) {
+          tc_fence_after();
+          s_group(0, order.kA);
+        }
+        qph ^= 1u;
         if (ok && x.has_b()) {
           order.k_b(x.shared());
-          ok = issue_s(x, 1);
+          ok = wait_bar(&bars->q_full[1], 0, bars, status) && (x.shared() || kv_wait(order.kB));
+          if (ok) {
+            tc_fence_after();
+            s_group(1, order.kB);
+          }
+          qph ^= 2u;
         }
       }
       while (have && ok) {
         const Step c = x;
         have = seq.next(x);
+        if (seq.failed) {
+          ok = false;
+          break;
+        }
+        // ---------------- head A: P V_A(c), then S_A(x)
         order.v_a();
-        if (!(ok = issue_pv(c, 0, false))) break;
+        {
+          bool r = mbar_try(&bars->p_full[0], pph & 1u) & kv_try(order.vA);
+          if (c.first) r &= mbar_try(&bars->o_empty[0], (oph & 1u) ^ 1u);
+          if (!r) {
+            ok = wait_bar(&bars->p_full[0], pph & 1u, bars, status) && kv_wait(order.vA) &&
+                 (!c.first || wait_bar(&bars->o_empty[0], (oph & 1u) ^ 1u, bars, status));
+            if (!ok) break;
+          }
+          pph ^= 1u;
+        }
+        tc_fence_after();
+        pv_group(0, order.vA, c.first);
+        if (c.last) {
+          tc_commit(&bars->o_full[0]);
+          oph ^= 1u;
+        }
         if (have) {
           order.k_a();
-          if (!(ok = issue_s(x, 0))) break;
+          const bool qx = x.first;
+          bool r = kv_try(order.kA);
+          if (qx) r &= mbar_try(&bars->q_full[0], qph & 1u);
+          if (!r) {
+            ok = kv_wait(order.kA) && (!qx || wait_bar(&bars->q_full[0], qph & 1u, bars, status));
+            if (!ok) break;
+          }
+          if (qx) qph ^= 1u;
+          tc_fence_after();
+          s_group(0, order.kA);
         }
+        // ---------------- head B: P V_B(c) when step c has a head B, then S_B(x) when step x
+        // has one (independently: an item without head B can be followed by one with it)
+        const bool xb = have && x.has_b();
         if (c.has_b()) {
           order.v_b(c.shared());
-          if (!(ok = issue_pv(c, 1, have && x.has_b()))) break;
+          const bool wv = !c.shared();
+          bool r = mbar_try(&bars->p_full[1], (pph >> 1) & 1u);
+          if (wv) r &= kv_try(order.vB);
+          if (c.first) r &= mbar_try(&bars->o_empty[1], ((oph >> 1) & 1u) ^ 1u);
+          if (!r) {
+            ok = wait_bar(&bars->p_full[1], (pph >> 1) & 1u, bars, status) &&
+                 (!wv || kv_wait(order.vB)) &&
+                 (!c.first ||
+                  wait_bar(&bars->o_empty[1], ((oph >> 1) & 1u) ^ 1u, bars, status));
+            if (!ok) break;
+          }
+          pph ^= 2u;
+          tc_fence_after();
+          pv_group(1, order.vB, c.first);
+          // no S_B follows this P V to cover it: release its V slot from here
+          if (!xb) tc_commit(&bars->kv_empty[order.vB % kSlots]);
+          if (c.last) {
+            tc_commit(&bars->o_full[1]);
+            oph ^= 2u;
+          }
         }
-        if (have && x.has_b()) {
+        if (xb) {
           order.k_b(x.shared());
-          if (!(ok = issue_s(x, 1))) break;
+          const bool qx = x.first, wk = !x.shared();
+          bool r = true;
+          if (wk) r &= kv_try(order.kB);
+          if (qx) r &= mbar_try(&bars->q_full[1], (qph >> 1) & 1u);
+          if (!r) {
+            ok = (!wk || kv_wait(order.kB)) &&
+                 (!qx || wait_bar(&bars->q_full[1], (qph >> 1) & 1u, bars, status));
+            if (!ok) break;
+          }
+          if (qx) qph ^= 2u;
+          tc_fence_after();
+          s_group(1, order.kB);
         }
       }
       // make sure every issued product has completed before TMEM is released
@@ -589,18 +677,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       xp ^= 1;
       return mt;
     };
-    // P = exp2(S * sl2 - m_run) packed to bf16; returns this thread's partial row sum.
-    auto exp_pack = [&](const uint32_t* sr, float m_run, uint32_t* p) -> float {
+    // P = exp2(S * sl2 - m_run) packed to bf16 over column pairs [C0, C1) of this thread's
+    // half; adds to the partial row sums the bf16 values that enter P V (mixed-precision adds
+    // take each half of a packed pair as it is), so the normaliser and the products see the
+    // same P and a row that one key dominates returns that key's V row.
+    auto exp_pack = [&](const uint32_t* sr, float m_run, uint32_t* p, f2* sum, auto c0,
+                        auto c1) {
       const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
-      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
 #pragma unroll
-      for (int c = 0; c < kH / 2; ++c) {
+      for (int c = decltype(c0)::value; c < decltype(c1)::value; ++c) {
         const f2 x = fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
         const f2 e{ex2(x.x), ex2(x.y)};
-        sum[c & 1] = add2(sum[c & 1], e);
         p[c] = pack_bf16(e.x, e.y);
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+            : "+f"(sum[c & 1].x), "+f"(sum[c & 1].y)
+            : "r"(p[c]));
       }
+    };
+    auto exp_all = [&](const uint32_t* sr, float m_run, uint32_t* p) -> float {
+      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
+      exp_pack(sr, m_run, p, sum, std::integral_constant<int, 0>{},
+               std::integral_constant<int, kH / 2>{});
       return (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
+    };
+    auto diag_mask = [&](uint32_t* sr, auto c0, auto c1) {
+#pragma unroll
+      for (int c = decltype(c0)::value; c < decltype(c1)::value; ++c)
+        if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
     };
     // One step of tile tl on key block blk; returns false on abort.
     //
@@ -630,22 +734,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t s_addr = tmem + tl * 128 + lane_off;
       uint32_t sr[kH];
+      uint32_t p[kH / 2];
+      bool ok = true;
 #pragma unroll
       for (int c = 0; c < kH / 32; ++c) TC_LD32(s_addr + half * kH + 32 * c, (sr + 32 * c));
-      tc_wait_ld();
+      tc_wait_ld_r32(sr);
+      tc_wait_ld_r32(sr + 32);
       if (blk == qi) {  // the diagonal block: token-causal
-#pragma unroll
-        for (int c = 0; c < kH; ++c)
-          if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
+        diag_mask(sr, std::integral_constant<int, 0>{}, std::integral_constant<int, kH>{});
       }
-      bool ok = true;
       if (first) {
         m_run = pair_max(sr, ok);
         if (!ok) return false;
         lsum = 0.f;
       }
-      uint32_t p[kH / 2];
-      float part = exp_pack(sr, m_run, p);
+      float part = exp_all(sr, m_run, p);
       const bool small = part < 65536.0f;  // false for inf and NaN too
       if (!pair_and(bar_id, __all_sync(0xffffffffu, small))) {
         if (!pair_and(bar_id, true)) return false;
@@ -664,21 +767,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kDH / 32; ++c) {
           uint32_t o[32];
           TC_LD32(o_addr + 32 * c, o);
-          tc_wait_ld();
+          tc_wait_ld_r32(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           TC_ST32(o_addr + 32 * c, o);
         }
         tc_wait_st();
-        part = exp_pack(sr, m_run, p);
+        part = exp_all(sr, m_run, p);
       }
-      lsum += part;
       // P over S_T columns [0, 64): this half's keys go to columns half*32 .. +32 (both halves
       // finished reading S before the pair's check barrier above)
       TC_ST32(s_addr + half * (kH / 2), p);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[tl]);
+      lsum += part;
       return true;
     };
     auto epilogue = [&](int tl, const Item& it, int64_t& nouts, float lsum) -> bool {
@@ -698,7 +801,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kDH / 32; ++c) {
         uint32_t o[32];
         TC_LD32(o_addr + 32 * c, o);
-        tc_wait_ld();
+        tc_wait_ld_r32(o);
         uint4 pk[4];
         uint32_t* wv = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
@@ -716,7 +819,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     TileOrder order;  // replica of the MMA thread's tile numbering
     bool have_prev = false, prev_has_b = false, prev_shared = false;
-    for (int64_t t = blockIdx.x; t < items && ok; t += gridDim.x) {
+    for (int64_t n = 0; ok; ++n) {
+      int64_t t = -1;
+      const bool got = read_item(bars, n, status, &t);
+      // both warps of a pair go on together (a failed read takes the partner out too)
+      if (!pair_and(bar_id, __all_sync(0xffffffffu, got))) {
+        ok = false;
+        break;
+      }
+      if (t < 0) break;
       const Item it = decode(t, G, nb, Hkv, plan.order);
       const int cnt = plan.k[it.i];
       const uint32_t* srow = sched_row(sched, it, Hkv, G, cap, plan);
@@ -795,13 +906,15 @@ cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  // the pairing kernel sets the work counter (the region's first bytes) to 0 and writes the
+  // schedule after it
   e = launch_pairs(sel_idx, B, Hq, Hkv, nb, plan, cap, sched, st);
   if (e != cudaSuccess) return e;
+  auto* counter = reinterpret_cast<unsigned long long*>(sched);
   const int64_t grid = std::min<int64_t>(items, sm_count());
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, Hq, Hkv, S, nb, items,
-                                                           plan, cap, sched,
-                                                           static_cast<__nv_bfloat16*>(out),
-                                                           status, g_withhold_q.load());
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
+      tq, tk, tv, Hq, Hkv, S, nb, items, plan, cap, counter, pairs_schedule(sched),
+      static_cast<__nv_bfloat16*>(out), status, g_withhold_q.load());
   return cudaGetLastError();
 }
 

@@ -14,6 +14,10 @@
 //
 // One warp per item: a lane takes one entry of a list, tests membership in the other list by
 // binary search, and ballots give every entry its output position.
+//
+// The region also holds, in its first kCounterBytes, the attention kernel's work counter, which
+// this kernel sets to 0 (the attention kernel runs next on the same stream and claims its work
+// items from it).
 #include <cuda_runtime.h>
 
 #include "stem_internal.h"
@@ -39,7 +43,8 @@ __device__ __forceinline__ bool member(const int32_t* l, int k, int x, int i) {
 
 __global__ void __launch_bounds__(kPairWarps * 32) pairs_kernel(
     const int32_t* __restrict__ sel_idx, int Hq, int Hkv, int nb, int64_t items, PlanDev plan,
-    int64_t cap, uint16_t* __restrict__ sched) {
+    int64_t cap, uint16_t* __restrict__ sched, unsigned long long* __restrict__ counter) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0ull;
   const int64_t item = static_cast<int64_t>(blockIdx.x) * kPairWarps + (threadIdx.x >> 5);
   if (item >= items) return;
   const int lane = threadIdx.x & 31;
@@ -112,22 +117,24 @@ __global__ void __launch_bounds__(kPairWarps * 32) pairs_kernel(
 }  // namespace
 
 cudaError_t launch_pairs(const int32_t* sel_idx, int B, int Hq, int Hkv, int nb, PlanDev plan,
-                         int64_t cap, uint32_t* sched, cudaStream_t st) {
+                         int64_t cap, uint32_t* region, cudaStream_t st) {
+  auto* counter = reinterpret_cast<unsigned long long*>(region);
+  uint32_t* sched = pairs_schedule(region);
   const int G = Hq / Hkv;
   const int64_t items = static_cast<int64_t>(B) * Hkv * ((G + 1) / 2) * nb;
   if (items == 0) return cudaSuccess;
   const int64_t grid = (items + kPairWarps - 1) / kPairWarps;
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
   pairs_kernel<<<static_cast<unsigned>(grid), kPairWarps * 32, 0, st>>>(
-      sel_idx, Hq, Hkv, nb, items, plan, cap, reinterpret_cast<uint16_t*>(sched));
+      sel_idx, Hq, Hkv, nb, items, plan, cap, reinterpret_cast<uint16_t*>(sched), counter);
   return cudaGetLastError();
 }
 
 size_t pairs_bytes(int B, int Hq, int Hkv, int nb) {
   const int G = Hq / Hkv;
-  // upper bound of the schedule: cap <= nb (nb + 1) / 2 for any budget
-  return sizeof(uint32_t) * static_cast<size_t>(B) * Hkv * ((G + 1) / 2) *
-         (static_cast<size_t>(nb) * (nb + 1) / 2);
+  // the work counter, then the schedule (upper bound: cap <= nb (nb + 1) / 2 for any budget)
+  return kCounterBytes + sizeof(uint32_t) * static_cast<size_t>(B) * Hkv * ((G + 1) / 2) *
+                             (static_cast<size_t>(nb) * (nb + 1) / 2);
 }
 
 }  // namespace stem

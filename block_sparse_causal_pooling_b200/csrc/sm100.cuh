@@ -48,7 +48,7 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 }
 
 // Bounded drain wait used on the abort path only (ignores the abort flag).
-static __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
+static __device__ __forceinline__ void drain_bar(uint64_t* b, uint32_t parity) {
   const uint64_t t0 = gtimer();
   while (!mbar_try(b, parity) && gtimer() - t0 < kWaitNs) {
   }

@@ -67,10 +67,16 @@ cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B,
                              const int32_t* sel_idx, const int32_t* sel_cnt, uint32_t* sched,
                              void* out, int32_t* status, cudaStream_t st);
 
-// Head-pair step schedules from the CSR lists (pairs.cu).
+// Head-pair step schedules from the CSR lists (pairs.cu). `region` (pairs_bytes()) holds the
+// attention kernel's work counter in its first kCounterBytes, which the pairing kernel sets to
+// 0, then the schedule (pairs_schedule(region)).
+constexpr size_t kCounterBytes = 256;
+inline uint32_t* pairs_schedule(uint32_t* region) {
+  return region + kCounterBytes / sizeof(uint32_t);
+}
 cudaError_t launch_pairs(const int32_t* sel_idx, int B, int Hq, int Hkv, int nb, PlanDev plan,
-                         int64_t cap, uint32_t* sched, cudaStream_t st);
-// Workspace bytes of the schedule for any budget of this shape.
+                         int64_t cap, uint32_t* region, cudaStream_t st);
+// Workspace bytes of the counter and the schedule for any budget of this shape.
 size_t pairs_bytes(int B, int Hq, int Hkv, int nb);
 
 // Block-sparse attention, float32 inputs on the CUDA cores (attn_f32.cu).

@@ -9,13 +9,12 @@ max(1, |M|): |M_a - M_b| <= REL_TIE * max(1, |M_a|, |M_b|).
 
 Attention output: max-abs error <= 2e-2 and mean-abs error <= 1e-3 against the oracle's
 double-precision result for bfloat16 inputs (float32 accumulation); tighter for float32 inputs.
-These bounds hold for every element of every named workload and of the small cases drawn with
-their value recipes; the tests assert that no element there needs more.
-
-One exception, for synthetic cases built to have very large outputs (many x5 V outliers in a
-short sequence, or key blocks scaled far above the sink): where |reference| >= 8 a bfloat16
-output cannot be within 2e-2 of it, since half a bfloat16 ulp there is 2^-5 or more. For those
-elements alone, and only in cases that declare outliers=True, the bound adds that half-ulp.
+The 2e-2 bound holds for every element whose reference is below 8 in magnitude. From 8 up a
+bfloat16 output cannot be within 2e-2 of the reference at all (half a bfloat16 ulp there is
+2^-5 or more, so even the exactly rounded value can miss by 0.031), and the named workloads
+have such outputs (rows whose attention peaks on a x5 V row of the 128K workload reach 13): for
+those elements alone the bound adds half a bfloat16 ulp of the reference, and the mean bound
+the mean of those half-ulps.
 
 Rows whose kept set differs from the oracle's by a tie swap are compared with the oracle's
 attention over the GPU's own kept set (several selections are correct there, and each has its
@@ -112,34 +111,31 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, np.floor(np.log2(ax)).astype(np.int64) - 8)
 
 
-def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = "",
-                     outliers: bool = False):
+def assert_out_close(gpu: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
     """Max-abs and mean-abs error against the oracle, element by element.
 
-    bfloat16: every element within 2e-2, mean within 1e-3. With outliers=True (synthetic cases
-    only) elements with |reference| >= 8 may also be off by half a bfloat16 ulp of the
-    reference (the output format's own rounding there exceeds 2e-2), and the mean bound grows
-    by the mean of those half-ulps. Without it, no element may use the widened bound."""
+    bfloat16: every element with |reference| < 8 within 2e-2; elements with |reference| >= 8
+    within 2e-2 plus half a bfloat16 ulp of the reference (the output format's own rounding);
+    mean within 1e-3 plus the mean of those half-ulps."""
     e = out_error(gpu, ref)
     t = tol_for(dtype)
     bound = np.full(ref.shape, t["max_abs"])
     mean_bound = t["mean_abs"]
     if dtype == torch.bfloat16 and ref.size:
         big = np.abs(ref) >= 8.0
+        extra = np.where(big, bf16_half_ulp(ref), 0.0)
+        bound = bound + extra
+        mean_bound += float(extra.mean())
+        err = np.abs(gpu - ref)
         e["n_ref_at_least_8"] = int(big.sum())
-        if outliers:
-            extra = np.where(big, bf16_half_ulp(ref), 0.0)
-            bound = bound + extra
-            mean_bound += float(extra.mean())
+        e["max_abs_below_8"] = float(err[~big].max()) if (~big).any() else 0.0
+        # elements that needed the format allowance (all of them at |reference| >= 8)
+        e["n_above_plain_bound"] = int((err > t["max_abs"]).sum())
         e["mean_bound"] = mean_bound
-        # elements whose error needed more than the plain 2e-2
-        e["n_bound_above_max_abs"] = int((np.abs(gpu - ref) > t["max_abs"]).sum())
         ref_b = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
         e["max_abs_vs_bf16_ref"] = float(np.abs(gpu - ref_b).max())
     worst = float(np.max(np.abs(gpu - ref) - bound)) if ref.size else 0.0
     assert worst <= 0 and e["mean_abs"] <= mean_bound, (what, e, t)
-    if dtype == torch.bfloat16 and not outliers:
-        assert e["n_bound_above_max_abs"] == 0, (what, e)
     return e
 
 
@@ -153,7 +149,7 @@ def gpu_csr(sel_idx, sel_cnt, B: int, Hq: int, nb: int, cap: int):
 
 def assert_prefill_out(out: torch.Tensor, cpu_inputs, block: int, ref_out: np.ndarray,
                        ref_rows, res: dict, sel_idx, sel_cnt, off, dtype: torch.dtype,
-                       what: str = "", outliers: bool = False):
+                       what: str = ""):
     """Output check of an end-to-end call. ref_out[t] is the oracle's output for ref_rows[t]
     on the oracle's selection. Rows whose GPU selection is a tie swap of the oracle's (listed
     in res["rows_bad"] by compare_selection) are instead compared with the oracle's attention
@@ -161,7 +157,7 @@ def assert_prefill_out(out: torch.Tensor, cpu_inputs, block: int, ref_out: np.nd
     swapped = set(res["rows_bad"])
     keep = [t for t, r in enumerate(ref_rows) if r not in swapped]
     e1 = assert_out_close(out_rows(out, [ref_rows[t] for t in keep], block), ref_out[keep],
-                          dtype, what, outliers)
+                          dtype, what)
     sw = [r for r in ref_rows if r in swapped]
     e2 = None
     if sw:
@@ -170,6 +166,5 @@ def assert_prefill_out(out: torch.Tensor, cpu_inputs, block: int, ref_out: np.nd
         nb = -(-S_ // block)
         gi, gc = gpu_csr(sel_idx, sel_cnt, B, Hq, nb, int(off[nb]))
         ref_sw = oracle.attention(q, k, v, block, gi, gc, off, sw)
-        e2 = assert_out_close(out_rows(out, sw, block), ref_sw, dtype, what + " (tie rows)",
-                              outliers)
+        e2 = assert_out_close(out_rows(out, sw, block), ref_sw, dtype, what + " (tie rows)")
     return e1, e2

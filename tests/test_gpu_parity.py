@@ -127,9 +127,15 @@ def test_end_to_end(name):
 def test_scores_growing_after_the_first_block(rho_min):
     """Two key blocks halfway through the sequence are scaled x6 and there is no sink, so the
     rows that keep them see scores far above those of their first block: the attention kernel's
-    reference max must be raised (O rescaled, P recomputed) for those rows."""
+    reference max must be raised (O rescaled, P recomputed) for those rows.
+
+    V is plain N(0,1) here (no x5 rows): the case is about the rescale. Its x6 keys make the
+    softmax of many rows peak on a few keys, and where those keys' V rows were x5 outliers the
+    bf16 rounding of P that enters P V (relative 2^-9 per weight, which bf16 products with bf16
+    V require) moves the output by up to 2^-9 * max|v - out|, about 0.04, beyond the 2e-2
+    bound at any |out|; that input belongs to no workload's recipe."""
     w = wl.LLAMA_32K.replace(name="growth", Hq=4, Hkv=2, S=4096, sink_scale=1.0,
-                             rho_min=rho_min, tau=8.0)
+                             rho_min=rho_min, tau=8.0, v_outlier_frac=0.0)
     q, k, v = wl.make_inputs(w, "cpu")
     k = k.clone()
     k[:, :, 16 * w.block:18 * w.block] *= 6
@@ -148,9 +154,8 @@ def test_scores_growing_after_the_first_block(rho_min):
             for h in range(w.Hq) for i in range(18, w.nb)]
     assert sum(kept) >= (len(kept) if rho_min == 1.0 else len(kept) // 4), sum(kept)
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    # synthetic large outputs: key blocks x6 with no sink make rows peaked on single x5 V rows
     parity.assert_prefill_out(out, (q, k, v), w.block, ref["out"], rows, res, sel_idx, sel_cnt,
-                              ref["off"], w.torch_dtype, "growth", outliers=True)
+                              ref["off"], w.torch_dtype, "growth")
 
 
 def test_dense_budget_matches_torch_sdpa():
@@ -222,3 +227,26 @@ def test_all_equal_metric_takes_lowest_blocks():
         for i in range(w.nb):
             want = [0] if i == 0 else sorted(set([0, i] + list(range(1, kk[i] - 1))))
             assert si[0, h, off[i]:off[i + 1]].tolist() == want
+
+
+@pytest.mark.parametrize("name", ["llama-4k", "llama-b2-2k", "qwen-3k", "bf16-d64-blk64", "nb37",
+                                  "ragged-blk128"])
+def test_select_split_and_fused_designs_agree(name):
+    """stem_select runs the split design (score triangles in the workspace, then one warp per
+    row) when the workspace has room for them and the fused kernel when it holds only the plan:
+    both compute every score with the same float32 chain, so lists, counts and the float32
+    metric must be identical."""
+    w = CASES[name]
+    cpu, dev = inputs(w)
+    qbar, kbar, vnorm = S.stem_pool(*dev, w.block)
+    full = S.alloc_workspace(dev[0], dev[1], w.block)
+    plan_only = torch.empty(256 + -(-4 * (3 * w.nb + 1) // 256) * 256, dtype=torch.uint8,
+                            device=DEV)
+    assert plan_only.numel() < full.numel()
+    a = S.stem_select(qbar, kbar, vnorm, w.rho_min, w.tau, w.k_min, with_metric=True,
+                      workspace=full)
+    b = S.stem_select(qbar, kbar, vnorm, w.rho_min, w.tau, w.k_min, with_metric=True,
+                      workspace=plan_only)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert torch.equal(a[2], b[2])

@@ -50,8 +50,12 @@ def draw(seed):
     strides = [s for s in (4, 8, 16, 32) if block % s == 0 and block // s <= 32 and S_ % s == 0]
     if dtype == "bf16" and strides and rng.random() < 0.5:
         md.update(score="antidiag", stride=rng.choice(strides))
+    # V outliers: the float32 tiny workload's 16 rows per kv head; bfloat16 cases take the
+    # bfloat16 workloads' density, 0.5% of the rows (16 x5 rows among a few hundred tokens put
+    # a bfloat16 kernel's P rounding, 2^-9 per weight, past 2e-2 on outputs below 8)
+    vo = dict(v_outlier_rows=None, v_outlier_frac=0.005) if dtype == "bf16" else {}
     w = wl.TINY.replace(name=f"random-{seed}", B=rng.choice([1, 2]), Hq=Hkv * G, Hkv=Hkv, S=S_,
-                        D=D, block=block, dtype=dtype, seed=wl.BASE_SEED + 500 + seed)
+                        D=D, block=block, dtype=dtype, seed=wl.BASE_SEED + 500 + seed, **vo)
     return w, md
 
 
@@ -83,7 +87,5 @@ def test_random_case(seed):
     assert not res["violations"], (w, md, res["violations"][:5])
     assert res["tie_swaps"] <= max(1, res["rows"] // 20), res
     rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.nb)]
-    # the tiny workload's recipe: 16 x5 V rows per kv head in sequences of a few hundred
-    # tokens, so rows peaked on one outlier reach |out| > 8 (synthetic large outputs)
     parity.assert_prefill_out(out, (q, k, v), w.block, ref["out"], rows, res, sel_idx, sel_cnt,
-                              ref["off"], w.torch_dtype, f"{w} {md}", outliers=True)
+                              ref["off"], w.torch_dtype, f"{w} {md}")
