@@ -51,6 +51,51 @@ __device__ __forceinline__ uint64_t order_bits(double x) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
+// The digit (0-255, taken from the largest) at which a count of `rem` keys is reached in a
+// warp's 256-bin histogram, the number of keys in larger digits, and the digit's own count.
+struct DigitPick {
+  int digit, above, dcount;
+};
+__device__ __forceinline__ DigitPick pick_digit(const int* hist, int lane, int rem) {
+  // lane l owns bins 255-8l .. 248-8l (descending)
+  int cnt[8];
+  int local = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    cnt[e] = hist[255 - 8 * lane - e];
+    local += cnt[e];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - local;
+  const bool owner = excl < rem && rem <= incl;
+  int digit = 0, above = 0, dcount = 0;
+  if (owner) {
+    int run = excl;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (run + cnt[e] >= rem) {
+        digit = 255 - 8 * lane - e;
+        above = run;
+        dcount = cnt[e];
+        break;
+      }
+      run += cnt[e];
+    }
+  }
+  const int src = __ffs(__ballot_sync(0xffffffffu, owner)) - 1;
+  DigitPick r;
+  r.digit = __shfl_sync(0xffffffffu, digit, src);
+  r.above = __shfl_sync(0xffffffffu, above, src);
+  r.dcount = __shfl_sync(0xffffffffu, dcount, src);
+  __syncwarp();
+  return r;
+}
+
 // Kept set of row i: {0, i} plus the k(i)-2 largest keys over j in [1, i-1] (equal keys: lower
 // j first), written ascending to dst + t*dstride for t < ndst (the same list at every
 // destination). One warp; key_bits(j) is the order-preserving image of column j's key; hist is
@@ -111,41 +156,8 @@ __device__ __forceinline__ void select_row(int i, int kk, KeyBits key_bits, int*
         if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 0xff], 1);
       }
       __syncwarp();
-      // lane l owns bins 255-8l .. 248-8l (descending)
-      int cnt[8];
-      int local = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        cnt[e] = hist[255 - 8 * lane - e];
-        local += cnt[e];
-      }
-      int incl = local;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const int excl = incl - local;
-      const bool owner = excl < rem && rem <= incl;
-      int digit = 0, above = 0, dcount = 0;
-      if (owner) {
-        int run = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (run + cnt[e] >= rem) {
-            digit = 255 - 8 * lane - e;
-            above = run;
-            dcount = cnt[e];
-            break;
-          }
-          run += cnt[e];
-        }
-      }
-      const int src = __ffs(__ballot_sync(0xffffffffu, owner)) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      dcount = __shfl_sync(0xffffffffu, dcount, src);
-      __syncwarp();
+      const DigitPick dp = pick_digit(hist, lane, rem);
+      const int digit = dp.digit, above = dp.above, dcount = dp.dcount;
       rem -= above;
       prefix = (prefix & ~(0xffull << shift)) | (static_cast<uint64_t>(digit) << shift);
       pmask |= 0xffull << shift;
@@ -322,6 +334,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(
   }
 }
 
+// 16-byte copy from global to shared memory; with full = false the destination is filled with 0
+// (nothing is read from src).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(full ? 16 : 0)
+               : "memory");
+}
+
 // ---- split design, step 1: pooled scores s_ij = qbar_i . kbar_j / sqrt(D) for j <= i of heads
 // [h0, h0 + nh) of the B*Hq, into tri[(head - h0) * nb(nb+1)/2 + i(i+1)/2 + j]. One CTA per 64 x 64
 // tile of (i, j) with the j tile at most the i tile; each thread holds the 4 x 4 scores of rows
@@ -350,23 +371,30 @@ __global__ void __launch_bounds__(kSelThreads) score_tri_kernel(
   const float* qsrc = qbar + bh * nb * D;
   const float* ksrc = kbar + (static_cast<int64_t>(b) * Hkv + h / G) * nb * D;
   const int i0 = ti * kScT, j0 = tj * kScT;
-  for (int idx = threadIdx.x; idx < kScT * D / 4; idx += kSelThreads) {
-    const int r = idx / (D / 4), c4 = idx % (D / 4);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
-    if (i0 + r < nb) a = reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(i0 + r) * D)[c4];
-    if (j0 + r < nb) c = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j0 + r) * D)[c4];
-    *reinterpret_cast<float4*>(qs + r * LD + 4 * c4) = a;
-    *reinterpret_cast<float4*>(ks + r * LD + 4 * c4) = c;
+  // Both tiles go straight from global to shared memory (cp.async, 16 bytes a copy; rows past
+  // nb are filled with 0) in two halves of D, each its own group: the second half is in flight
+  // while the first is multiplied.
+  constexpr int kHalf = D / 2;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    for (int idx = threadIdx.x; idx < kScT * kHalf / 4; idx += kSelThreads) {
+      const int r = idx / (kHalf / 4), c4 = hf * (kHalf / 4) + idx % (kHalf / 4);
+      const bool qin = i0 + r < nb, kin = j0 + r < nb;
+      cp_async16(qs + r * LD + 4 * c4, qsrc + static_cast<int64_t>(qin ? i0 + r : 0) * D + 4 * c4,
+                 qin);
+      cp_async16(ks + r * LD + 4 * c4, ksrc + static_cast<int64_t>(kin ? j0 + r : 0) * D + 4 * c4,
+                 kin);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  __syncthreads();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 2
-  for (int d = 0; d < D; d += 4) {
+  // d ascending, the same multiply-add chain per score as select_kernel
+  auto madd = [&](int d) {
     float4 qv[4], kv[4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4*>(qs + (ty + 16 * a) * LD + d);
@@ -381,7 +409,15 @@ __global__ void __launch_bounds__(kSelThreads) score_tri_kernel(
         acc[a][c] = fmaf(qv[a].z, kv[c].z, acc[a][c]);
         acc[a][c] = fmaf(qv[a].w, kv[c].w, acc[a][c]);
       }
-  }
+  };
+  asm volatile("cp.async.wait_group 1;" ::: "memory");  // first half landed (this thread's)
+  __syncthreads();                                       // ... and every thread's
+#pragma unroll 2
+  for (int d = 0; d < kHalf; d += 4) madd(d);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+#pragma unroll 2
+  for (int d = kHalf; d < D; d += 4) madd(d);
   const float scale = rsqrtf(static_cast<float>(D));  // as in select_kernel
   float* dst = tri + static_cast<int64_t>(hl) * (static_cast<int64_t>(nb) * (nb + 1) / 2);
 #pragma unroll
