@@ -50,8 +50,8 @@ SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615687168 + 1021676032,
-                "sources_sha256": "1f6e9fcd47619c5d4f09c6ecdb805e5904cdfe10ffad7825983ebd96bfeaab5c"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1617127936 + 1022252032,
+                "sources_sha256": "f1f6a322377075784866d5bc74d1f634f3e5a8dbecca15077f713344646eb0da"}
 # The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,

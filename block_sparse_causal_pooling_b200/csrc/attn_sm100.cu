@@ -10,42 +10,40 @@
 // Work item: two GQA sibling heads A and B at one query block, which keep the same number of key
 // blocks; a step schedule (pairs.cu) pairs their lists so a block both keep is one K/V tile.
 //
-// Persistent kernel, one CTA per SM, 10 warps. Work items are claimed at run time from a global
+// Persistent kernel, one CTA per SM, 12 warps. Work items are claimed at run time from a global
 // counter in heavy-first order (the producer claims, the other roles read the claimed indices
 // from a ring in shared memory), so the CTAs finish together.
-//   warp 0      TMA producer: claims items; Q_A, Q_B (one tile each) and K/V tiles into a 4-slot
-//               ring of 128B-swizzled shared-memory tiles (boxes of 128 rows x 64 columns),
-//               filled in the order the products first use them.
+//   warp 0      TMA producer: claims items; Q_A, Q_B (one tile each) and K/V tiles into a ring
+//               of 128B-swizzled shared-memory tiles (boxes of 128 rows x 64 columns), filled
+//               in the order the products use them.
 //   warp 1      allocates the 512 TMEM columns; lane 0 issues every tcgen05.mma:
 //                 S_T = Q_T K^T     (M 128, N 128, K = D; A and B K-major in shared memory)
-//                 O_T += P_T V      (A = P read from TMEM over the first half of S_T, B = V
-//                                    MN-major in shared memory)
-//               in the order P V_A(c), S_A(c+1), P V_B(c), S_B(c+1), so one head's products run
-//               while the softmax works on the other head; one commit per S, none per P V.
-//   warps 2-9   softmax, two threads per query row (warps w and w+4 share TMEM lanes
-//               32*(w%4).. and take 64 columns each; tcgen05.ld 32x32b): row max (halves
-//               exchanged through shared memory at a barrier of the warp pair that also makes
-//               both warps agree on going on, so an abort cannot strand one), exp2 with the
-//               1/sqrt(D) scale folded in; P packed to bf16 and stored over the first half of
-//               S_T (tcgen05.st); the per-thread partial row sums add the bf16 values that
-//               enter P V, in fp32. Only an item's first step takes the exact row max; later steps
-//               use it as the reference and fall back to the exact max, an O rescale in TMEM
-//               and a recompute only when a partial row sum reaches 2^16 (exact: the final
-//               1/l uses the same reference as P). At an item's end: O * (1/l) -> bf16 ->
-//               global (streaming stores).
+//                 O_T += P_T V      (A = P K-major in shared memory, B = V MN-major)
+//               S_T of the next step goes out as soon as the softmax has read S_T of this step
+//               into registers, so it runs while the softmax works: a head is no serial chain
+//               of softmax, P V and the next S.
+//   warps 2-3   idle (they complete the first warpgroup, which hands its registers over).
+//   warps 4-7   softmax of head A, warps 8-11 of head B: one thread per query row (warp w reads
+//               TMEM lanes 32*(w%4)..), all 128 key columns (tcgen05.ld 32x32b): row max,
+//               exp2 with the 1/sqrt(D) scale folded in, P packed to bf16 and written to the
+//               head's P tile in shared memory (the layout a TMA box of Q has), row sums over
+//               the bf16 values that enter P V, in fp32. The running reference max moves only
+//               when a row's max exceeds it by more than 8 (log2 units): then O's row is
+//               rescaled in TMEM; otherwise P stays below 2^8 and the reference is kept (exact
+//               either way: the final 1/l uses the same reference as P). At an item's end:
+//               O * (1/l) -> bf16 -> global (streaming stores).
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).
 //
-// Synchronisation is by mbarriers, plus the warp-pair barrier above. Every mbarrier wait is
-// bounded by the global nanosecond timer: on expiry the CTA records STEM_ERR_TIMEOUT in the
-// status word, every role leaves its loop, the MMA thread drains its issued products, the
-// producer drains its issued copies (both bounded), TMEM is freed and the kernel returns.
+// Synchronisation is by mbarriers only. Every mbarrier wait is bounded by the global
+// nanosecond timer: on expiry the CTA records STEM_ERR_TIMEOUT in the status word, every role
+// leaves its loop, the MMA thread drains its issued products, the producer drains its issued
+// copies (both bounded), TMEM is freed and the kernel returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <type_traits>
 #include <atomic>
 #include <mutex>
 
@@ -70,39 +68,49 @@ using namespace sm100;
 
 constexpr int kM = 128;             // query rows per tile (= block)
 constexpr int kN = 128;             // keys per kept block
-constexpr int kSlots = 4;           // K/V ring slots
-constexpr int kThreads = 320;       // 10 warps
-constexpr int kSoftmaxThreads = 256;
+constexpr int kMaxSlots = 4;        // K/V ring slots (at most)
+constexpr int kThreads = 384;       // 12 warps: three warpgroups
+constexpr int kGroupThreads = 128;  // softmax threads of one head
+constexpr int kSoftmaxThreads = 2 * kGroupThreads;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kItemRing = 8;                       // claimed work items in flight
 constexpr int kItemReaders = 1 + kSoftmaxThreads;  // MMA thread and softmax threads
-
-template <int D>
-struct Cfg {
-  static constexpr uint32_t kTile = kM * D * 2;  // bytes of a 128 x D bf16 tile
-  static constexpr int kBoxes = D / 64;          // 128B-swizzled boxes of 64 columns
-  static constexpr int kKSteps = D / 16;         // MMA k-steps of QK^T
-};
+constexpr float kRescale = 8.0f;  // a row's reference max moves when exceeded by this (log2)
 
 struct __align__(8) Bars {
   uint64_t q_full[2], q_empty[2];            // per tile (A, B)
-  uint64_t kv_full[kSlots], kv_empty[kSlots];
-  uint64_t s_full[2], p_full[2];             // per tile
-  uint64_t o_full[2], o_empty[2];            // per tile
+  uint64_t kv_full[kMaxSlots], kv_empty[kMaxSlots];
+  uint64_t s_full[2];   // S_T complete (commit)
+  uint64_t s_free[2];   // S_T read into registers by the head's softmax threads
+  uint64_t p_full[2];   // P_T written to shared memory
+  uint64_t pv_done[2];  // P V_T complete (commit): P_T may be rewritten, O_T read
+  uint64_t o_empty[2];  // the epilogue has read O_T
   uint64_t iq_full[kItemRing], iq_empty[kItemRing];  // claimed items, producer -> readers
   int64_t iq[kItemRing];                     // item index, or -1: none left
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
-  float xch[2][2][kM];  // [parity][half][row] partial row maxima of the two halves
-  float xl[2][2][kM];   // [tile][half][row] partial row sums (epilogue)
 };
+
+template <int D>
+struct Cfg {
+  static constexpr uint32_t kTile = kM * D * 2;   // bytes of a 128 x D bf16 tile
+  static constexpr uint32_t kPTile = kM * kN * 2; // bytes of a 128 x 128 bf16 P tile
+  static constexpr int kBoxes = D / 64;           // 128B-swizzled boxes of 64 columns
+  static constexpr int kKSteps = D / 16;          // MMA k-steps of QK^T
+  static constexpr int kSlots = D == 128 ? 3 : 4; // what fits beside Q and P
+  static constexpr size_t kSmem =
+      1024 + 2 * kTile + 2 * kPTile + kSlots * static_cast<size_t>(kTile) + sizeof(Bars);
+};
+static_assert(Cfg<128>::kSmem <= 232448, "shared memory of the D = 128 kernel");
+static_assert(Cfg<64>::kSmem <= 232448, "shared memory of the D = 64 kernel");
 
 // ---------------------------------------------------------------- PTX helpers
 
 // Bounded wait for the phase of parity `parity` of barrier b. Returns false (after recording
-// the timeout) if it expired or another role already aborted.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, Bars* bars,
+// the timeout) if it expired or another role already aborted. Inlined: a call inside the
+// register-reallocated regions of the kernel would pin every warp to one register count.
+__device__ __forceinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, Bars* bars,
                                            int32_t* status) {
   const uint64_t t0 = gtimer();
   while (true) {
@@ -118,21 +126,6 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, Bars* b
 __device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, Bars* bars,
                                          int32_t* status) {
   return mbar_try(b, parity) || wait_bar_slow(b, parity, bars, status);
-}
-// Barrier of the two warps that share TMEM lanes, which also agree on whether to go on: both
-// get the AND of their flags, so a warp that gave up (a timed-out wait) takes its partner with
-// it instead of leaving it at the barrier. Both warps make the same sequence of these calls.
-__device__ __forceinline__ bool pair_and(int id, bool go) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred a, b;\n\t"
-      "setp.ne.u32 a, %1, 0;\n\t"
-      "barrier.cta.red.and.pred b, %2, 64, a;\n\t"
-      "selp.u32 %0, 1, 0, b;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(go)), "r"(id)
-      : "memory");
-  return r != 0;
 }
 // Two fp32 lanes per instruction (sm_100 f32x2 arithmetic).
 struct f2 {
@@ -193,26 +186,38 @@ __device__ __forceinline__ void mma_s4(uint32_t d, uint32_t alo, uint32_t blo, u
       : "memory");
 }
 #undef STEM_MMA_SS
-// P V group: O += P V over the 128 keys, A = P from TMEM (bf16 pairs, 8 columns per k-step of
-// 16 keys: keys 16kk.. at column a0 + kPCol[kk]), B = V MN-major in shared memory (16 key rows
-// of 128 bytes per k-step: descriptor offset kk * 128). acc0 = 0 starts O afresh.
-// operands: %0 d, %1 a0, %2 b_lo, %3 hi, %4 idesc, %5 acc0
-#define STEM_MMA_TS(COL, OFF)                                                              \
-  "add.u32 x, %1, " #COL ";\n\tadd.u32 y, %2, " #OFF ";\n\tmov.b64 b, {y, %3};\n\t"       \
-  "tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %4, pt;\n\t"
-__device__ __forceinline__ void mma_pv8(uint32_t d, uint32_t a0, uint32_t blo, uint32_t hi,
+// P V group: O += P V over the 128 keys, both operands in shared memory. A = P, K-major
+// 128B-swizzled like a Q tile (keys 16kk.. of k-step kk at descriptor offset
+// (kk / 4) * 1024 + (kk % 4) * 2); B = V MN-major (16 key rows of 128 bytes per k-step:
+// descriptor offset kk * 128). acc0 = 0 starts O afresh.
+// operands: %0 d, %1 a_lo, %2 b_lo, %3 hi, %4 idesc, %5 acc0
+#define STEM_MMA_PV(AOFF, BOFF)                                                            \
+  "add.u32 x, %1, " #AOFF ";\n\tadd.u32 y, %2, " #BOFF ";\n\t"                             \
+  "mov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"                                        \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, pt;\n\t"
+__device__ __forceinline__ void mma_pv8(uint32_t d, uint32_t alo, uint32_t blo, uint32_t hi,
                                         uint32_t idesc, uint32_t acc0) {
   asm volatile(
-      "{\n\t.reg .pred p0, pt;\n\t.reg .b32 x, y;\n\t.reg .b64 b;\n\t"
+      "{\n\t.reg .pred p0, pt;\n\t.reg .b32 x, y;\n\t.reg .b64 a, b;\n\t"
       "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 pt, %4, %4;\n\t"
-      "mov.b64 b, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p0;\n\t"
-      STEM_MMA_TS(8, 128) STEM_MMA_TS(16, 256) STEM_MMA_TS(24, 384) STEM_MMA_TS(32, 512)
-      STEM_MMA_TS(40, 640) STEM_MMA_TS(48, 768) STEM_MMA_TS(56, 896)
-      "}" ::"r"(d), "r"(a0), "r"(blo), "r"(hi), "r"(idesc), "r"(acc0)
+      "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p0;\n\t"
+      STEM_MMA_PV(2, 128) STEM_MMA_PV(4, 256) STEM_MMA_PV(6, 384) STEM_MMA_PV(1024, 512)
+      STEM_MMA_PV(1026, 640) STEM_MMA_PV(1028, 768) STEM_MMA_PV(1030, 896)
+      "}" ::"r"(d), "r"(alo), "r"(blo), "r"(hi), "r"(idesc), "r"(acc0)
       : "memory");
 }
-#undef STEM_MMA_TS
+#undef STEM_MMA_PV
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
 
 // Work item t -> (b, g, i, head pair): kv-head-group-major, query blocks in the plan's
 // heavy-first order, the ceil(G/2) head pairs of a group adjacent. Tile A is head g*G + 2p,
@@ -346,20 +351,6 @@ struct Seq {
   }
 };
 
-// Fill indices of the K/V tiles each step's products take, in the MMA thread's issue order:
-// S_A(0), S_B(0), then for every step c with successor x: P V_A(c), S_A(x), P V_B(c), S_B(x).
-// A block both heads keep is one tile. The MMA thread (which takes the tiles) and the release
-// thread (which frees them) run this same recurrence, so both agree on every slot.
-struct TileOrder {
-  int32_t next = 0;
-  int32_t kA = 0, kB = 0, vA = 0, vB = 0;  // tiles of the latest S_A, S_B, PV_A, PV_B
-  // call in issue order: k_a(x0), k_b(x0); then per step c: v_a(), k_a(x), v_b(c), k_b(x)
-  __device__ __forceinline__ void k_a() { kA = next++; }
-  __device__ __forceinline__ void k_b(bool shared) { kB = shared ? kA : next++; }
-  __device__ __forceinline__ void v_a() { vA = next++; }
-  __device__ __forceinline__ void v_b(bool shared) { vB = shared ? vA : next++; }
-};
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -369,11 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const uint32_t* __restrict__ sched, __nv_bfloat16* __restrict__ out,
                       int32_t* status, int withhold_q) {
   using C = Cfg<D>;
+  constexpr int kSlots = C::kSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* q_tiles = smem;                   // [tile A, tile B][kTile]
-  unsigned char* kv_tiles = smem + 2 * C::kTile;   // [kSlots][kTile]
+  unsigned char* q_tiles = smem;                        // [tile A, tile B][kTile]
+  unsigned char* p_tiles = smem + 2 * C::kTile;         // [tile A, tile B][kPTile]
+  unsigned char* kv_tiles = p_tiles + 2 * C::kPTile;    // [kSlots][kTile]
   Bars* bars = reinterpret_cast<Bars*>(kv_tiles + kSlots * C::kTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -384,9 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], kSoftmaxThreads);
-      mbar_init(&bars->o_full[s], 1);
-      mbar_init(&bars->o_empty[s], kSoftmaxThreads);
+      mbar_init(&bars->s_free[s], kGroupThreads);
+      mbar_init(&bars->p_full[s], kGroupThreads);
+      mbar_init(&bars->pv_done[s], 1);
+      mbar_init(&bars->o_empty[s], kGroupThreads);
     }
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -411,18 +405,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
+  // Registers: the launch gives every thread 168 (12 warps; a scheduler holds three). The
+  // producer / MMA warpgroup needs few and gives them to the two softmax warpgroups, whose
+  // threads each hold a row of 128 scores and its 64 packed P words: 4 x 32 x 72 +
+  // 8 x 32 x 216 = 384 x 168.
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
+   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)));
       const uint64_t pol_kv = policy_evict_last(), pol_q = policy_evict_first();
-      // The ring is filled in the order the MMA thread first uses tiles: for step c with
-      // lookahead x: V(c, A), K(x, A), V(c, B), K(x, B); a block both heads keep is one tile.
+      // The ring is filled in the order the MMA thread uses tiles: per step c with successor
+      // x, K(x, A), K(x, B), V(c, A), V(c, B) inside an item, V before K when x starts the
+      // next item; a block both heads keep is one tile.
       int64_t f = 0;
-      int64_t slot_round[kSlots];
-      for (int s = 0; s < kSlots; ++s) slot_round[s] = -1;
+      int64_t slot_round[kMaxSlots];
+      for (int s = 0; s < kMaxSlots; ++s) slot_round[s] = -1;
       int64_t q_loads[2] = {0, 0};
       bool ok = true;
       auto fill = [&](const CUtensorMap* map, const Step& st, int blk) -> bool {
@@ -452,22 +453,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_loads[tile];
         return true;
       };
-      auto start_step = [&](const Step& st) -> bool {  // Q at item start, then K of tile A
+      auto fill_k = [&](const Step& st) -> bool {  // Q at an item's start, then the K tiles
         if (st.first) {
           if (!load_q(st, 0)) return false;
           if (st.has_b() && !load_q(st, 1)) return false;
         }
-        return fill(&tm_k, st, st.ba);
+        if (!fill(&tm_k, st, st.ba)) return false;
+        return !(st.has_b() && !st.shared()) || fill(&tm_k, st, st.bb);
+      };
+      auto fill_v = [&](const Step& st) -> bool {
+        if (!fill(&tm_v, st, st.ba)) return false;
+        return !(st.has_b() && !st.shared()) || fill(&tm_v, st, st.bb);
       };
       Seq seq;
       seq.init(items, G, nb, Hkv, Hq, cap, plan, sched, bars, counter, status);
       Step x;
       bool have = seq.next(x);
       if (seq.failed) ok = false;
-      if (have) {
-        ok = start_step(x);
-        if (ok && x.has_b() && !x.shared()) ok = fill(&tm_k, x, x.bb);
-      }
+      if (have) ok = fill_k(x);
       while (have && ok) {
         const Step c = x;
         have = seq.next(x);
@@ -475,10 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        if (!(ok = fill(&tm_v, c, c.ba))) break;
-        if (have && !(ok = start_step(x))) break;
-        if (c.has_b() && !c.shared() && !(ok = fill(&tm_v, c, c.bb))) break;
-        if (have && x.has_b() && !x.shared() && !(ok = fill(&tm_k, x, x.bb))) break;
+        if (have && !x.first)
+          ok = fill_k(x) && fill_v(c);
+        else
+          ok = fill_v(c) && (!have || fill_k(x));
       }
       if (!ok) {  // abort: let issued copies land before the CTA can exit
         for (int s = 0; s < kSlots; ++s)
@@ -489,34 +492,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per head step T of step c (lookahead x): the waits for P_T(c) and the V tile of c (and,
-    // at an item's first step, the epilogue's release of O_T) are tested together, so their
-    // latencies overlap, then P V_T(c) goes out; then the wait for the K tile of x (and, when
-    // x starts an item, its Q tile) and S_T(x), with one commit after the S group. Bookkeeping
-    // is 32-bit: phase bits and tile numbers (tile f sits in slot f % kSlots, fill round
-    // f / kSlots).
+    // Inside an item, per step c with successor x: S_A(x), S_B(x), P V_A(c), P V_B(c). S_T(x)
+    // waits for its K tile, its Q tile when x starts an item and the softmax's read of the
+    // previous S_T (s_free); P V_T(c) for P_T(c), its V tile and, at an item's first step,
+    // the epilogue's read of O_T. When x starts the next item, P V of c goes first. A tile
+    // is released by a commit after the last product that reads it.
     if (lane == 0) {
       constexpr uint32_t idesc_s = instr_desc(kM, kN, false);
       constexpr uint32_t idesc_o = instr_desc(kM, D, true);
-      constexpr uint32_t kTileU = C::kTile >> 4;  // a tile's size in descriptor units
+      constexpr uint32_t kTileU = C::kTile >> 4;    // a tile's size in descriptor units
+      constexpr uint32_t kPTileU = C::kPTile >> 4;
       const uint32_t hi = smem_desc_hi(1024);
       const uint32_t q_lo = smem_desc_lo(su32(q_tiles), 16);
+      const uint32_t p_lo = smem_desc_lo(su32(p_tiles), 16);
       const uint32_t k_lo = smem_desc_lo(su32(kv_tiles), 16);
       const uint32_t v_lo = smem_desc_lo(su32(kv_tiles), kN * 128);
-      uint32_t qph = 0;  // bit T: parity of the next q_full[T] wait
-      uint32_t pph = 0;  // bit T: parity of the next p_full[T] wait
-      uint32_t oph = 0;  // bit T: items finished on tile T, mod 2 (o_empty waits take the other)
+      int32_t f = 0;               // K/V tiles taken, in fill order
+      int32_t nq[2] = {0, 0};      // Q tiles taken per tile (q_full phases)
+      int32_t ns[2] = {0, 0};      // S products issued per tile
+      int32_t np[2] = {0, 0};      // P V groups issued per tile (p_full phases)
+      int32_t no[2] = {0, 0};      // items started per tile (o_empty phases)
       bool ok = true;
-      TileOrder order;
-      auto kv_try = [&](int32_t f) {
-        return mbar_try(&bars->kv_full[f % kSlots], static_cast<uint32_t>(f / kSlots) & 1u);
+      auto kv_try = [&](int32_t t) {
+        return mbar_try(&bars->kv_full[t % kSlots], static_cast<uint32_t>(t / kSlots) & 1u);
       };
-      auto kv_wait = [&](int32_t f) {
-        return wait_bar(&bars->kv_full[f % kSlots], static_cast<uint32_t>(f / kSlots) & 1u, bars,
+      auto kv_wait = [&](int32_t t) {
+        return wait_bar(&bars->kv_full[t % kSlots], static_cast<uint32_t>(t / kSlots) & 1u, bars,
                         status);
       };
-      auto s_group = [&](int tl, int32_t f) {
-        const uint32_t a = q_lo + tl * kTileU, b = k_lo + static_cast<uint32_t>(f % kSlots) * kTileU;
+      auto issue_s = [&](const Step& s, int tl, int32_t kt, bool wait_k, bool release_k) -> bool {
+        const uint32_t qp = static_cast<uint32_t>(nq[tl]) & 1u;
+        const uint32_t sp = static_cast<uint32_t>(ns[tl] - 1) & 1u;
+        bool r = !wait_k || kv_try(kt);
+        if (s.first) r &= mbar_try(&bars->q_full[tl], qp);
+        if (ns[tl] > 0) r &= mbar_try(&bars->s_free[tl], sp);
+        if (!r && !((!wait_k || kv_wait(kt)) &&
+                    (!s.first || wait_bar(&bars->q_full[tl], qp, bars, status)) &&
+                    (ns[tl] == 0 || wait_bar(&bars->s_free[tl], sp, bars, status))))
+          return false;
+        if (s.first) ++nq[tl];
+        ++ns[tl];
+        tc_fence_after();
+        const uint32_t a = q_lo + tl * kTileU;
+        const uint32_t b = k_lo + static_cast<uint32_t>(kt % kSlots) * kTileU;
         if constexpr (C::kKSteps == 8) {
           mma_s8(tmem + tl * 128, a, b, hi, idesc_s);
         } else {
@@ -524,35 +542,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_s4(tmem + tl * 128, a, b, hi, idesc_s);
         }
         tc_commit(&bars->s_full[tl]);
+        if (s.last) tc_commit(&bars->q_empty[tl]);
+        if (release_k) tc_commit(&bars->kv_empty[kt % kSlots]);
+        return true;
       };
-      auto pv_group = [&](int tl, int32_t f, bool first) {
-        static_assert(kN / 16 == 8, "one P V group is 8 products of 16 keys");
-        mma_pv8(tmem + 256 + tl * 128, tmem + tl * 128,
-                v_lo + static_cast<uint32_t>(f % kSlots) * kTileU, hi, idesc_o, first ? 0u : 1u);
+      auto issue_pv = [&](const Step& c, int tl, int32_t vt, bool wait_v,
+                          bool release_v) -> bool {
+        const uint32_t pp = static_cast<uint32_t>(np[tl]) & 1u;
+        const uint32_t op = static_cast<uint32_t>(no[tl] - 1) & 1u;
+        const bool wo = c.first && no[tl] > 0;
+        bool r = mbar_try(&bars->p_full[tl], pp);
+        if (wait_v) r &= kv_try(vt);
+        if (wo) r &= mbar_try(&bars->o_empty[tl], op);
+        if (!r && !(wait_bar(&bars->p_full[tl], pp, bars, status) &&
+                    (!wait_v || kv_wait(vt)) &&
+                    (!wo || wait_bar(&bars->o_empty[tl], op, bars, status))))
+          return false;
+        if (c.first) ++no[tl];
+        ++np[tl];
+        tc_fence_after();
+        mma_pv8(tmem + 256 + tl * 128, p_lo + tl * kPTileU,
+                v_lo + static_cast<uint32_t>(vt % kSlots) * kTileU, hi, idesc_o,
+                c.first ? 0u : 1u);
+        tc_commit(&bars->pv_done[tl]);
+        if (release_v) tc_commit(&bars->kv_empty[vt % kSlots]);
+        return true;
+      };
+      auto s_step = [&](const Step& s) -> bool {
+        const bool sh = s.has_b() && s.shared();
+        const int32_t ka = f++;
+        if (!issue_s(s, 0, ka, true, !sh)) return false;
+        if (!s.has_b()) return true;
+        const int32_t kb = sh ? ka : f++;
+        return issue_s(s, 1, kb, !sh, true);
+      };
+      auto pv_step = [&](const Step& c) -> bool {
+        const bool sh = c.has_b() && c.shared();
+        const int32_t va = f++;
+        if (!issue_pv(c, 0, va, true, !sh)) return false;
+        if (!c.has_b()) return true;
+        const int32_t vb = sh ? va : f++;
+        return issue_pv(c, 1, vb, !sh, true);
       };
       Seq seq;
       seq.init(items, G, nb, Hkv, Hq, cap, plan, sched, bars, nullptr, status);
       Step x;
       bool have = seq.next(x);
       if (seq.failed) ok = false;
-      if (have) {  // S of the first step
-        order.k_a();
-        ok = wait_bar(&bars->q_full[0], 0, bars, status) && kv_wait(order.kA);
-        if (ok) {
-          tc_fence_after();
-          s_group(0, order.kA);
-        }
-        qph ^= 1u;
-        if (ok && x.has_b()) {
-          order.k_b(x.shared());
-          ok = wait_bar(&bars->q_full[1], 0, bars, status) && (x.shared() || kv_wait(order.kB));
-          if (ok) {
-            tc_fence_after();
-            s_group(1, order.kB);
-          }
-          qph ^= 2u;
-        }
-      }
+      if (have) ok = s_step(x);
       while (have && ok) {
         const Step c = x;
         have = seq.next(x);
@@ -560,245 +597,142 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // ---------------- head A: P V_A(c), then S_A(x)
-        order.v_a();
-        {
-          bool r = mbar_try(&bars->p_full[0], pph & 1u) & kv_try(order.vA);
-          if (c.first) r &= mbar_try(&bars->o_empty[0], (oph & 1u) ^ 1u);
-          if (!r) {
-            ok = wait_bar(&bars->p_full[0], pph & 1u, bars, status) && kv_wait(order.vA) &&
-                 (!c.first || wait_bar(&bars->o_empty[0], (oph & 1u) ^ 1u, bars, status));
-            if (!ok) break;
-          }
-          pph ^= 1u;
-        }
-        tc_fence_after();
-        pv_group(0, order.vA, c.first);
-        if (c.last) {
-          tc_commit(&bars->o_full[0]);
-          oph ^= 1u;
-        }
-        if (have) {
-          order.k_a();
-          const bool qx = x.first;
-          bool r = kv_try(order.kA);
-          if (qx) r &= mbar_try(&bars->q_full[0], qph & 1u);
-          if (!r) {
-            ok = kv_wait(order.kA) && (!qx || wait_bar(&bars->q_full[0], qph & 1u, bars, status));
-            if (!ok) break;
-          }
-          if (qx) qph ^= 1u;
-          tc_fence_after();
-          s_group(0, order.kA);
-        }
-        // ---------------- head B: P V_B(c) when step c has a head B, then S_B(x) when step x
-        // has one (independently: an item without head B can be followed by one with it)
-        const bool xb = have && x.has_b();
-        if (c.has_b()) {
-          order.v_b(c.shared());
-          const bool wv = !c.shared();
-          bool r = mbar_try(&bars->p_full[1], (pph >> 1) & 1u);
-          if (wv) r &= kv_try(order.vB);
-          if (c.first) r &= mbar_try(&bars->o_empty[1], ((oph >> 1) & 1u) ^ 1u);
-          if (!r) {
-            ok = wait_bar(&bars->p_full[1], (pph >> 1) & 1u, bars, status) &&
-                 (!wv || kv_wait(order.vB)) &&
-                 (!c.first ||
-                  wait_bar(&bars->o_empty[1], ((oph >> 1) & 1u) ^ 1u, bars, status));
-            if (!ok) break;
-          }
-          pph ^= 2u;
-          tc_fence_after();
-          pv_group(1, order.vB, c.first);
-          // no S_B follows this P V to cover it: release its V slot from here
-          if (!xb) tc_commit(&bars->kv_empty[order.vB % kSlots]);
-          if (c.last) {
-            tc_commit(&bars->o_full[1]);
-            oph ^= 2u;
-          }
-        }
-        if (xb) {
-          order.k_b(x.shared());
-          const bool qx = x.first, wk = !x.shared();
-          bool r = true;
-          if (wk) r &= kv_try(order.kB);
-          if (qx) r &= mbar_try(&bars->q_full[1], (qph >> 1) & 1u);
-          if (!r) {
-            ok = (!wk || kv_wait(order.kB)) &&
-                 (!qx || wait_bar(&bars->q_full[1], (qph >> 1) & 1u, bars, status));
-            if (!ok) break;
-          }
-          if (qx) qph ^= 2u;
-          tc_fence_after();
-          s_group(1, order.kB);
-        }
+        if (have && !x.first)
+          ok = s_step(x) && pv_step(c);
+        else
+          ok = pv_step(c) && (!have || s_step(x));
       }
       // make sure every issued product has completed before TMEM is released
       tc_commit(&bars->drain);
       drain_bar(&bars->drain, 0);
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
     // ------------------------------------------------------------ softmax + epilogue
-    constexpr int kH = kN / 2;          // key columns per thread
-    constexpr int kDH = D / 2;          // output columns per thread
+    const int tl = (warp - 4) >> 2;     // 0: head A (warps 4-7), 1: head B (warps 8-11)
     const int sub = warp & 3;           // TMEM sub-partition of this warp
-    const int half = (warp - 2) >> 2;   // 0: columns [0, 64), 1: [64, 128)
     const int row = sub * 32 + lane;    // query row within the tile
-    const int bar_id = 1 + sub;         // named barrier of the warp pair (sub, sub + 4)
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const uint32_t s_addr = tmem + tl * 128 + lane_off;
+    const uint32_t o_addr = tmem + 256 + tl * 128 + lane_off;
+    const uint32_t p_row = su32(p_tiles + tl * C::kPTile) + static_cast<uint32_t>(row) * 128;
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
     const float sl2 = 1.4426950408889634f * rsqrtf(static_cast<float>(D));
-    // per-tile state lives in scalars (passed by reference) so it stays in registers
-    int64_t steps_a = 0, steps_b = 0, outs_a = 0, outs_b = 0;
-    int xp = 0;  // exchange-slot parity
-    float m_a = 0.f, m_b = 0.f, l_a = 0.f, l_b = 0.f;
+    int32_t ns = 0;       // S_T tiles read
+    int32_t np = 0;       // P_T tiles written (each followed by one P V_T group)
+    int32_t pv_seen = 0;  // P V_T groups known complete
+    float m_run = 0.f, lsum = 0.f;
     bool ok = true;
-    // The release thread frees ring slots and Q tiles: when S_T of a step is complete, so is
-    // every product issued before it (K of this step unless head B still needs it, V of the
-    // previous step, Q after the item's last S).
-    const bool releaser = (warp == 2 && lane == 0);
-    auto release = [&](int64_t tile) {
-      if (tile >= 0) mbar_arrive(&bars->kv_empty[tile % kSlots]);
-    };
-    // one step of tile tl on key block blk; returns false on abort
-    // Row max of this thread's half of S (log2 units, scale folded in) agreed with the partner
-    // half through shared memory; both warps of the pair call it at the same point.
-    auto pair_max = [&](const uint32_t* sr, bool& ok) -> float {
-      float mx[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
-#pragma unroll
-      for (int c = 4; c < kH; c += 2)
-        mx[(c >> 1) & 3] =
-            max3(mx[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-      float mt = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      bars->xch[xp][half][row] = mt;
-      ok = pair_and(bar_id, true);
-      mt = fmaxf(mt, bars->xch[xp][half ^ 1][row]) * sl2;  // both halves alike
-      xp ^= 1;
-      return mt;
-    };
-    // P = exp2(S * sl2 - m_run) packed to bf16 over column pairs [C0, C1) of this thread's
-    // half; adds to the partial row sums the bf16 values that enter P V (mixed-precision adds
-    // take each half of a packed pair as it is), so the normaliser and the products see the
-    // same P and a row that one key dominates returns that key's V row.
-    auto exp_pack = [&](const uint32_t* sr, float m_run, uint32_t* p, f2* sum, auto c0,
-                        auto c1) {
-      const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
-#pragma unroll
-      for (int c = decltype(c0)::value; c < decltype(c1)::value; ++c) {
-        const f2 x = fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
-        const f2 e{ex2(x.x), ex2(x.y)};
-        p[c] = pack_bf16(e.x, e.y);
-        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-            "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-            : "+f"(sum[c & 1].x), "+f"(sum[c & 1].y)
-            : "r"(p[c]));
-      }
-    };
-    auto exp_all = [&](const uint32_t* sr, float m_run, uint32_t* p) -> float {
-      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
-      exp_pack(sr, m_run, p, sum, std::integral_constant<int, 0>{},
-               std::integral_constant<int, kH / 2>{});
-      return (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
-    };
-    auto diag_mask = [&](uint32_t* sr, auto c0, auto c1) {
-#pragma unroll
-      for (int c = decltype(c0)::value; c < decltype(c1)::value; ++c)
-        if (half * kH + c > row) sr[c] = __float_as_uint(-INFINITY);
-    };
-    // One step of tile tl on key block blk; returns false on abort.
-    //
-    // The exponentials use the row's running reference max m_run. The first step of an item
-    // sets it to the exact row max; later steps form P against it without looking for their
-    // own max, and only if some row's partial sum reaches 2^16 (a score that grew by ~10 in
-    // log2 units, or an overflow) does the pair take the exact max, rescale O and recompute.
-    // The result is exact either way: the final 1/l uses the same reference as P.
-    //
-    // Barriers of the warp pair per step, the same sequence on both warps: [first step: max
-    // exchange] check; if the check fails: agree on going on, then the max exchange. A warp
-    // that gives up joins every barrier its partner will meet with "stop".
-    auto step = [&](int tl, int blk, int qi, bool first, int64_t& nsteps, float& m_run,
-                    float& lsum, int64_t rel_k, int64_t rel_v, bool rel_q) -> bool {
-      const int64_t r = nsteps++;
-      bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(r & 1), bars, status);
-      if (!__all_sync(0xffffffffu, w)) {
-        pair_and(bar_id, false);  // [first: the max exchange | the check]
-        if (!first) pair_and(bar_id, false);  // the agreement after a failed check
-        return false;
-      }
-      if (releaser) {
-        release(rel_k);
-        release(rel_v);
-        if (rel_q) mbar_arrive(&bars->q_empty[tl]);
-      }
-      tc_fence_after();
-      const uint32_t s_addr = tmem + tl * 128 + lane_off;
-      uint32_t sr[kH];
-      uint32_t p[kH / 2];
-      bool ok = true;
-#pragma unroll
-      for (int c = 0; c < kH / 32; ++c) TC_LD32(s_addr + half * kH + 32 * c, (sr + 32 * c));
-      tc_wait_ld_r32(sr);
-      tc_wait_ld_r32(sr + 32);
-      if (blk == qi) {  // the diagonal block: token-causal
-        diag_mask(sr, std::integral_constant<int, 0>{}, std::integral_constant<int, kH>{});
-      }
-      if (first) {
-        m_run = pair_max(sr, ok);
-        if (!ok) return false;
-        lsum = 0.f;
-      }
-      float part = exp_all(sr, m_run, p);
-      const bool small = part < 65536.0f;  // false for inf and NaN too
-      if (!pair_and(bar_id, __all_sync(0xffffffffu, small))) {
-        if (!pair_and(bar_id, true)) return false;
-        // a row's scores grew past the reference (never on a first step, whose reference is
-        // the exact max): the warp rescales its part of O_T (each row by its own factor, 1
-        // where the max did not grow) and recomputes P. The previous P V of this tile is
-        // complete: this S was issued after it and s_full tracks every earlier product.
-        const float mt = pair_max(sr, ok);
-        if (!ok) return false;
-        const float m_new = fmaxf(m_run, mt);
-        const float alpha = ex2(m_run - m_new);
-        m_run = m_new;
-        lsum *= alpha;
-        const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
-#pragma unroll 1
-        for (int c = 0; c < kDH / 32; ++c) {
-          uint32_t o[32];
-          TC_LD32(o_addr + 32 * c, o);
-          tc_wait_ld_r32(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          TC_ST32(o_addr + 32 * c, o);
-        }
-        tc_wait_st();
-        part = exp_all(sr, m_run, p);
-      }
-      // P over S_T columns [0, 64): this half's keys go to columns half*32 .. +32 (both halves
-      // finished reading S before the pair's check barrier above)
-      TC_ST32(s_addr + half * (kH / 2), p);
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[tl]);
-      lsum += part;
+    // Until the latest P V_T has completed: P_T may then be rewritten and O_T is final.
+    auto pv_wait = [&]() -> bool {
+      if (pv_seen >= np) return true;
+      const bool w = wait_bar(&bars->pv_done[tl], static_cast<uint32_t>(np - 1) & 1u, bars,
+                              status);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      pv_seen = np;
       return true;
     };
-    auto epilogue = [&](int tl, const Item& it, int64_t& nouts, float lsum) -> bool {
-      const int64_t r = nouts++;
-      bool w = wait_bar(&bars->o_full[tl], static_cast<uint32_t>(r & 1), bars, status);
-      w = __all_sync(0xffffffffu, w);
-      bars->xl[tl][half][row] = lsum;
-      if (!pair_and(bar_id, w)) return false;
-      const float inv = 1.0f / (lsum + bars->xl[tl][half ^ 1][row]);
+    // One step of this head on key block blk; returns false on abort.
+    auto step = [&](int blk, int qi, bool first) -> bool {
+      const bool w = wait_bar(&bars->s_full[tl], static_cast<uint32_t>(ns) & 1u, bars, status);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      ++ns;
+      tc_fence_after();
+      uint32_t sr[kN];
+      TC_LD32(s_addr, sr);
+      TC_LD32(s_addr + 32, (sr + 32));
+      TC_LD32(s_addr + 64, (sr + 64));
+      TC_LD32(s_addr + 96, (sr + 96));
+      tc_wait_ld_r32(sr);
+      tc_wait_ld_r32(sr + 32);
+      tc_wait_ld_r32(sr + 64);
+      tc_wait_ld_r32(sr + 96);
+      tc_fence_before();
+      mbar_arrive(&bars->s_free[tl]);  // the next S_T may overwrite these columns
+      if (blk == qi) {  // the diagonal block: token-causal
+#pragma unroll
+        for (int c = 0; c < kN; ++c)
+          if (c > row) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float mq[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mq[e] = __uint_as_float(sr[e]);
+#pragma unroll
+      for (int c = 4; c < kN; c += 2)
+        mq[(c >> 1) & 3] =
+            max3(mq[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      const float mx = max3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * sl2;
+      if (first) {
+        m_run = mx;
+        lsum = 0.f;
+      } else {
+        const bool need = mx > m_run + kRescale;
+        if (__any_sync(0xffffffffu, need)) {
+          // rows whose max moved past the reference take the new max and rescale their row
+          // of O_T (complete once the latest P V_T is); the others multiply by 1
+          if (!pv_wait()) return false;
+          const float alpha = need ? ex2(m_run - mx) : 1.0f;
+          if (need) m_run = mx;
+          lsum *= alpha;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            TC_LD32(o_addr + 32 * c, o);
+            tc_wait_ld_r32(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            TC_ST32(o_addr + 32 * c, o);
+          }
+          tc_wait_st();
+        }
+      }
+      // P = exp2(S * sl2 - m_run) packed to bf16; the row sum adds the bf16 values that enter
+      // P V (mixed-precision adds take each half of a packed pair as it is), so the
+      // normaliser and the products see the same P and a row that one key dominates returns
+      // that key's V row.
+      uint32_t p[kN / 2];
+      f2 sum[2] = {f2{0.f, 0.f}, f2{0.f, 0.f}};
+      {
+        const f2 scl{sl2, sl2}, neg{-m_run, -m_run};
+#pragma unroll
+        for (int c = 0; c < kN / 2; ++c) {
+          const f2 x =
+              fma2(f2{__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])}, scl, neg);
+          p[c] = pack_bf16(ex2(x.x), ex2(x.y));
+          asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+              "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+              : "+f"(sum[c & 1].x), "+f"(sum[c & 1].y)
+              : "r"(p[c]));
+        }
+      }
+      if (!pv_wait()) return false;  // the previous P V_T has read P_T
+      // the row's 256 bytes in the 128B-swizzled K-major layout of a TMA box (two boxes of 64
+      // keys, 16 KB apart; 16-byte chunk j of row r at r*128 + ((j ^ (r % 8)) * 16))
+#pragma unroll
+      for (int k = 0; k < kN / 8; ++k)
+        st_shared_v4(p_row + (k >> 3) * (kM * 128) + (((k & 7) ^ swz) << 4), p[4 * k],
+                     p[4 * k + 1], p[4 * k + 2], p[4 * k + 3]);
+      fence_proxy_async_smem();  // the tensor cores read P through the async proxy
+      tc_fence_before();         // and O_T after a rescale
+      mbar_arrive(&bars->p_full[tl]);
+      ++np;
+      lsum += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
+      return true;
+    };
+    // At the item's end: when its last P V is complete, O * (1/l) -> bf16 -> global
+    // (streaming stores), then O_T is released.
+    auto epilogue = [&](const Item& it) -> bool {
+      if (!pv_wait()) return false;
+      const float inv = 1.0f / lsum;
       tc_fence_after();
       const int h = tl == 0 ? it.hA : it.hB;
       __nv_bfloat16* dst = out + ((static_cast<int64_t>(it.b) * Hq + h) * S +
-                                  static_cast<int64_t>(it.i) * kM + row) * D + half * kDH;
+                                  static_cast<int64_t>(it.i) * kM + row) * D;
       const bool valid = static_cast<int64_t>(it.i) * kM + row < S;  // partial last block
-      const uint32_t o_addr = tmem + 256 + tl * 128 + half * kDH + lane_off;
-#pragma unroll
-      for (int c = 0; c < kDH / 32; ++c) {
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         TC_LD32(o_addr + 32 * c, o);
         tc_wait_ld_r32(o);
@@ -817,46 +751,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->o_empty[tl]);
       return true;
     };
-    TileOrder order;  // replica of the MMA thread's tile numbering
-    bool have_prev = false, prev_has_b = false, prev_shared = false;
     for (int64_t n = 0; ok; ++n) {
       int64_t t = -1;
-      const bool got = read_item(bars, n, status, &t);
-      // both warps of a pair go on together (a failed read takes the partner out too)
-      if (!pair_and(bar_id, __all_sync(0xffffffffu, got))) {
+      if (!__all_sync(0xffffffffu, read_item(bars, n, status, &t))) {
         ok = false;
         break;
       }
       if (t < 0) break;
       const Item it = decode(t, G, nb, Hkv, plan.order);
+      if (tl == 1 && it.hB < 0) continue;  // a lone head A
       const int cnt = plan.k[it.i];
       const uint32_t* srow = sched_row(sched, it, Hkv, G, cap, plan);
       uint32_t e_next = srow[0];  // loaded one step ahead, as in Seq
       for (int j = 0; j < cnt && ok; ++j) {
         const uint32_t e = e_next;
         if (j + 1 < cnt) e_next = srow[j + 1];
-        Step x;
-        x.it = it;
-        sched_step(e, it.i, x.ba, x.bb);
-        const bool has_b = x.has_b(), shared = x.shared();
-        if (have_prev) order.v_a();
-        order.k_a();
-        if (have_prev && prev_has_b) order.v_b(prev_shared);
-        if (has_b) order.k_b(shared);
-        const int64_t rka = (has_b && shared) ? -1 : order.kA;
-        const int64_t rva = (have_prev && !(prev_has_b && prev_shared)) ? order.vA : -1;
-        ok = step(0, x.ba, it.i, j == 0, steps_a, m_a, l_a, rka, rva, j == cnt - 1);
-        if (ok && has_b) {
-          const int64_t rvb = (have_prev && prev_has_b) ? order.vB : -1;
-          ok = step(1, x.bb, it.i, j == 0, steps_b, m_b, l_b, order.kB, rvb, j == cnt - 1);
-        }
-        have_prev = true;
-        prev_has_b = has_b;
-        prev_shared = shared;
+        int ba, bb;
+        sched_step(e, it.i, ba, bb);
+        ok = step(tl == 0 ? ba : bb, it.i, j == 0);
       }
       if (!ok) break;
-      ok = epilogue(0, it, outs_a, l_a);
-      if (ok && it.hB >= 0) ok = epilogue(1, it, outs_b, l_b);
+      ok = epilogue(it);
     }
   }
 
@@ -900,8 +815,7 @@ cudaError_t launch_sm100(const void* q, const void* k, const void* v, int B, int
       !make_map(&tv, v, static_cast<uint64_t>(B) * Hkv, S, D))
     return cudaErrorInvalidValue;
   // one CTA per SM: each CTA takes all 512 TMEM columns
-  const size_t smem = std::max<size_t>(1024 + (2 + kSlots) * Cfg<D>::kTile + sizeof(Bars),
-                                       120 * 1024);
+  const size_t smem = std::max<size_t>(Cfg<D>::kSmem, 120 * 1024);
   auto kern = attn_sm100_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
