@@ -52,10 +52,11 @@ SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # to the revision that capture measured.
 ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1617127936 + 1022252032,
                 "sources_sha256": "f1f6a322377075784866d5bc74d1f634f3e5a8dbecca15077f713344646eb0da"}
-# The same for the anti-diagonal estimator (stride 16) at that workload, from the capture in
-# profiles/antidiag_sm100_llama3-8b-128k.md.
-AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16, "bytes": 9513621504 + 749666816,
-              "sources_sha256": "a170d26289c250b936c431969e85cbcdbe77282f17e7f2640721f48784d9b454"}
+# The same for the anti-diagonal estimator (stride 16) at that workload: its two kernels (the
+# partials, then their merge into p), from the capture in profiles/antidiag_sm100_llama3-8b-128k.md.
+AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,
+              "bytes": 1427185920 + 673577728 + 681591808 + 59151104,
+              "sources_sha256": "aa36c32394ef44a84b0a36806edf3c23b6ef1f6a62623bd02499d8a7747b4312"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -284,8 +284,10 @@ int stem_sparse_attn_m(const void* q, const void* k, const void* v, int dtype, i
 
 /* Workspace bytes stem_prefill_ex needs for this shape and method. With STEM_SCORE_ANTIDIAG it
  * also holds the block probabilities (4 * B * Hq * nb * (nb+1) / 2 bytes) and the estimator's
- * scratch: up to 148 CTAs x 2 slots x (nb + 8 * ceil(S / (256 * stride))) x 512 bytes (about
- * 194 MB at S = 131072, block 128, stride 16). 0 for an invalid or empty request. Host only. */
+ * partials, per head 4 * (R*nb*(nb+1)/2 + c*n - 32*c*(c-1)/2 + 256*t*parts) bytes with
+ * n = S/stride groups, R = block/stride, c = ceil(n/32), t = ceil(n/128) and
+ * parts = ceil(ceil(n/256)/4) (about 690 MB at S = 131072, block 128, stride 16, B*Hq = 32).
+ * 0 for an invalid or empty request. Host only. */
 size_t stem_workspace_size_m(int B, int Hq, int Hkv, int S, int D, int block,
                              const stem_method_t* m);
 
