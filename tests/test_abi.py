@@ -144,15 +144,21 @@ def test_workspace_size_layout():
         S.stem_workspace_size(B, Hq, Hkv, 1024, D, block) > 0
     assert S.stem_workspace_size(B, Hq, Hkv, 1000, 96, block) == 0  # unsupported D
     assert S.stem_workspace_size(0, Hq, Hkv, Sq, D, block) == 0  # empty
-    # anti-diagonal scoring adds p (packed rows) and the estimator's per-CTA scratch:
-    # min(units, 148) CTAs x 2 slots of (nb + 8 * ceil((S/stride)/256)) * 128 floats
+    # anti-diagonal scoring adds p (packed rows) and the estimator's partials, per head:
+    # R*nb*(nb+1)/2 block sums, c*n - 32*c*(c-1)/2 chunk maxima (c = ceil(n/32) chunks of the
+    # n = S/stride groups) and each part's max and sum (t = ceil(n/128) query tiles, parts =
+    # ceil(ceil(n/256)/4) per tile), after a 256-byte work counter
     ad = S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8, score="antidiag", stride=16)
     assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad.__class__.from_buffer_copy(
         S.make_method("exp", rho_min=0.05, tau=64.0, k_min=8))) == n
     na = S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad)
     p_bytes = 4 * B * Hq * nb * (nb + 1) // 2
-    nred = Sq // 16
-    scratch = 4 * min(B * Hq * (nred // 128), 148) * 2 * (nb + 8 * (nred // 256)) * 128
+    nred, R = Sq // 16, block // 16
+    c, t = -(-nred // 32), -(-nred // 128)
+    parts = -(-(-(-nred // 256)) // 4)
+    scratch = 4 * B * Hq * (R * nb * (nb + 1) // 2 + c * nred - 32 * c * (c - 1) // 2 +
+                            2 * 128 * t * parts)
+    assert scratch == 688914432  # about 690 MB
     assert n + p_bytes + scratch + 256 <= na < n + p_bytes + scratch + 1024  # + work counter
     ad.stride = 24
     assert S.stem_workspace_size(B, Hq, Hkv, Sq, D, block, ad) == 0
