@@ -59,8 +59,8 @@ cudaError_t launch_select_p(const float* p, const float* vnorm, int B, int Hq, i
                             PlanDev plan, int64_t cap, SelMetric metric, int32_t* sel_idx,
                             int32_t* sel_cnt, float* m_out, cudaStream_t st);
 
-// Block-sparse attention, bfloat16 inputs on the tensor cores (attn_sm100.cu; block 64 falls to
-// the mma.sync kernel of attn_bf16.cu). `sched` is workspace of pairs_bytes() for the head-pair
+// Block-sparse attention, bfloat16 inputs on the tensor cores (attn_sm100.cu for block 128,
+// attn_sm100_b64.cu for block 64). `sched` is workspace of pairs_bytes() for the head-pair
 // step schedule (pairs.cu).
 cudaError_t launch_attn_bf16(const void* q, const void* k, const void* v, int B, int Hq,
                              int Hkv, int S, int D, int block, PlanDev plan, int64_t cap,
