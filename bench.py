@@ -50,8 +50,8 @@ SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1617127936 + 1022252032,
-                "sources_sha256": "f1f6a322377075784866d5bc74d1f634f3e5a8dbecca15077f713344646eb0da"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615689472 + 1021989632,
+                "sources_sha256": "12e6ae00e390bc7f6452bb88950792b384c32793118c2c968bb304839760462c"}
 # The same for the anti-diagonal estimator (stride 16) at that workload: its two kernels (the
 # partials, then their merge into p), from the capture in profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,
@@ -98,7 +98,7 @@ def _sources_sha(files):
 
 def attn_traffic(workload_name):
     if (workload_name == ATTN_TRAFFIC["workload"] and
-            _sources_sha(("attn_sm100.cu", "pairs.cu", "sm100.cuh")) ==
+            _sources_sha(("attn_sm100.cu", "attn_common.cuh", "pairs.cu", "sm100.cuh")) ==
             ATTN_TRAFFIC["sources_sha256"]):
         return ATTN_TRAFFIC["bytes"]
     return None

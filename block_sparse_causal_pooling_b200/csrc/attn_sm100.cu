@@ -389,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c.first) ++no[tl];
         ++np[tl];
         tc_fence_after();
+        static_assert(kN / 16 == 8, "one P V group is 8 products of 16 keys");
         mma_pv8(tmem + 256 + tl * 128, p_lo + tl * kPTileU,
                 v_lo + static_cast<uint32_t>(vt % kSlots) * kTileU, hi, idesc_o,
                 c.first ? 0u : 1u);
