@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           const __grid_constant__ CUtensorMap tm_v, int Hq, int Hkv, int S,
                           int nb, int64_t items, PlanDev plan, int64_t cap,
                           unsigned long long* counter, const uint32_t* __restrict__ sched,
-                          __nv_bfloat16* __restrict__ out, int32_t* status) {
+                          __nv_bfloat16* __restrict__ out, int32_t* status, int withhold_q) {
   using C = Cfg64<D>;
   constexpr int kSlots = C::kSlots;
   extern __shared__ unsigned char smem_raw[];
@@ -259,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Q of a tile at an item's start: block i of its pair's first head into rows 0-63, of the
       // second head (when there is one) into rows 64-127
       auto load_q = [&](const Step64& st, int tl) -> bool {
+        if (withhold_q && tl == 0 && q_loads[0] == 0) return true;  // test switch: never sent
         const int64_t r = q_loads[tl];
         if (!wait_bar(&bars->q_empty[tl], static_cast<uint32_t>((r & 1) ^ 1), bars, status))
           return false;
@@ -634,7 +635,7 @@ cudaError_t launch_b64(const void* q, const void* k, const void* v, int B, int H
   const int64_t grid = std::min<int64_t>(items, sm_count());
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(
       tq, tk, tv, Hq, Hkv, S, nb, items, plan, cap, counter, pairs_schedule(sched),
-      static_cast<__nv_bfloat16*>(out), status);
+      static_cast<__nv_bfloat16*>(out), status, g_withhold_q.load());
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
-"""The tensor-core kernels' bounded waits, on a B200 (attention, and the anti-diagonal
-estimator below): a wait that runs out (a Q tile the producer
+"""The tensor-core kernels' bounded waits, on a B200 (attention at block 128 and 64, and the
+anti-diagonal estimator below): a wait that runs out (a Q tile the producer
 never sends, via the library's test switch) ends the kernel with STEM_ERR_TIMEOUT in the status
 word instead of hanging it, and the CUDA context stays usable: the next call is exact again.
 """
@@ -19,8 +19,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def test_expired_wait_reports_timeout_and_the_context_survives():
-    w = wl.LLAMA_32K.replace(name="timeout-4k", Hq=8, Hkv=2, S=4096)
+@pytest.mark.parametrize("block", [128, 64])
+def test_expired_wait_reports_timeout_and_the_context_survives(block):
+    w = wl.LLAMA_32K.replace(name=f"timeout-4k-blk{block}", Hq=8, Hkv=2, S=4096, block=block)
     q, k, v = wl.make_inputs(w, "cpu")
     dq, dk, dv = (t.to(DEV) for t in (q, k, v))
     status = torch.full((1,), 7, dtype=torch.int32, device=DEV)
