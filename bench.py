@@ -582,12 +582,16 @@ def run_ours(args, world, rank, local):
         nred = w.S // mp["stride"]
         ad_flop = share * w.B * w.Hq * 2.0 * mp["stride"] * w.D * nred * (nred + 1) / 2
         ad_tf = ad_flop / (sel_ms * 1e-3) / 1e12
-        line["kernels"]["select"].update({
-            "what": "antidiag estimator + selection from p", "bound": "tensor",
-            "estimator_tflop": ad_flop / 1e12, "tflops": ad_tf, "frac": ad_tf / peak_tf,
-            "estimator_traffic": antidiag_traffic(w.name, mp["stride"]),
-            "estimator_algorithmic_bytes": 2 * w.B * (w.Hq + w.Hkv) * w.S * w.D +
-                                           4 * w.B * w.Hq * w.nb * (w.nb + 1) // 2})
+        ad_bytes = share * (2 * w.B * (w.Hq + w.Hkv) * w.S * w.D +
+                            4 * w.B * w.Hq * w.nb * (w.nb + 1) // 2)  # Q, K read; p written
+        ad_gbs = ad_bytes / (sel_ms * 1e-3) / 1e9
+        line["kernels"]["select"] = {
+            "ms": sel_ms, "what": "antidiag estimator + selection from p", "bound": "tensor",
+            "flop": ad_flop, "tflops": ad_tf, "peak": peak_tf,
+            "peak_unit": "TFLOP/s bf16 dense", "frac": ad_tf / peak_tf,
+            "bytes": ad_bytes, "GB/s": ad_gbs, "hbm_frac": ad_gbs / pk["hbm_gbs"],
+            "traffic": antidiag_traffic(w.name, mp["stride"]),
+            "peak_derivation": "the attention roofline's peak"}
 
     if e2e is not None:
         line["e2e"] = e2e
