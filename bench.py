@@ -50,8 +50,8 @@ SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # DRAM bytes (read + write) of one attention launch at the 128K workload, from the ncu capture in
 # profiles/attn_sm100_dram_llama3-8b-128k.md; reported only while the kernel sources still hash
 # to the revision that capture measured.
-ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1615689472 + 1021989632,
-                "sources_sha256": "12e6ae00e390bc7f6452bb88950792b384c32793118c2c968bb304839760462c"}
+ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616291840 + 1018593792,
+                "sources_sha256": "c3109ce70917af63022b2abe8b312a05f35b3bc096546960d6d91ef4cf73f62f"}
 # The same for the anti-diagonal estimator (stride 16) at that workload: its two kernels (the
 # partials, then their merge into p), from the capture in profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,

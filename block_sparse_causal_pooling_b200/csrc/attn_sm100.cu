@@ -31,7 +31,8 @@
 //               when a row's max exceeds it by more than 8 (log2 units): then O's row is
 //               rescaled in TMEM; otherwise P stays below 2^8 and the reference is kept (exact
 //               either way: the final 1/l uses the same reference as P). At an item's end:
-//               O * (1/l) -> bf16 -> global (streaming stores).
+//               O * (1/l) -> bf16, staged in the head's P tile (free until the next item's
+//               first P) and copied out by each warp with coalesced streaming stores.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).
 //
 // Synchronisation is by mbarriers only. Every mbarrier wait is bounded by the global
@@ -550,34 +551,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       lsum += (sum[0].x + sum[0].y) + (sum[1].x + sum[1].y);
       return true;
     };
-    // At the item's end: when its last P V is complete, O * (1/l) -> bf16 -> global
-    // (streaming stores), then O_T is released.
+    // At the item's end: when its last P V is complete, O * (1/l) -> bf16 into P_T's buffer
+    // (free until the next item's first P), each thread its own row in the 128B-swizzled
+    // layout P uses; O_T is released. Each warp then copies out the 32 rows its own lanes
+    // wrote (so a warp barrier orders it), two rows (512 contiguous bytes of the output) per
+    // instruction for D 128, with streaming stores: a thread storing its own row would touch
+    // 32 rows per warp instruction.
     auto epilogue = [&](const Item& it) -> bool {
       if (!pv_wait()) return false;
       const float inv = 1.0f / lsum;
       tc_fence_after();
-      const int h = tl == 0 ? it.hA : it.hB;
-      __nv_bfloat16* dst = out + ((static_cast<int64_t>(it.b) * Hq + h) * S +
-                                  static_cast<int64_t>(it.i) * kM + row) * D;
-      const bool valid = static_cast<int64_t>(it.i) * kM + row < S;  // partial last block
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         TC_LD32(o_addr + 32 * c, o);
         tc_wait_ld_r32(o);
-        uint4 pk[4];
-        uint32_t* wv = reinterpret_cast<uint32_t*>(pk);
+        uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-        if (valid) {
+          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) __stcs(d4 + e, pk[e]);  // evict-first: keep K/V in L2
+        for (int q = 0; q < 4; ++q) {
+          const int k = 4 * c + q;  // 16-byte chunk of the row
+          st_shared_v4(p_row + (k >> 3) * (kM * 128) + (((k & 7) ^ swz) << 4), w[4 * q],
+                       w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
       }
       tc_fence_before();
       mbar_arrive(&bars->o_empty[tl]);
+      __syncwarp();
+      const int h = tl == 0 ? it.hA : it.hB;
+      constexpr int kChunks = D / 8;      // 16-byte chunks of a row
+      constexpr int kRows = 32 / kChunks;  // rows per instruction
+      const int cj = lane % kChunks, rr = lane / kChunks;
+      const int64_t row0 = static_cast<int64_t>(it.i) * kM + sub * 32;  // the warp's first row
+      uint4* dst = reinterpret_cast<uint4*>(
+                       out + ((static_cast<int64_t>(it.b) * Hq + h) * S + row0) * D) + cj;
+      const uint32_t src = su32(p_tiles + tl * C::kPTile) + (cj >> 3) * (kM * 128);
+#pragma unroll 4
+      for (int t = 0; t < 32 / kRows; ++t) {
+        const int r = sub * 32 + t * kRows + rr;  // row within the tile
+        const uint4 v = ld_shared_v4(src + r * 128 + (((cj & 7) ^ (r & 7)) << 4));
+        if (row0 + t * kRows + rr < S)  // rows past S in a partial last block are not written
+          __stcs(dst + (t * kRows + rr) * kChunks, v);  // evict-first: keep K/V in L2
+      }
       return true;
     };
     for (int64_t n = 0; ok; ++n) {
