@@ -52,11 +52,12 @@ SCORE_CAP = 128 << 20  # most bytes of score triangles the workspace holds
 # to the revision that capture measured.
 ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616291840 + 1018593792,
                 "sources_sha256": "c3109ce70917af63022b2abe8b312a05f35b3bc096546960d6d91ef4cf73f62f"}
-# The same for the anti-diagonal estimator (stride 16) at that workload: its two kernels (the
-# partials, then their merge into p), from the capture in profiles/antidiag_sm100_llama3-8b-128k.md.
+# The same for the anti-diagonal estimator (stride 16) at that workload: its three kernels (the
+# partials, each query group's row statistics, then the merge into p), from the capture in
+# profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,
-              "bytes": 1427185920 + 673577728 + 681591808 + 59151104,
-              "sources_sha256": "aa36c32394ef44a84b0a36806edf3c23b6ef1f6a62623bd02499d8a7747b4312"}
+              "bytes": 1411807744 + 673798656 + 9449216 + 688407808 + 45303040,
+              "sources_sha256": "0866c1eab871738625075b283d59245848553e8754ea0902001adb30f6c6c606"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -330,7 +331,7 @@ def launches_per_call(w, views, mp=None) -> int:
     for vs in views:
         B, Hq, Hkv = vs[0].shape[0], vs[0].shape[1], vs[1].shape[1]
         if mp is not None and mp.get("score") == "antidiag":
-            n += KERNELS_PER_CALL + 2  # estimator + selection from p
+            n += KERNELS_PER_CALL + 4  # estimator, row statistics, merge, selection from p
         elif mp is not None and mp.get("share") == "group" and Hq != Hkv:
             n += KERNELS_PER_CALL + 1  # one fused group-selection kernel
         else:

@@ -35,10 +35,10 @@
 //             TMEM read per chunk; per key block the sum of exp2(a - m) over its key groups
 //             goes to the partials in global memory, and each chunk's m (its snapshot) beside
 //             it; at the part's end its m and l.
-// antidiag_merge_kernel, one CTA per (b, h, query block i): combines the parts' m and l of each
-// of the block's query groups into the row's final max M and sum L, rescales every block sum to
-// M and divides by L, sums the block's query groups with shuffles and writes p_ij; a
-// bandwidth-bound pass over the partials.
+// antidiag_rowstat_kernel, one thread per (b, h, query group u): combines the parts' m and l of
+// the group into the row's final max M and sum L. antidiag_merge_kernel, one thread per p_ij:
+// rescales the R block sums of block i's query groups to their M, divides by L, adds them and
+// writes p_ij; a bandwidth-bound pass over the partials.
 // Q' tiles load with evict_last (a part re-reads its Q' tile for each of its key tiles); the
 // partials move with streaming stores.
 // Every mbarrier wait is bounded by the global nanosecond timer; on expiry the CTA records
@@ -439,77 +439,72 @@ __global__ void __launch_bounds__(kAThreads, 1)
   }
 }
 
-// p_ij of query block i of head bh from the estimator's partials: per query group u of the
-// block, the parts' maxima and sums combine into M_u = max m and L_u = sum l * 2^(m - M_u);
-// p_ij = (1/n_i) sum_u e_uj * 2^(snap_u,c(j) - M_u) / L_u, with c(j) the 32-group chunk that
-// holds block j. One CTA per (bh, i), 256 threads; a warp takes 32/R blocks j at a time, one
-// lane per (j, u), and sums the block's query groups with shuffles.
-__global__ void __launch_bounds__(256)
-    antidiag_merge_kernel(AdParams P) {
-  const int i = blockIdx.x % P.nb;
-  const int bh = blockIdx.x / P.nb;
-  const int R = P.R;
-  const int u0 = i * R;
-  const int n_i = min(R, P.nred - u0);
-  const int qt = u0 / kAM;  // a block's groups lie in one 128-group tile (R | 128)
+// Per query group u of head bh: the parts' maxima and sums combine into the row's
+// M_u = max m and L_u = sum l * 2^(m - M_u), written over part 0's entries as M_u and 1/L_u.
+// One thread per (bh, u); consecutive threads take consecutive u (coalesced).
+__global__ void __launch_bounds__(256) antidiag_rowstat_kernel(AdParams P, int64_t rows) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (t >= rows) return;
+  const int64_t bh = t / P.nred;
+  const int u = static_cast<int>(t - bh * P.nred);
+  const int qt = u / kAM;
   const int np = ad_nparts(qt, P.nred);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per = 32 / R;  // blocks j per warp step
-  const int uu = lane % R, jj = lane / R;
-  const bool urow = uu < n_i;
-  const int u = u0 + (urow ? uu : 0);
-  const float* eh = P.e + static_cast<int64_t>(bh) * P.tri_e + static_cast<int64_t>(R) * i * (i + 1) / 2;
-  const float* sh = P.snap + static_cast<int64_t>(bh) * P.tri_s;
-  float* prow = P.p + static_cast<int64_t>(bh) * P.nb * (P.nb + 1) / 2 +
-                static_cast<int64_t>(i) * (i + 1) / 2;
-  const float inv_n = 1.f / static_cast<float>(n_i);
-  // every lane loads its row's part maxima and sums together with its first partials (the
-  // partials are read-only here: written by the estimator kernel before this one)
-  const int64_t mb = (static_cast<int64_t>(bh) * P.nqt + qt) * P.maxparts * kAM + (u - qt * kAM);
-  float pmv[8], plv[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    pmv[q] = q < np ? __ldg(P.pm + mb + q * kAM) : -INFINITY;
-    plv[q] = q < np ? __ldg(P.pl + mb + q * kAM) : 0.f;
-  }
-  for (int q = 8; q < np; ++q) {  // more than eight parts: S/stride above 8192 * 8 groups
-    const float mq = __ldg(P.pm + mb + q * kAM), lq = __ldg(P.pl + mb + q * kAM);
-    const float mn = fmaxf(pmv[7], mq);
-    plv[7] = plv[7] * ex2(pmv[7] - mn) + lq * ex2(mq - mn);
-    pmv[7] = mn;
-  }
-  constexpr int kUn = 4;
-  float ev[kUn], sv[kUn];
-  auto load = [&](int jb) {
-#pragma unroll
-    for (int q = 0; q < kUn; ++q) {
-      const int j = jb + q * 8 * per + jj;
-      const bool in = j <= i && urow;
-      ev[q] = in ? __ldg(eh + j * R + uu) : 0.f;  // the block's partials: one range
-      sv[q] = in ? __ldg(sh + ad_tri((j * R) >> 5, u, P.nred, 32)) : 0.f;
-    }
-  };
-  int jb = warp * per;
-  if (jb <= i) load(jb);
-  float M = pmv[0];
-#pragma unroll
-  for (int q = 1; q < 8; ++q) M = fmaxf(M, pmv[q]);
+  const int64_t mb = (bh * P.nqt + qt) * P.maxparts * kAM + (u - qt * kAM);
+  float M = -INFINITY;
+  for (int q = 0; q < np; ++q) M = fmaxf(M, P.pm[mb + q * kAM]);
   float L = 0.f;
+  for (int q = 0; q < np; ++q) L += P.pl[mb + q * kAM] * ex2(P.pm[mb + q * kAM] - M);
+  P.pm[mb] = M;
+  P.pl[mb] = 1.0f / L;
+}
+
+// p_ij from the partials: p_ij = (1/n_i) sum_u e_uj * 2^(snap_u,c(j) - M_u) / L_u over the n_i
+// query groups u of block i, with c(j) the 32-group chunk that holds block j. One thread per
+// entry of a head's p triangle (entry g = i(i+1)/2 + j), so consecutive threads read
+// consecutive runs of R partials (e holds entry g's R partials at R*g) and write consecutive p;
+// the row's M_u and 1/L_u and the chunk's snapshots are R consecutive floats each, shared by
+// the threads of a row or a chunk (served by L1). The grid strides over the heads' chunks of
+// 256 entries.
+template <int kR>
+__global__ void __launch_bounds__(256) antidiag_merge_kernel(AdParams P, int64_t tri,
+                                                             int64_t ctas_per_head,
+                                                             int64_t chunks) {
+  for (int64_t blk = blockIdx.x; blk < chunks; blk += gridDim.x) {
+  const int64_t bh = blk / ctas_per_head;
+  const int64_t g = (blk - bh * ctas_per_head) * 256 + threadIdx.x;
+  if (g >= tri) continue;
+  // i, j of entry g: the float root is within one of i, then corrected
+  int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(g) + 1.0f) - 1.0f) * 0.5f);
+  while (static_cast<int64_t>(i) * (i + 1) / 2 > g) --i;
+  while (static_cast<int64_t>(i + 1) * (i + 2) / 2 <= g) ++i;
+  const int j = static_cast<int>(g - static_cast<int64_t>(i) * (i + 1) / 2);
+  const int u0 = i * kR;
+  const int n_i = min(kR, P.nred - u0);
+  const int qt = u0 / kAM;  // a block's groups lie in one 128-group tile (R | 128)
+  const int c = (j * kR) >> 5;
+  const float* ep = P.e + bh * P.tri_e + kR * g;
+  const float* sp = P.snap + bh * P.tri_s + ad_tri(c, u0, P.nred, 32);
+  const int64_t mb = (bh * P.nqt + qt) * P.maxparts * kAM + (u0 - qt * kAM);
+  const float* mp = P.pm + mb;
+  const float* lp = P.pl + mb;
+  float acc = 0.f;
+  if (kR >= 4 && n_i == kR && (reinterpret_cast<uintptr_t>(sp) & 15) == 0) {
+    // whole block, every run 16-byte aligned (e, M and 1/L always are; the snapshot run is
+    // unless S/stride is not a multiple of 4)
 #pragma unroll
-  for (int q = 0; q < 8; ++q) L += plv[q] * ex2(pmv[q] - M);
-  const float inv_l = 1.f / L;
-  for (; jb <= i; jb += 8 * per * kUn) {
-    float val[kUn];
-#pragma unroll
-    for (int q = 0; q < kUn; ++q) val[q] = ev[q] * ex2(sv[q] - M) * inv_l;
-    if (jb + 8 * per * kUn <= i) load(jb + 8 * per * kUn);  // the next step's loads in flight
-#pragma unroll
-    for (int q = 0; q < kUn; ++q) {
-      const int j = jb + q * 8 * per + jj;
-      float v = val[q];
-      for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (j <= i && uu == 0) __stcs(prow + j, v * inv_n);
+    for (int q = 0; q < (kR >= 4 ? kR / 4 : 1); ++q) {
+      const float4 e4 = __ldcs(reinterpret_cast<const float4*>(ep) + q);
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sp) + q);
+      const float4 m4 = __ldg(reinterpret_cast<const float4*>(mp) + q);
+      const float4 l4 = __ldg(reinterpret_cast<const float4*>(lp) + q);
+      acc += (e4.x * ex2(s4.x - m4.x) * l4.x + e4.y * ex2(s4.y - m4.y) * l4.y) +
+             (e4.z * ex2(s4.z - m4.z) * l4.z + e4.w * ex2(s4.w - m4.w) * l4.w);
     }
+  } else {
+    for (int uu = 0; uu < n_i; ++uu)
+      acc += __ldcs(ep + uu) * ex2(__ldg(sp + uu) - __ldg(mp + uu)) * __ldg(lp + uu);
+  }
+  P.p[bh * tri + g] = acc * (1.0f / static_cast<float>(n_i));
   }
 }
 
@@ -630,8 +625,21 @@ cudaError_t launch_antidiag(const void* q, const void* k, int B, int Hq, int Hkv
   if (e != cudaSuccess) return e;
   antidiag_sm100_kernel<<<static_cast<unsigned>(grid), kAThreads, smem, st>>>(tq, tk, P);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  antidiag_merge_kernel<<<static_cast<unsigned>(static_cast<int64_t>(B) * Hq * P.nb), 256, 0,
-                          st>>>(P);
+  const int64_t rows = static_cast<int64_t>(B) * Hq * P.nred;
+  antidiag_rowstat_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, st>>>(P, rows);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t tri = static_cast<int64_t>(P.nb) * (P.nb + 1) / 2;
+  const int64_t per_head = (tri + 255) / 256;
+  const int64_t chunks = static_cast<int64_t>(B) * Hq * per_head;
+  const unsigned gm = static_cast<unsigned>(std::min<int64_t>(chunks, int64_t{1} << 20));
+  switch (P.R) {
+    case 1: antidiag_merge_kernel<1><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+    case 2: antidiag_merge_kernel<2><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+    case 4: antidiag_merge_kernel<4><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+    case 8: antidiag_merge_kernel<8><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+    case 16: antidiag_merge_kernel<16><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+    default: antidiag_merge_kernel<32><<<gm, 256, 0, st>>>(P, tri, per_head, chunks); break;
+  }
   return cudaGetLastError();
 }
 

@@ -37,9 +37,9 @@ WORKLOADS = {
     "short": wl.LLAMA_32K.replace(name="short", Hq=2, Hkv=1, S=200, tau=2.0),
 }
 
-P_CASES = [("llama-4k", 16), ("llama-4k", 4), ("llama-4k", 32), ("llama-4k", 128),
-           ("llama-ragged", 16), ("qwen-3k", 16), ("d64-blk64", 8), ("d64-blk64", 2),
-           ("short", 8)]
+P_CASES = [("llama-4k", 16), ("llama-4k", 4), ("llama-4k", 32), ("llama-4k", 64),
+           ("llama-4k", 128), ("llama-ragged", 16), ("qwen-3k", 16), ("d64-blk64", 8),
+           ("d64-blk64", 2), ("short", 8)]
 
 
 def inputs(w):
