@@ -57,7 +57,7 @@ ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616291840 + 1018593792,
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,
               "bytes": 1411807744 + 673798656 + 9449216 + 688407808 + 45303040,
-              "sources_sha256": "0866c1eab871738625075b283d59245848553e8754ea0902001adb30f6c6c606"}
+              "sources_sha256": "5e8522bc29f044f5066d27e58018126b13b63751cab6e0a86a724459a4892a97"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

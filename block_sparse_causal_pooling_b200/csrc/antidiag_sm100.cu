@@ -470,41 +470,41 @@ __global__ void __launch_bounds__(256) antidiag_merge_kernel(AdParams P, int64_t
                                                              int64_t ctas_per_head,
                                                              int64_t chunks) {
   for (int64_t blk = blockIdx.x; blk < chunks; blk += gridDim.x) {
-  const int64_t bh = blk / ctas_per_head;
-  const int64_t g = (blk - bh * ctas_per_head) * 256 + threadIdx.x;
-  if (g >= tri) continue;
-  // i, j of entry g: the float root is within one of i, then corrected
-  int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(g) + 1.0f) - 1.0f) * 0.5f);
-  while (static_cast<int64_t>(i) * (i + 1) / 2 > g) --i;
-  while (static_cast<int64_t>(i + 1) * (i + 2) / 2 <= g) ++i;
-  const int j = static_cast<int>(g - static_cast<int64_t>(i) * (i + 1) / 2);
-  const int u0 = i * kR;
-  const int n_i = min(kR, P.nred - u0);
-  const int qt = u0 / kAM;  // a block's groups lie in one 128-group tile (R | 128)
-  const int c = (j * kR) >> 5;
-  const float* ep = P.e + bh * P.tri_e + kR * g;
-  const float* sp = P.snap + bh * P.tri_s + ad_tri(c, u0, P.nred, 32);
-  const int64_t mb = (bh * P.nqt + qt) * P.maxparts * kAM + (u0 - qt * kAM);
-  const float* mp = P.pm + mb;
-  const float* lp = P.pl + mb;
-  float acc = 0.f;
-  if (kR >= 4 && n_i == kR && (reinterpret_cast<uintptr_t>(sp) & 15) == 0) {
-    // whole block, every run 16-byte aligned (e, M and 1/L always are; the snapshot run is
-    // unless S/stride is not a multiple of 4)
+    const int64_t bh = blk / ctas_per_head;
+    const int64_t g = (blk - bh * ctas_per_head) * 256 + threadIdx.x;
+    if (g >= tri) continue;
+    // i, j of entry g: the float root may be off by one either way; the integer tests fix it
+    int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(g) + 1.0f) - 1.0f) * 0.5f);
+    while (static_cast<int64_t>(i) * (i + 1) / 2 > g) --i;
+    while (static_cast<int64_t>(i + 1) * (i + 2) / 2 <= g) ++i;
+    const int j = static_cast<int>(g - static_cast<int64_t>(i) * (i + 1) / 2);
+    const int u0 = i * kR;
+    const int n_i = min(kR, P.nred - u0);
+    const int qt = u0 / kAM;  // a block's groups lie in one 128-group tile (R | 128)
+    const int c = (j * kR) >> 5;
+    const float* ep = P.e + bh * P.tri_e + kR * g;
+    const float* sp = P.snap + bh * P.tri_s + ad_tri(c, u0, P.nred, 32);
+    const int64_t mb = (bh * P.nqt + qt) * P.maxparts * kAM + (u0 - qt * kAM);
+    const float* mp = P.pm + mb;
+    const float* lp = P.pl + mb;
+    float acc = 0.f;
+    if (kR >= 4 && n_i == kR && (reinterpret_cast<uintptr_t>(sp) & 15) == 0) {
+      // whole block, every run 16-byte aligned (e, M and 1/L always are; the snapshot run is
+      // unless S/stride is not a multiple of 4)
 #pragma unroll
-    for (int q = 0; q < (kR >= 4 ? kR / 4 : 1); ++q) {
-      const float4 e4 = __ldcs(reinterpret_cast<const float4*>(ep) + q);
-      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sp) + q);
-      const float4 m4 = __ldg(reinterpret_cast<const float4*>(mp) + q);
-      const float4 l4 = __ldg(reinterpret_cast<const float4*>(lp) + q);
-      acc += (e4.x * ex2(s4.x - m4.x) * l4.x + e4.y * ex2(s4.y - m4.y) * l4.y) +
-             (e4.z * ex2(s4.z - m4.z) * l4.z + e4.w * ex2(s4.w - m4.w) * l4.w);
+      for (int q = 0; q < (kR >= 4 ? kR / 4 : 1); ++q) {
+        const float4 e4 = __ldcs(reinterpret_cast<const float4*>(ep) + q);
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(sp) + q);
+        const float4 m4 = __ldg(reinterpret_cast<const float4*>(mp) + q);
+        const float4 l4 = __ldg(reinterpret_cast<const float4*>(lp) + q);
+        acc += (e4.x * ex2(s4.x - m4.x) * l4.x + e4.y * ex2(s4.y - m4.y) * l4.y) +
+               (e4.z * ex2(s4.z - m4.z) * l4.z + e4.w * ex2(s4.w - m4.w) * l4.w);
+      }
+    } else {
+      for (int uu = 0; uu < n_i; ++uu)
+        acc += __ldcs(ep + uu) * ex2(__ldg(sp + uu) - __ldg(mp + uu)) * __ldg(lp + uu);
     }
-  } else {
-    for (int uu = 0; uu < n_i; ++uu)
-      acc += __ldcs(ep + uu) * ex2(__ldg(sp + uu) - __ldg(mp + uu)) * __ldg(lp + uu);
-  }
-  P.p[bh * tri + g] = acc * (1.0f / static_cast<float>(n_i));
+    P.p[bh * tri + g] = acc * (1.0f / static_cast<float>(n_i));
   }
 }
 
