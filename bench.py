@@ -538,6 +538,9 @@ def run_ours(args, world, rank, local):
     achieved = wl.effective_flops(rank_pairs, w.block, w.D) / (attn_ms * 1e-3) / 1e12
     elt = 2 if w.dtype == "bf16" else 4
     share = rank_pairs / pairs  # this rank's fraction of the (b, head) units
+    # the captured traffic is that of one launch over the whole problem: a rank that runs a
+    # share of it, or several calls per step, has no captured figure
+    whole = share == 1.0 and len(views) == 1
     pool_bytes = share * (w.B * (w.Hq + 2 * w.Hkv) * w.S * w.D * elt +
                           4 * (w.B * (w.Hq + w.Hkv) * w.nb * w.D + w.B * w.Hkv * w.nb))
     line = {
@@ -558,7 +561,7 @@ def run_ours(args, world, rank, local):
                        causal_fraction=int(kk.sum()) / (w.nb * (w.nb + 1) / 2)),
         "roofline": {"kernel": "sparse_attn", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                     "traffic": attn_traffic(w.name) if mp is None else None,
+                     "traffic": attn_traffic(w.name) if mp is None and whole else None,
                      "peak_source": f"{pk_kind} {'sustained' if long_region else 'burst'} "
                                     "bf16 dense"},
         "kernels": {
@@ -591,7 +594,7 @@ def run_ours(args, world, rank, local):
             "flop": ad_flop, "tflops": ad_tf, "peak": peak_tf,
             "peak_unit": "TFLOP/s bf16 dense", "frac": ad_tf / peak_tf,
             "bytes": ad_bytes, "GB/s": ad_gbs, "hbm_frac": ad_gbs / pk["hbm_gbs"],
-            "traffic": antidiag_traffic(w.name, mp["stride"]),
+            "traffic": antidiag_traffic(w.name, mp["stride"]) if whole else None,
             "peak_derivation": "the attention roofline's peak"}
 
     if e2e is not None:
