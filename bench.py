@@ -57,7 +57,7 @@ ATTN_TRAFFIC = {"workload": "llama3-8b-128k", "bytes": 1616291840 + 1018593792,
 # profiles/antidiag_sm100_llama3-8b-128k.md.
 AD_TRAFFIC = {"workload": "llama3-8b-128k", "stride": 16,
               "bytes": 1411807744 + 673798656 + 9449216 + 688407808 + 45303040,
-              "sources_sha256": "5e8522bc29f044f5066d27e58018126b13b63751cab6e0a86a724459a4892a97"}
+              "sources_sha256": "2006ed9beacf780952bfedd0ae35d62ed920b342b2ea5cae5737a2825706b83f"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

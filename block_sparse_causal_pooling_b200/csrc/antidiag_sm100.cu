@@ -105,8 +105,9 @@ struct AdParams {
   // chunk-major: entry (c, u) at c*nred - 32*c*(c-1)/2 + (u - 32*c).
   float* e;             // [B*Hq][tri_e]
   float* snap;          // [B*Hq][tri_s]
-  float* pm;            // [B*Hq][nqt][maxparts][128] each part's max m
-  float* pl;            // the same for its sum l
+  float* pm;            // [B*Hq][nqt][maxparts][128] each part's max m; after the row
+                        // statistics, part 0's entry holds the query group's final max M
+  float* pl;            // the same for its sum l; part 0's entry then holds 1/L
   int64_t tri_e, tri_s;
   int32_t* status;
   int withhold;         // test switch: the first stage's copies are never sent
